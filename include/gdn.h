@@ -1,0 +1,180 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated-delta-rule forward library
+ *          (libgdn_b200.so).
+ *
+ * What is computed. Per sequence n and head h, the gated delta rule
+ *
+ *     alpha_t = exp(g_t)
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,    o_t = S_t q_t
+ *
+ * with S a d_v x d_k fp32 matrix (row = value index). This is the recurrent
+ * layer of the hybrid gated delta network backbone in "A Modern Multimodal
+ * Assistant on a 6 GB 2011 GPU" (page 1, abstract, result (i)), which runs
+ * it in two forms: chunk by chunk (prefill) and one token at a time (the
+ * sequential scan; decode). The update rule is that of the Gated Delta
+ * Networks paper listed among page 3's references. The pages print no
+ * interface; this one is the library's own.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous,
+ *     owned by the caller. The library allocates no memory, never synchronises
+ *     the stream (except gdn_chunk_fwd_check, which exists to do so), and
+ *     launches everything on `stream` (a cudaStream_t passed as void*; NULL =
+ *     the legacy default stream).
+ *   - Layouts are token-major and row-major:
+ *       q, k : [T][H][dk]   v, o : [T][H][dv]   (dtype gdn_dtype: fp32 or bf16)
+ *       g, beta : [T][H] fp32   (g = natural-log decay, finite, g <= 0 expected;
+ *                                beta in [0,1] expected)
+ *       S, S0, S_T : [N][H][dv][dk] fp32
+ *     q and k are expected L2-normalised by the caller; no normalisation,
+ *     gating or scaling happens inside (o_t = S_t q_t, no query scale).
+ *   - Supported head sizes: dk = dv in {64, 128}.
+ *   - o is written in the input dtype (bf16: rounded to nearest even from the
+ *     fp32 accumulator). States are fp32.
+ *   - NaN/Inf inputs are undefined behaviour; they are not checked on the hot
+ *     path. Decays below ~1e-38 may be flushed to zero.
+ *   - Errors are returned as gdn_status, never thrown or trapped;
+ *     gdn_last_error() gives a message for the calling thread's last non-OK
+ *     status. Launch failures map to GDN_ERR_CUDA with the CUDA error text.
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL = 1,      /* a required pointer is NULL */
+    GDN_ERR_SHAPE = 2,     /* unsupported or inconsistent sizes */
+    GDN_ERR_DTYPE = 3,     /* unknown dtype code */
+    GDN_ERR_ALIGN = 4,     /* a pointer is not 16-byte aligned */
+    GDN_ERR_SEQLENS = 5,   /* cu_seqlens not 0 = c0 <= c1 <= ... <= cN = T_tot */
+    GDN_ERR_WORKSPACE = 6, /* workspace missing or smaller than required */
+    GDN_ERR_CUDA = 7,      /* a CUDA launch or runtime call failed */
+    GDN_ERR_TIMEOUT = 8    /* a bounded device-side wait gave up */
+} gdn_status;
+
+typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int gdn_version(void);
+
+/* Message for the calling thread's last non-OK status ("" if none). The
+ * string is owned by the library and valid until the thread's next call. */
+const char *gdn_last_error(void);
+
+/*
+ * Workspace bytes gdn_chunk_fwd needs for these sizes (0 is never returned:
+ * the workspace always holds at least the device error word). The workspace
+ * is scratch owned by the caller: its contents on entry are ignored and on
+ * exit are meaningless except for the error word read by gdn_chunk_fwd_check.
+ * Two calls that overlap on the GPU must not share a workspace.
+ */
+size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype);
+
+/*
+ * Prefill: the chunked form of the rule over N packed sequences (page 1,
+ * abstract, result (i): the recurrent layers rewritten chunk-wise; page 2,
+ * "Resumen Tecnico", Metodologia, recurrent-layer item: an intra-chunk part,
+ * an inter-chunk part and a forward-substitution step).
+ *
+ *   q, k      [T_tot][H][dk]  dtype      v [T_tot][H][dv] dtype
+ *   g, beta   [T_tot][H]      fp32
+ *   S0        [N][H][dv][dk]  fp32, or NULL for a zero initial state.
+ *             May alias S_T (in-place state update).
+ *   cu_seqlens [N+1] int32 on the device: sequence n is tokens
+ *             [cu_seqlens[n], cu_seqlens[n+1]). NULL means N equal sequences
+ *             of T_tot/N tokens (T_tot % N must be 0). Chunks restart at every
+ *             sequence start; the last chunk of a sequence may be partial;
+ *             an empty sequence gives S_T = S0 (or 0).
+ *   o         [T_tot][H][dv] dtype  (output; must not alias any input)
+ *   S_T       [N][H][dv][dk] fp32   (output: state after each sequence)
+ *   workspace, ws_bytes: >= gdn_chunk_fwd_workspace_size(...) bytes of device
+ *             memory, 256-byte aligned.
+ *
+ * A device-side cu_seqlens is validated on the device (the host cannot read
+ * it without a synchronisation): if it is malformed, the kernels write
+ * nothing to o / S_T and record GDN_ERR_SEQLENS in the workspace's error
+ * word; gdn_chunk_fwd itself returns GDN_OK and gdn_chunk_fwd_check reports
+ * the error. fp32 inputs run an fp32 (CUDA-core) chunked path; bf16 inputs
+ * the tensor-core path (bf16 operands, fp32 accumulation and state).
+ */
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *g, const float *beta, const float *S0,
+                         const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                         int dtype, void *o, float *S_T,
+                         void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream` and reads the device error word that the last
+ * gdn_chunk_fwd on this workspace wrote: GDN_OK, GDN_ERR_SEQLENS or
+ * GDN_ERR_TIMEOUT (a bounded inter-block wait gave up; outputs are then
+ * incomplete). The word is reset by every gdn_chunk_fwd call.
+ */
+gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Decode: one single-token step of the rule for B independent sequences
+ * (the token-at-a-time form of page 2, "Resumen Tecnico", Metodologia,
+ * recurrent-layer item). For every (b, h) and every row i of S:
+ *     a = S_i . k,  b_i = S_i . q,  S_i <- alpha S_i + beta (v_i - alpha a) k,
+ *     o_i = alpha b_i + beta (v_i - alpha a) (k . q)       (= (S_new q)_i)
+ *   q, k [B][H][dk] dtype; v [B][H][dv] dtype; g, beta [B][H] fp32;
+ *   S [B][H][dv][dk] fp32, updated in place; o [B][H][dv] dtype (output).
+ * S is read once and written once per call.
+ */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *g, const float *beta, float *S,
+                           int B, int H, int dk, int dv, int dtype, void *o, void *stream);
+
+/*
+ * The sequential (token-by-token) scan on the GPU: the same result as
+ * gdn_chunk_fwd, computed one token at a time with the decode step's row
+ * update. It is the comparator for the chunked path's speed-up (page 1,
+ * abstract, result (i) reports the chunked form 2.8 times faster than the
+ * scan on a Fermi C2075), not a production path. Arguments as gdn_chunk_fwd, without a workspace. A
+ * malformed device cu_seqlens is clamped into [0, T_tot] per sequence (no
+ * access leaves the buffers) and gives meaningless results: validate it
+ * with gdn_chunk_fwd + gdn_chunk_fwd_check.
+ */
+gdn_status gdn_seq_scan(const void *q, const void *k, const void *v,
+                        const float *g, const float *beta, const float *S0,
+                        const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                        int dtype, void *o, float *S_T, void *stream);
+
+/*
+ * Diagnostic (used by the tests, not by the forward path): one tensor-core
+ * tile D = A * B^T computed with the same shared-memory descriptors, TMEM
+ * allocation and tcgen05.mma / tcgen05.ld helpers as the chunked kernel.
+ *   A [M][K] bf16 row-major, B [N][K] bf16 row-major (device);
+ *   D [128][N] fp32 (device): every TMEM lane is dumped, so for M = 64 the
+ *     rows the hardware leaves unused are visible as well.
+ *   a_mn / b_mn: 1 = stage that operand as an MN-major tile, 0 = K-major.
+ *   variant: 0 or 1, the two core-matrix stride conventions of the kernels.
+ * Limits: M in {64, 128}; 16 <= N <= 256 (multiple of 16 for M = 128, of 8
+ * for M = 64); 16 <= K <= 128, multiple of 16. Launches one CTA on `stream`.
+ */
+gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, int M, int N, int K,
+                             int a_mn, int b_mn, int variant, void *stream);
+
+/*
+ * Kernel timing (measurement support, off by default). While enabled, every
+ * entry point records a CUDA event pair on its stream around each kernel it
+ * launches. gdn_profile_read waits for those events, writes per kernel name
+ * the summed milliseconds (ms[i]) and launch count (counts[i]), the names
+ * newline-separated into `names` (truncated to names_len), clears the record
+ * and returns the number of kernel names (at most max_kernels). ms / counts /
+ * names may be NULL. Not for use while a CUDA graph is being captured.
+ */
+void gdn_profile_enable(int on);
+int gdn_profile_read(char *names, size_t names_len, float *ms, int *counts, int max_kernels);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GDN_B200_H */

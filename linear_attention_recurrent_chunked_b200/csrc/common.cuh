@@ -1,0 +1,49 @@
+// Device helpers shared by the library's kernels (not by the oracle).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/gdn.h"
+
+namespace gdn {
+
+// Device error word layout (first 4 bytes of the chunk workspace).
+enum : uint32_t { ERRBIT_SEQLENS = 1u, ERRBIT_TIMEOUT = 2u };
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float *p) { return *p; }
+    static __device__ __forceinline__ void store(float *p, float x) { *p = x; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+};
+
+// Four consecutive elements as fp32 (8-byte load for bf16, 16-byte load for fp32).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+    uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+}
+
+// Sequence bounds from cu_seqlens (device) or equal split, clamped to [0, T_tot].
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int n, int N, int T_tot, int &t0, int &t1) {
+    if (cu) {
+        t0 = cu[n];
+        t1 = cu[n + 1];
+    } else {
+        const int L = T_tot / N;
+        t0 = n * L;
+        t1 = t0 + L;
+    }
+    t0 = min(max(t0, 0), T_tot);
+    t1 = min(max(t1, t0), T_tot);
+}
+
+}  // namespace gdn

@@ -1,0 +1,289 @@
+// C ABI of the library (declared in include/gdn.h): argument validation,
+// error reporting and dispatch to the kernels. Host code only, apart from the
+// small cu_seqlens validation kernel.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+gdn_status fail(gdn_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+gdn_status ok() {
+    g_msg[0] = '\0';
+    return GDN_OK;
+}
+
+gdn_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(GDN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool misaligned(const void *p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+constexpr size_t kErrWordBytes = 256;  // error word, padded to keep later regions 256-byte aligned
+
+// ---- optional per-kernel timing (gdn_profile_*): CUDA events recorded on the
+// launching stream around each kernel the entry points launch.
+struct ProfRec {
+    const char *name;
+    cudaEvent_t start, stop;
+};
+struct Prof {
+    std::mutex mu;
+    bool on = false;
+    std::vector<ProfRec> recs;
+    std::vector<cudaEvent_t> pool;
+} g_prof;
+
+cudaEvent_t prof_event() {
+    if (!g_prof.pool.empty()) {
+        cudaEvent_t e = g_prof.pool.back();
+        g_prof.pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// RAII: records a start event now and a stop event (plus the record) at scope exit.
+struct ProfScope {
+    const char *name;
+    cudaStream_t st;
+    cudaEvent_t start = nullptr;
+    ProfScope(const char *n, cudaStream_t s) : name(n), st(s) {
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        if (g_prof.on) {
+            start = prof_event();
+            cudaEventRecord(start, st);
+        }
+    }
+    ~ProfScope() {
+        if (!start) return;
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        cudaEvent_t stop = prof_event();
+        cudaEventRecord(stop, st);
+        g_prof.recs.push_back({name, start, stop});
+    }
+};
+
+gdn_status check_common(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                        const void *o, int T_tot, int H, int dk, int dv, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return fail(GDN_ERR_DTYPE, "dtype %d is not GDN_F32 or GDN_BF16", dtype);
+    if (H < 1 || T_tot < 0) return fail(GDN_ERR_SHAPE, "H=%d T=%d out of range", H, T_tot);
+    if (dk != dv || (dk != 64 && dk != 128))
+        return fail(GDN_ERR_SHAPE, "head sizes dk=%d dv=%d unsupported (need dk == dv in {64, 128})", dk, dv);
+    if (T_tot > 0 && (!q || !k || !v || !g || !beta || !o)) return fail(GDN_ERR_NULL, "q, k, v, g, beta and o are required");
+    const void *ptrs[] = {q, k, v, g, beta, o};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return fail(GDN_ERR_ALIGN, "tensor pointer %p is not 16-byte aligned", p);
+    if ((double)T_tot * H * dk >= 9.0e18) return fail(GDN_ERR_SHAPE, "sizes overflow");
+    return GDN_OK;
+}
+
+}  // namespace
+
+namespace gdn {
+
+__global__ void k_validate_seqlens(const int32_t *__restrict__ cu, int N, int T_tot, uint32_t *__restrict__ err) {
+    // One warp: err = ERRBIT_SEQLENS unless cu[0] == 0, cu non-decreasing, cu[N] == T_tot.
+    bool bad = false;
+    if (cu) {
+        for (int n = threadIdx.x; n < N; n += 32) bad |= cu[n + 1] < cu[n];
+        if (threadIdx.x == 0) bad |= (cu[0] != 0) || (cu[N] != T_tot);
+    }
+    bad = __any_sync(0xffffffffu, bad);
+    if (threadIdx.x == 0) *err = bad ? ERRBIT_SEQLENS : 0u;
+}
+
+cudaError_t launch_validate_seqlens(const int32_t *cu, int N, int T_tot, uint32_t *err, cudaStream_t st) {
+    k_validate_seqlens<<<1, 32, 0, st>>>(cu, N, T_tot, err);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn
+
+extern "C" {
+
+int gdn_version(void) { return 100; }
+
+const char *gdn_last_error(void) { return g_msg; }
+
+size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype) {
+    (void)N; (void)T_tot; (void)H; (void)dk; (void)dv; (void)dtype;
+    return kErrWordBytes;
+}
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                         const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                         int dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
+    gdn_status s = check_common(q, k, v, g, beta, o, T_tot, H, dk, dv, dtype);
+    if (s != GDN_OK) return s;
+    if (N < 1) return fail(GDN_ERR_SHAPE, "N=%d must be >= 1", N);
+    if (!S_T) return fail(GDN_ERR_NULL, "S_T is required");
+    if (misaligned(S0) || misaligned(S_T) || misaligned(cu_seqlens))
+        return fail(GDN_ERR_ALIGN, "S0, S_T and cu_seqlens must be 16-byte aligned");
+    if (!cu_seqlens && T_tot % N != 0)
+        return fail(GDN_ERR_SEQLENS, "cu_seqlens is NULL and T_tot=%d is not a multiple of N=%d", T_tot, N);
+    const size_t need = gdn_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dtype);
+    if (!workspace || ws_bytes < need)
+        return fail(GDN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return fail(GDN_ERR_ALIGN, "workspace must be 256-byte aligned");
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t *err = static_cast<uint32_t *>(workspace);
+    cudaError_t e;
+    {
+        ProfScope ps("validate_seqlens", st);
+        e = gdn::launch_validate_seqlens(cu_seqlens, N, T_tot, err, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens validation launch");
+
+    ProfScope ps("chunk_simt", st);
+    if (dtype == GDN_F32) {
+        const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+                    *vf = static_cast<const float *>(v);
+        float *of = static_cast<float *>(o);
+        e = (dk == 64) ? gdn::launch_chunk_simt<float, 64>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st)
+                       : gdn::launch_chunk_simt<float, 128>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st);
+    } else {
+        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k),
+                            *vb = static_cast<const __nv_bfloat16 *>(v);
+        __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+        e = (dk == 64)
+                ? gdn::launch_chunk_simt<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st)
+                : gdn::launch_chunk_simt<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "chunked forward launch");
+    return ok();
+}
+
+gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *stream) {
+    if (!workspace || ws_bytes < sizeof(uint32_t)) return fail(GDN_ERR_WORKSPACE, "workspace missing");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (word & gdn::ERRBIT_SEQLENS) return fail(GDN_ERR_SEQLENS, "cu_seqlens is not 0 = c0 <= c1 <= ... <= cN = T_tot");
+    if (word & gdn::ERRBIT_TIMEOUT) return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    return ok();
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta, float *S,
+                           int B, int H, int dk, int dv, int dtype, void *o, void *stream) {
+    if (B < 1) return fail(GDN_ERR_SHAPE, "B=%d must be >= 1", B);
+    gdn_status s = check_common(q, k, v, g, beta, o, B, H, dk, dv, dtype);
+    if (s != GDN_OK) return s;
+    if (!S) return fail(GDN_ERR_NULL, "S is required");
+    if (misaligned(S)) return fail(GDN_ERR_ALIGN, "S must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    ProfScope ps("decode_step", st);
+    if (dtype == GDN_F32) {
+        const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+                    *vf = static_cast<const float *>(v);
+        float *of = static_cast<float *>(o);
+        e = (dk == 64) ? gdn::launch_decode_step<float, 64>(qf, kf, vf, g, beta, S, B, H, of, st)
+                       : gdn::launch_decode_step<float, 128>(qf, kf, vf, g, beta, S, B, H, of, st);
+    } else {
+        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k),
+                            *vb = static_cast<const __nv_bfloat16 *>(v);
+        __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+        e = (dk == 64) ? gdn::launch_decode_step<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S, B, H, ob, st)
+                       : gdn::launch_decode_step<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S, B, H, ob, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "decode step launch");
+    return ok();
+}
+
+gdn_status gdn_seq_scan(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                        const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                        int dtype, void *o, float *S_T, void *stream) {
+    gdn_status s = check_common(q, k, v, g, beta, o, T_tot, H, dk, dv, dtype);
+    if (s != GDN_OK) return s;
+    if (N < 1) return fail(GDN_ERR_SHAPE, "N=%d must be >= 1", N);
+    if (!S_T) return fail(GDN_ERR_NULL, "S_T is required");
+    if (misaligned(S0) || misaligned(S_T) || misaligned(cu_seqlens))
+        return fail(GDN_ERR_ALIGN, "S0, S_T and cu_seqlens must be 16-byte aligned");
+    if (!cu_seqlens && T_tot % N != 0)
+        return fail(GDN_ERR_SEQLENS, "cu_seqlens is NULL and T_tot=%d is not a multiple of N=%d", T_tot, N);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    ProfScope ps("seq_scan", st);
+    if (dtype == GDN_F32) {
+        const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+                    *vf = static_cast<const float *>(v);
+        float *of = static_cast<float *>(o);
+        e = (dk == 64) ? gdn::launch_seq_scan<float, 64>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, st)
+                       : gdn::launch_seq_scan<float, 128>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, st);
+    } else {
+        const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k),
+                            *vb = static_cast<const __nv_bfloat16 *>(v);
+        __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+        e = (dk == 64) ? gdn::launch_seq_scan<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, st)
+                       : gdn::launch_seq_scan<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "sequential scan launch");
+    return ok();
+}
+
+void gdn_profile_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.on = on != 0;
+}
+
+int gdn_profile_read(char *names, size_t names_len, float *ms, int *counts, int max_kernels) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    std::vector<std::string> keys;
+    std::vector<float> tot;
+    std::vector<int> cnt;
+    for (const ProfRec &r : g_prof.recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess)
+            t = -1.f;
+        size_t i = 0;
+        while (i < keys.size() && keys[i] != r.name) ++i;
+        if (i == keys.size()) {
+            keys.push_back(r.name);
+            tot.push_back(0.f);
+            cnt.push_back(0);
+        }
+        tot[i] += t;
+        cnt[i] += 1;
+        g_prof.pool.push_back(r.start);
+        g_prof.pool.push_back(r.stop);
+    }
+    g_prof.recs.clear();
+    std::string joined;
+    int n = 0;
+    for (size_t i = 0; i < keys.size() && n < max_kernels; ++i, ++n) {
+        if (ms) ms[n] = tot[i];
+        if (counts) counts[n] = cnt[i];
+        joined += keys[i];
+        joined += '\n';
+    }
+    if (names && names_len) {
+        strncpy(names, joined.c_str(), names_len - 1);
+        names[names_len - 1] = '\0';
+    }
+    return n;
+}
+
+}  // extern "C"

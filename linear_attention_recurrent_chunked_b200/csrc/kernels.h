@@ -1,0 +1,29 @@
+// Internal launchers of the library's kernels (host side). Not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+template <typename T, int D>
+cudaError_t launch_decode_step(const T *q, const T *k, const T *v, const float *g, const float *beta, float *S,
+                               int B, int H, T *o, cudaStream_t st);
+
+template <typename T, int D>
+cudaError_t launch_seq_scan(const T *q, const T *k, const T *v, const float *g, const float *beta, const float *S0,
+                            const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, cudaStream_t st);
+
+template <typename T, int D>
+cudaError_t launch_chunk_simt(const T *q, const T *k, const T *v, const float *g, const float *beta, const float *S0,
+                              const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, const uint32_t *err,
+                              cudaStream_t st);
+
+// Writes the workspace error word: ERRBIT_SEQLENS if cu_seqlens (device, N+1
+// entries) is not 0 = c0 <= ... <= cN = T_tot, else 0. With cu == NULL it
+// just clears the word.
+cudaError_t launch_validate_seqlens(const int32_t *cu, int N, int T_tot, uint32_t *err, cudaStream_t st);
+
+}  // namespace gdn

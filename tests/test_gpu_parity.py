@@ -1,0 +1,207 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs. Tolerance: max|gpu - oracle| / max|oracle| <= 1e-4 for
+fp32 inputs and 2e-2 for bf16 inputs, for o and for the final state."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrent_chunked_b200 import gdn
+from linear_attention_recurrent_chunked_b200.workloads import make_decode, make_prefill
+from tests.gpu_util import TOL, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gdn.load_library()
+
+
+def run_oracle(w):
+    return oracle.scan(w["q"], w["k"], w["v"], w["g"], w["beta"], S0=w["S0"], cu_seqlens=w["cu_seqlens"])
+
+
+def check(o, S_T, o_ref, S_ref, dtype, what=""):
+    eo, es = rel_err(o, o_ref), rel_err(S_T, S_ref)
+    assert eo <= TOL[dtype] and es <= TOL[dtype], "%s: err(o)=%.3g err(S_T)=%.3g" % (what, eo, es)
+    return eo, es
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_chain_small(dtype, d):
+    w = make_decode(steps=6, B=3, H=2, d=d, dtype=dtype, seed=1)
+    dw = to_dev(w)
+    S = dw["S"].clone()
+    S_ref = w["S"].double().numpy()
+    for t in range(w["steps"]):
+        o = gdn.decode_step(dw["q"][t], dw["k"][t], dw["v"][t], dw["g"][t], dw["beta"][t], S)
+        o_ref, S_ref = oracle.decode_step(w["q"][t], w["k"][t], w["v"][t], w["g"][t], w["beta"][t], S_ref)
+        assert rel_err(o, o_ref) <= TOL[dtype]
+    assert rel_err(S, S_ref) <= TOL[dtype]
+
+
+def test_decode_full_size_sampled_pairs():
+    """Decode workload at full size (B=64, H=16, d=128, 256 steps). The GPU runs
+    every (b, h); the oracle replays a sample of (b, h) pairs (independent by
+    construction) as 256-token scans; all outputs must stay finite."""
+    w = make_decode(seed=0)
+    dw = to_dev(w)
+    S = dw["S"].clone()
+    outs = torch.empty_like(dw["v"])
+    for t in range(w["steps"]):
+        gdn.decode_step(dw["q"][t], dw["k"][t], dw["v"][t], dw["g"][t], dw["beta"][t], S, o=outs[t])
+    torch.cuda.synchronize()
+    assert torch.isfinite(outs.float()).all() and torch.isfinite(S).all()
+    rng = np.random.default_rng(0)
+    pairs = [(0, 0), (63, 15)] + [tuple(x) for x in zip(rng.integers(0, 64, 6), rng.integers(0, 16, 6))]
+    for b, h in pairs:
+        sl = (slice(None), b, slice(h, h + 1))
+        o_ref, S_ref = oracle.scan(w["q"][sl], w["k"][sl], w["v"][sl], w["g"][:, b, h:h + 1],
+                                   w["beta"][:, b, h:h + 1], S0=w["S"][b:b + 1, h:h + 1])
+        assert rel_err(outs[sl], o_ref) <= TOL["bf16"], (b, h)
+        assert rel_err(S[b, h], S_ref[0, 0]) <= TOL["bf16"], (b, h)
+
+
+# ------------------------------------------------------------------ sequential scan (GPU comparator)
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128)])
+def test_seq_scan_varlen(dtype, d):
+    w = make_prefill("varlen", seqlens=[1, 63, 0, 130], H=2, d=d, dtype=dtype, s0=True, seed=2)
+    dw = to_dev(w)
+    o, S_T = gdn.seq_scan(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], dw["cu_seqlens"])
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, dtype, "seq_scan")
+
+
+# ------------------------------------------------------------------ chunked prefill
+
+def chunk(dw, **kw):
+    return gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], dw["cu_seqlens"], check=True, **kw)
+
+
+def test_chunk_tiny_fp32_config():
+    w = make_prefill("tiny", seed=0)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "f32", "tiny")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+def test_chunk_ragged_small(dtype, d):
+    # several tiles, partial chunks, one-token and empty sequences
+    w = make_prefill("varlen", seqlens=[1, 63, 64, 65, 0, 200], H=3, d=d, dtype=dtype, s0=True, seed=3)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, dtype, "ragged")
+    # empty sequence (index 4) returns its initial state exactly
+    assert torch.equal(S_T[4].cpu(), w["S0"][4])
+
+
+def test_chunk_no_initial_state_equal_split():
+    w = make_prefill("prefill_2k", seqlens=[192, 192], H=2, s0=False, seed=4)
+    dw = to_dev(w)
+    o, S_T = gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], None, None, N=2, check=True)
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "equal split")
+
+
+def test_chunk_slow_decay_stress():
+    """Slow decay, beta near one: the state carries information across many chunks."""
+    w = make_prefill("prefill_2k", seqlens=[1500], H=2, s0=True, stress=True, seed=5)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "stress")
+
+
+@pytest.mark.parametrize("name", ["prefill_2k", "prefill_10k", "varlen"])
+def test_chunk_full_configs(name):
+    w = make_prefill(name, seed=0)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, w["dtype"], name)
+
+
+@pytest.mark.parametrize("T1", [64, 100])
+def test_chunk_resume_from_state(T1):
+    """Running [0, T) equals running [0, T1) then [T1, T) from S_T1 (on and off a chunk boundary)."""
+    w = make_prefill("prefill_2k", seqlens=[300], H=2, s0=True, seed=6)
+    dw = to_dev(w)
+    o_full, S_full = chunk(dw)
+    a = {k: (v[:T1] if k in ("q", "k", "v", "g", "beta") else v) for k, v in dw.items()}
+    a["cu_seqlens"] = None
+    o1, S1 = gdn.chunk_fwd(a["q"], a["k"], a["v"], a["g"], a["beta"], dw["S0"], None, check=True)
+    b = {k: (v[T1:].contiguous() if k in ("q", "k", "v", "g", "beta") else v) for k, v in dw.items()}
+    o2, S2 = gdn.chunk_fwd(b["q"], b["k"], b["v"], b["g"], b["beta"], S1, None, check=True)
+    ref = torch.cat([o1, o2]).float()
+    assert rel_err(ref, o_full.double().cpu().numpy()) <= 1e-2
+    assert rel_err(S2, S_full.double().cpu().numpy()) <= 1e-2
+
+
+def test_chunk_in_place_state():
+    """S0 may alias S_T."""
+    w = make_prefill("varlen", seqlens=[100, 37], H=2, d=128, s0=True, seed=7)
+    dw = to_dev(w)
+    S = dw["S0"].clone()
+    o, S_T = gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], S, dw["cu_seqlens"], S_T=S, check=True)
+    o_ref, S_ref = run_oracle(w)
+    check(o, S, o_ref, S_ref, "bf16", "in place")
+
+
+def test_chunk_equals_decode_steps():
+    """Prefill over T tokens equals T decode steps (one sequence)."""
+    w = make_prefill("prefill_2k", seqlens=[70], H=2, s0=True, seed=8)
+    dw = to_dev(w)
+    o, S_T = chunk(dw)
+    S = dw["S0"].clone()
+    outs = [gdn.decode_step(dw["q"][t:t + 1], dw["k"][t:t + 1], dw["v"][t:t + 1], dw["g"][t:t + 1],
+                            dw["beta"][t:t + 1], S) for t in range(70)]
+    assert rel_err(o, torch.cat(outs).double().cpu().numpy()) <= 2e-2
+    assert rel_err(S_T, S.double().cpu().numpy()) <= 2e-2
+
+
+def test_chunk_malformed_seqlens_reported_not_written():
+    w = make_prefill("varlen", seqlens=[50, 50, 28], H=2, d=64, dtype="f32", s0=True, seed=9)
+    dw = to_dev(w)
+    bad = torch.tensor([0, 100, 50, 128], dtype=torch.int32, device="cuda")  # decreasing offset
+    o = torch.full_like(dw["v"], 7.0)
+    S_T = torch.full_like(dw["S0"], 7.0)
+    with pytest.raises(gdn.GdnError) as ei:
+        gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], bad, o=o, S_T=S_T, check=True)
+    assert ei.value.status == 5
+    assert bool((o == 7.0).all()) and bool((S_T == 7.0).all())
+
+
+# ------------------------------------------------------------------ tensor-core tile diagnostics
+
+@pytest.mark.parametrize("variant", [0, 1])
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (256, 32)])
+def test_diag_mma_m128(variant, a_mn, b_mn, N, K):
+    g = torch.Generator().manual_seed(N + K)
+    A = torch.randn(128, K, generator=g).bfloat16()
+    B = torch.randn(N, K, generator=g).bfloat16()
+    D = gdn.diag_mma_tile(A.cuda(), B.cuda(), a_mn, b_mn, variant).cpu()
+    ref = A.float() @ B.float().T
+    assert torch.allclose(D, ref, atol=1e-3, rtol=1e-3), (D - ref).abs().max()
+
+
+def test_diag_mma_m64_lane_map():
+    """Where the rows of an M=64 accumulator land in TMEM (recorded for the kernels)."""
+    g = torch.Generator().manual_seed(64)
+    A = torch.randn(64, 64, generator=g).bfloat16()
+    B = torch.randn(64, 64, generator=g).bfloat16()
+    D = gdn.diag_mma_tile(A.cuda(), B.cuda(), 0, 0, 0).cpu()
+    ref = A.float() @ B.float().T
+    lanes = []
+    for r in range(64):
+        hit = [ln for ln in range(128) if torch.allclose(D[ln], ref[r], atol=1e-3, rtol=1e-3)]
+        lanes.append(hit[0] if hit else -1)
+    print("M64 row->lane:", lanes)
+    assert all(x >= 0 for x in lanes), lanes
