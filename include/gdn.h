@@ -16,8 +16,8 @@
  * interface; this one is the library's own.
  *
  * Conventions shared by every entry point
- *   - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous,
- *     owned by the caller. The library allocates no memory, never synchronises
+ *   - All tensor pointers are DEVICE pointers, contiguous, owned by the
+ *     caller, and 16-byte aligned (g and beta: 4-byte aligned). The library allocates no memory, never synchronises
  *     the stream (except gdn_chunk_fwd_check, which exists to do so), and
  *     launches everything on `stream` (a cudaStream_t passed as void*; NULL =
  *     the legacy default stream).

@@ -1,0 +1,458 @@
+// Chunked gated delta rule on the sm_100a tensor cores (bf16 inputs, d = 128,
+// chunk C = 64): tcgen05.mma with bf16 operands staged in shared memory and
+// fp32 accumulators in TMEM; the fp32 state lives in TMEM for the whole
+// sequence.
+//
+// The pages give the shape of the method only: the token-by-token scan of
+// the recurrent layers becomes a chunk-wise delta-rule form with an
+// intra-chunk part, an inter-chunk part and a forward-substitution step,
+// whose one slow kernel had to be fixed before the chunked form won (page 1,
+// abstract, result (i); page 2, "Resumen Tecnico", Metodologia,
+// recurrent-layer item, and the narrative's second finding). Per chunk of
+// one (sequence, head), with S the d_v x d_k state entering the chunk,
+// G_r = sum_{s<=r} g_s, gamma_r = exp(G_r), e_s = exp(G_C - G_s):
+//
+//   X1 = [K;Q] K^T                  A_rs = beta_r exp(G_r-G_s) (KK^T)_rs, s<r
+//                                   P_rs = exp(G_r-G_s) (QK^T)_rs,      s<=r
+//   T  = (I + A)^{-1}               fp32 forward substitution, 16x16 blocks
+//   W^T = K^T (T diag(beta gamma))^T,   U^T = V^T (T diag(beta))^T
+//   O1 = S Q^T,   Dl = U^T - S W^T  (= Delta^T),   Dt = Delta^T diag(e)
+//   O^T = O1 diag(gamma) + Dl P^T   (written to o)
+//   S  <- gamma_C S + Dt K          (the state entering the next chunk)
+//
+// Every product is one M = 128 tcgen05.mma group (D = A B^T): the rows of an
+// accumulator map 1:1 to TMEM lanes and to the CTA's 128 threads, so each
+// thread owns one row of every accumulator (a key row, a position row or a
+// value row of S) and writes it back in whichever shared-memory orientation
+// the next MMA wants. No operand is ever transposed through shared memory:
+// a tile written with 16-byte runs along one axis is read either K-major or
+// MN-major (see tc.cuh).
+//
+// One CTA (4 warps) per (sequence, head) walks its chunks in order; chunk
+// c+1's K, Q, V, g, beta are fetched with cp.async while chunk c computes.
+// Partial chunks are zero-filled (k = q = v = 0, g = 0, beta = 0), which
+// zeroes their rows of A, W, U, Delta and keeps G flat.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace gdn {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int C = 64;     // chunk length
+constexpr int D = 128;    // head size (dk = dv)
+constexpr int NT = 128;   // threads per CTA (one per TMEM lane)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---- shared memory map (bytes). Tiles use 8x16-byte core matrices with
+// X-neighbouring core matrices adjacent (sx = 128) and sy = 16 * rows.
+namespace sm {
+// double-buffered chunk inputs, buffer b in {0, 1}
+__device__ __forceinline__ constexpr uint32_t KQ(int b) { return b ? 32768u : 0u; }      // [K rows 0..63; Q rows 64..127] x 128 d, sy = 2048
+__device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 81920u : 65536u; }   // 64 s x 128 d, sy = 1024
+__device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 98816u : 98304u; }  // raw g[64], beta[64] (fp32)
+constexpr uint32_t T1 = 99328;                  // 64 r x 64 s, sy = 1024   (T diag(beta gamma))
+constexpr uint32_t T2 = 107520;                 // 64 r x 64 s               (T diag(beta))
+constexpr uint32_t P = 115712;                  // 64 r x 64 s
+constexpr uint32_t W = 123904;                  // 128 k x 64 r, sy = 2048 (runs along r)
+constexpr uint32_t S = 140288;                  // 128 v x 128 k, sy = 2048 (bf16 copy of the state)
+constexpr uint32_t UNI = 173056;                // union: {Dl, Dt} bf16  |  {A, T} fp32 [64][65]
+constexpr uint32_t DL = UNI, DT = UNI + 16384;  // 128 v x 64 s, sy = 2048
+constexpr uint32_t AF = UNI, TF = UNI + 16640;
+constexpr uint32_t VEC = UNI + 33280;           // G (log2 units), gamma, e, beta: 4 x 64 fp32
+constexpr uint32_t BAR = VEC + 1024;            // 4 mbarriers + TMEM slot
+constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t SCR = W;                     // fp32 scratch of the solve (W is free then)
+}  // namespace sm
+constexpr int AP = 65;  // pitch of the fp32 A / T matrices
+
+// TMEM columns (512 allocated): fp32 state S, state update, X1 then W^T, U^T,
+// Delta-part then O2, O1.
+constexpr uint32_t TM_S = 0, TM_SU = 128, TM_XW = 256, TM_U = 320, TM_DD = 384, TM_O1 = 448;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+// Eight fp32 values as one 16-byte bf16 run.
+__device__ __forceinline__ void st_run8(uint32_t addr, const float *x) {
+    st_shared_v4(addr, tc::pack_bf16x2(x[0], x[1]), tc::pack_bf16x2(x[2], x[3]), tc::pack_bf16x2(x[4], x[5]),
+                 tc::pack_bf16x2(x[6], x[7]));
+}
+
+// Issue the cp.async copies of chunk [cs, cs + L) of head h into buffer b.
+__device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q, const bf16 *k, const bf16 *v,
+                                           const float *g, const float *beta, int cs, int L, int H, int h) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    const uint32_t kq = sbase + sm::KQ(b), vt = sbase + sm::V(b);
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int idx = it * NT + tid;
+        const int row = ((idx >> 5) & 7) * 8 + (lane >> 2);
+        const int j = (idx >> 8) * 4 + (lane & 3);  // 16-byte run along d
+        const bool ok = row < L;
+        const size_t off = ((size_t)(cs + (ok ? row : 0)) * H + h) * D + 8 * j;
+        const uint32_t nb = ok ? 16u : 0u;
+        cp_async16(kq + tc::tile_off(row, 8 * j, 128, 2048), k + off, nb);
+        cp_async16(kq + tc::tile_off(64 + row, 8 * j, 128, 2048), q + off, nb);
+        cp_async16(vt + tc::tile_off(row, 8 * j, 128, 1024), v + off, nb);
+    }
+    if (tid < C) {
+        const bool ok = tid < L;
+        const size_t off = (size_t)(cs + (ok ? tid : 0)) * H + h;
+        cp_async4(sbase + sm::GB(b) + 4 * tid, g + off, ok ? 4u : 0u);
+        cp_async4(sbase + sm::GB(b) + 256 + 4 * tid, beta + off, ok ? 4u : 0u);
+    }
+    cp_async_commit();
+}
+
+// T = (I + A)^{-1} for the strictly lower-triangular 64x64 fp32 A (pitch AP):
+// the four diagonal 16x16 blocks by forward substitution (one warp each),
+// then off-diagonal blocks level by level, T_ij = -T_ii sum_{m=j}^{i-1} A_im T_mj.
+__device__ void ut_solve(const float *A, float *T, float *X) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // zero the strictly upper block triangle
+    for (int e = tid; e < 6 * 256; e += NT) {
+        const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
+        const int bi = (b < 3) ? 0 : (b < 5 ? 1 : 2);
+        const int bj = (b < 3) ? b + 1 : (b < 5 ? b - 1 : 3);
+        T[(16 * bi + ri) * AP + 16 * bj + cj] = 0.f;
+    }
+    if (lane < 16) {
+        const int j = lane, o = 16 * warp;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float acc = (i == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int s = 0; s < i; ++s) acc = fmaf(-A[(o + i) * AP + o + s], x[s], acc);
+            x[i] = acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) T[(o + i) * AP + o + j] = x[i];
+    }
+    __syncthreads();
+    for (int lvl = 1; lvl < 4; ++lvl) {
+        const int nb = 4 - lvl;
+        for (int e = tid; e < nb * 256; e += NT) {
+            const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
+            const int bi = b + lvl, bj = b;
+            float acc = 0.f;
+            for (int m = bj; m < bi; ++m)
+#pragma unroll
+                for (int s = 0; s < 16; ++s)
+                    acc = fmaf(A[(16 * bi + ri) * AP + 16 * m + s], T[(16 * m + s) * AP + 16 * bj + cj], acc);
+            X[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < nb * 256; e += NT) {
+            const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
+            const int bi = b + lvl, bj = b;
+            float acc = 0.f;
+#pragma unroll
+            for (int s = 0; s < 16; ++s) acc = fmaf(T[(16 * bi + ri) * AP + 16 * bi + s], X[b * 256 + s * 16 + cj], acc);
+            T[(16 * bi + ri) * AP + 16 * bj + cj] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+// All threads agree whether the wait failed (bounded wait on the MMA barrier).
+__device__ __forceinline__ bool wait_all_ok(uint64_t *bar, uint32_t parity) {
+    const bool ok = tc::mbar_wait(bar, parity);
+    tc::fence_after_sync();
+    return __syncthreads_and(ok) != 0;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    k_chunk_tc(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
+               const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
+               const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o, float *S_T,
+               uint32_t *__restrict__ err) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;  // malformed cu_seqlens: write nothing
+    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+    int t0, t1;
+    seq_bounds(cu, n, N, T_tot, t0, t1);
+    const uint32_t sb = tc::smem_u32(smem);
+    float *Gl = reinterpret_cast<float *>(smem + sm::VEC);  // G * log2(e)
+    float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + sm::BAR);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + sm::BAR + 32);
+
+    if (warp == 0) tc::tmem_alloc(tslot, 512);
+    if (tid == 0) {
+        for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = *tslot;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
+    const size_t sidx = ((size_t)n * H + h) * D * D;
+
+    // ---- initial state: thread v owns row v (fp32 in TMEM, bf16 copy in the S tile)
+    {
+        const float *src = S0 ? S0 + sidx + (size_t)tid * D : nullptr;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float r[16];
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                float4 x = src ? *reinterpret_cast<const float4 *>(src + c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[i] = x.x; r[i + 1] = x.y; r[i + 2] = x.z; r[i + 3] = x.w;
+            }
+            tc::tmem_st16(tm + lane_off + TM_S + c0, r);
+            st_run8(sb + sm::S + tc::tile_off(tid, c0, 128, 2048), r);
+            st_run8(sb + sm::S + tc::tile_off(tid, c0 + 8, 128, 2048), r + 8);
+        }
+        tc::tmem_st_wait();
+    }
+    const int nchunks = (t1 - t0 + C - 1) / C;
+    if (nchunks > 0) load_chunk(sb, 0, q, k, v, g, beta, t0, min(C, t1 - t0), H, h);
+
+    const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
+    const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+    const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
+    const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+    bool ok = true;
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int cs = t0 + c * C, L = min(C, t1 - cs), b = c & 1;
+        const uint32_t par = (uint32_t)(c & 1);
+        const uint32_t kq = sb + sm::KQ(b), vt = sb + sm::V(b);
+        const float *graw = reinterpret_cast<const float *>(smem + sm::GB(b));
+        cp_async_wait_all();
+        tc::fence_smem_to_async();
+        __syncthreads();
+        // ---- G = cumsum(g) in log2 units (warp 0, two positions per lane), gamma, e, beta
+        if (warp == 0) {
+            const int l = tid;
+            const float a = graw[2 * l] * kLog2e, b2 = a + graw[2 * l + 1] * kLog2e;
+            float sc = b2;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, off);
+                if (l >= off) sc += y;
+            }
+            const float base = sc - b2;
+            Gl[2 * l] = base + a;
+            Gl[2 * l + 1] = sc;
+        }
+        __syncthreads();
+        if (tid < C) {
+            gam[tid] = exp2f(Gl[tid]);
+            dte[tid] = exp2f(Gl[C - 1] - Gl[tid]);
+            bet[tid] = graw[64 + tid];
+        }
+        // ---- MMA group 1: X1 = [K;Q] K^T and O1 = S Q^T
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::make_desc(kq + kk * 4096, 2048, 128);
+                tc::mma_bf16(tm + TM_XW, a, a, id_kk64, kk > 0);  // B = first 64 rows of the same tile (K)
+            }
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::make_desc(sb + sm::S + kk * 4096, 2048, 128);
+                const uint64_t bq = tc::make_desc(kq + 1024 + kk * 4096, 2048, 128);
+                tc::mma_bf16(tm + TM_O1, a, bq, id_kk64, kk > 0);
+            }
+            tc::mma_commit(&bars[0]);
+        }
+        if (c + 1 < nchunks) load_chunk(sb, b ^ 1, q, k, v, g, beta, cs + C, min(C, t1 - cs - C), H, h);
+        if (!(ok = wait_all_ok(&bars[0], par))) break;
+        // ---- X1 epilogue: rows 0..63 -> A (fp32), rows 64..127 -> P (bf16 tile)
+        {
+            float *A = reinterpret_cast<float *>(smem + sm::AF);
+            const int r = tid & 63;
+            const float Gr = Gl[r];
+#pragma unroll
+            for (int c0 = 0; c0 < C; c0 += 16) {
+                float x[16];
+                tc::tmem_ld16(tm + lane_off + TM_XW + c0, x);
+                if (tid < 64) {
+                    const float br = bet[r];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int s = c0 + i;
+                        A[r * AP + s] = (s < r) ? br * exp2f(Gr - Gl[s]) * x[i] : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int s = c0 + i;
+                        x[i] = (s <= r) ? exp2f(Gr - Gl[s]) * x[i] : 0.f;
+                    }
+                    st_run8(sb + sm::P + tc::tile_off(r, c0, 128, 1024), x);
+                    st_run8(sb + sm::P + tc::tile_off(r, c0 + 8, 128, 1024), x + 8);
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- T = (I + A)^{-1}; T1 = T diag(beta gamma), T2 = T diag(beta) as bf16 tiles
+        {
+            const float *A = reinterpret_cast<const float *>(smem + sm::AF);
+            float *T = reinterpret_cast<float *>(smem + sm::TF);
+            ut_solve(A, T, reinterpret_cast<float *>(smem + sm::SCR));
+            const int r = tid & 63;
+            const uint32_t dst = sb + (tid < 64 ? sm::T1 : sm::T2);
+#pragma unroll
+            for (int s0 = 0; s0 < C; s0 += 8) {
+                float x[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int s = s0 + i;
+                    x[i] = T[r * AP + s] * bet[s] * (tid < 64 ? gam[s] : 1.f);
+                }
+                st_run8(dst + tc::tile_off(r, s0, 128, 1024), x);
+            }
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- MMA group 2: W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views)
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                tc::mma_bf16(tm + TM_XW, tc::make_desc(kq + kk * 256, 128, 2048),
+                             tc::make_desc(sb + sm::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                tc::mma_bf16(tm + TM_U, tc::make_desc(vt + kk * 256, 128, 1024),
+                             tc::make_desc(sb + sm::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+            }
+            tc::mma_commit(&bars[1]);
+        }
+        if (!(ok = wait_all_ok(&bars[1], par))) break;
+        // ---- W epilogue: thread k writes W[., k] as a row of the W tile (runs along r)
+#pragma unroll
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float x[16];
+            tc::tmem_ld16(tm + lane_off + TM_XW + c0, x);
+            st_run8(sb + sm::W + tc::tile_off(tid, c0, 128, 2048), x);
+            st_run8(sb + sm::W + tc::tile_off(tid, c0 + 8, 128, 2048), x + 8);
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- MMA group 3: S W^T (B operand: MN-major view of the W tile)
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + sm::S + kk * 4096, 2048, 128),
+                             tc::make_desc(sb + sm::W + kk * 256, 128, 2048), id_km64, kk > 0);
+            tc::mma_commit(&bars[2]);
+        }
+        if (!(ok = wait_all_ok(&bars[2], par))) break;
+        // ---- Delta epilogue: Delta^T[v][s] = U^T[v][s] - (S W^T)[v][s]; Dl = Delta^T, Dt = Delta^T diag(e)
+#pragma unroll
+        for (int c0 = 0; c0 < C; c0 += 16) {
+            float u[16], d[16];
+            tc::tmem_ld16(tm + lane_off + TM_U + c0, u);
+            tc::tmem_ld16(tm + lane_off + TM_DD + c0, d);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) u[i] -= d[i];
+            st_run8(sb + sm::DL + tc::tile_off(tid, c0, 128, 2048), u);
+            st_run8(sb + sm::DL + tc::tile_off(tid, c0 + 8, 128, 2048), u + 8);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) u[i] *= dte[c0 + i];
+            st_run8(sb + sm::DT + tc::tile_off(tid, c0, 128, 2048), u);
+            st_run8(sb + sm::DT + tc::tile_off(tid, c0 + 8, 128, 2048), u + 8);
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+        // ---- MMA group 4: O2 = Dl P^T (into the Delta-part columns), SU = Dt K (B: MN-major view of K)
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + sm::DL + kk * 4096, 2048, 128),
+                             tc::make_desc(sb + sm::P + kk * 2048, 1024, 128), id_kk64, kk > 0);
+                tc::mma_bf16(tm + TM_SU, tc::make_desc(sb + sm::DT + kk * 4096, 2048, 128),
+                             tc::make_desc(kq + kk * 256, 128, 2048), id_km128, kk > 0);
+            }
+            tc::mma_commit(&bars[3]);
+        }
+        if (!(ok = wait_all_ok(&bars[3], par))) break;
+        // ---- outputs: o[cs + r][h][v] = gamma_r O1[v][r] + O2[v][r]  (thread v, r < L)
+        {
+            bf16 *orow = o + ((size_t)cs * H + h) * D + tid;
+#pragma unroll
+            for (int c0 = 0; c0 < C; c0 += 16) {
+                float a[16], d[16];
+                tc::tmem_ld16(tm + lane_off + TM_O1 + c0, a);
+                tc::tmem_ld16(tm + lane_off + TM_DD + c0, d);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (c0 + i < L) orow[(size_t)(c0 + i) * H * D] = __float2bfloat16_rn(fmaf(gam[c0 + i], a[i], d[i]));
+            }
+        }
+        // ---- state: S <- gamma_C S + SU (fp32 in TMEM), bf16 copy to the S tile
+        {
+            const float gC = gam[C - 1];
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float s[16], u[16];
+                tc::tmem_ld16(tm + lane_off + TM_S + c0, s);
+                tc::tmem_ld16(tm + lane_off + TM_SU + c0, u);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) s[i] = fmaf(gC, s[i], u[i]);
+                tc::tmem_st16(tm + lane_off + TM_S + c0, s);
+                st_run8(sb + sm::S + tc::tile_off(tid, c0, 128, 2048), s);
+                st_run8(sb + sm::S + tc::tile_off(tid, c0 + 8, 128, 2048), s + 8);
+            }
+            tc::tmem_st_wait();
+        }
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
+    }
+    cp_async_wait_all();
+    if (!ok) {
+        if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
+    } else {
+        // ---- final state
+        float *dst = S_T + sidx + (size_t)tid * D;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float r[16];
+            tc::tmem_ld16(tm + lane_off + TM_S + c0, r);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<float4 *>(dst + c0 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+}  // namespace
+
+size_t chunk_tc_smem_bytes() { return sm::TOTAL; }
+
+cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
+                            const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
+                            uint32_t *err, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm::TOTAL);
+    if (e != cudaSuccess) return e;
+    dim3 grid(H, N);
+    k_chunk_tc<<<grid, NT, sm::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -89,9 +89,11 @@ gdn_status check_common(const void *q, const void *k, const void *v, const float
     if (dk != dv || (dk != 64 && dk != 128))
         return fail(GDN_ERR_SHAPE, "head sizes dk=%d dv=%d unsupported (need dk == dv in {64, 128})", dk, dv);
     if (T_tot > 0 && (!q || !k || !v || !g || !beta || !o)) return fail(GDN_ERR_NULL, "q, k, v, g, beta and o are required");
-    const void *ptrs[] = {q, k, v, g, beta, o};
+    const void *ptrs[] = {q, k, v, o};
     for (const void *p : ptrs)
         if (misaligned(p)) return fail(GDN_ERR_ALIGN, "tensor pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(g) | reinterpret_cast<uintptr_t>(beta)) & 3u)
+        return fail(GDN_ERR_ALIGN, "g and beta must be 4-byte aligned");
     if ((double)T_tot * H * dk >= 9.0e18) return fail(GDN_ERR_SHAPE, "sizes overflow");
     return GDN_OK;
 }
@@ -155,6 +157,14 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
     }
     if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens validation launch");
 
+    if (dtype == GDN_BF16 && dk == 128) {
+        ProfScope ps("chunk_tc", st);
+        e = gdn::launch_chunk_tc(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                                 static_cast<const __nv_bfloat16 *>(v), g, beta, S0, cu_seqlens, N, T_tot, H,
+                                 static_cast<__nv_bfloat16 *>(o), S_T, err, st);
+        if (e != cudaSuccess) return cuda_fail(e, "chunked forward (tensor-core) launch");
+        return ok();
+    }
     ProfScope ps("chunk_simt", st);
     if (dtype == GDN_F32) {
         const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),

@@ -21,6 +21,12 @@ cudaError_t launch_chunk_simt(const T *q, const T *k, const T *v, const float *g
                               const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, const uint32_t *err,
                               cudaStream_t st);
 
+// Tensor-core chunked forward, bf16 inputs, dk = dv = 128 (one CTA per (sequence, head)).
+cudaError_t launch_chunk_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const float *g,
+                            const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
+                            __nv_bfloat16 *o, float *S_T, uint32_t *err, cudaStream_t st);
+size_t chunk_tc_smem_bytes();
+
 // Writes the workspace error word: ERRBIT_SEQLENS if cu_seqlens (device, N+1
 // entries) is not 0 = c0 <= ... <= cN = T_tot, else 0. With cu == NULL it
 // just clears the word.

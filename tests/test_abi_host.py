@@ -71,6 +71,7 @@ def chunk_args(**over):
     (dict(q=None), 1),
     (dict(S_T=None), 1),
     (dict(k=FAKE_MIS), 4),                # alignment
+    (dict(g=ctypes.c_void_p((1 << 20) + 2)), 4),
     (dict(N=3, T=128), 5),                # equal split impossible
     (dict(ws=None), 6),
     (dict(ws_bytes=8), 6),

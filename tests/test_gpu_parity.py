@@ -1,6 +1,8 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
 same seeded inputs. Tolerance: max|gpu - oracle| / max|oracle| <= 1e-4 for
 fp32 inputs and 2e-2 for bf16 inputs, for o and for the final state."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -166,8 +168,9 @@ def test_chunk_equals_decode_steps():
     assert rel_err(S_T, S.double().cpu().numpy()) <= 2e-2
 
 
-def test_chunk_malformed_seqlens_reported_not_written():
-    w = make_prefill("varlen", seqlens=[50, 50, 28], H=2, d=64, dtype="f32", s0=True, seed=9)
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128)])
+def test_chunk_malformed_seqlens_reported_not_written(dtype, d):
+    w = make_prefill("varlen", seqlens=[50, 50, 28], H=2, d=d, dtype=dtype, s0=True, seed=9)
     dw = to_dev(w)
     bad = torch.tensor([0, 100, 50, 128], dtype=torch.int32, device="cuda")  # decreasing offset
     o = torch.full_like(dw["v"], 7.0)
@@ -203,5 +206,7 @@ def test_diag_mma_m64_lane_map():
     for r in range(64):
         hit = [ln for ln in range(128) if torch.allclose(D[ln], ref[r], atol=1e-3, rtol=1e-3)]
         lanes.append(hit[0] if hit else -1)
-    print("M64 row->lane:", lanes)
+    os.makedirs("gpurun_out", exist_ok=True)
+    with open(os.path.join("gpurun_out", "m64_lane_map.txt"), "w") as f:
+        f.write("M=64 accumulator row -> TMEM lane: %s\n" % lanes)
     assert all(x >= 0 for x in lanes), lanes
