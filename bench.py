@@ -446,6 +446,33 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+def case_arm(args):
+    """Run one workload's library calls back to back (for ncu / launch lists): WARMUP+STEPS calls."""
+    import torch
+
+    from linear_attention_recurrent_chunked_b200 import gdn
+    from linear_attention_recurrent_chunked_b200.workloads import make_decode, make_prefill
+    dev = torch.device("cuda", 0)
+    gdn.load_library()
+    n = args.warmup + args.steps
+    if args.case == "decode":
+        w = make_decode(seed=0)
+        t = {k: w[k].to(dev) for k in ("q", "k", "v", "g", "beta", "S")}
+        for i in range(n):
+            j = i % w["steps"]
+            gdn.decode_step(t["q"][j], t["k"][j], t["v"][j], t["g"][j], t["beta"][j], t["S"])
+    else:
+        name = args.case[5:] if args.case.startswith("scan_") else args.case
+        name = {"2k": "prefill_2k", "10k": "prefill_10k"}.get(name, name)
+        w = make_prefill(name, seed=0)
+        t = {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in w.items()}
+        fn = gdn.seq_scan if args.case.startswith("scan_") else gdn.chunk_fwd
+        for _ in range(n):
+            fn(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], t["cu_seqlens"])
+    torch.cuda.synchronize()
+    print("case %s: %d calls done" % (args.case, n))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -453,10 +480,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--quick", action="store_true", help="main workload only (no 10k/varlen/decode/scan extras)")
+    ap.add_argument("--case", default=None,
+                    help="profiling mode: run only WARMUP+STEPS calls of one workload (prefill_2k, prefill_10k, "
+                         "varlen, tiny, decode, scan_2k) and print nothing but a one-line summary")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.case:
+        case_arm(args)
+    elif args.impl == "reference":
         reference_arm(args)
     else:
         gpu_arm(args)
