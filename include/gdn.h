@@ -111,6 +111,32 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd without a caller-provided workspace, for callers that cannot
+ * allocate device memory: code running under a memory manager that has
+ * already reserved the GPU's memory, plugins whose host application owns
+ * every device allocation, and latency-critical paths that must not pay
+ * cudaMalloc's implicit synchronisation. The paper has no counterpart of
+ * this entry point; it is a property of this library only.
+ *
+ * Arguments, results and dtype dispatch are those of gdn_chunk_fwd; the
+ * workspace comes from an 8 MiB array built into the library, which every
+ * GPU that loads the library holds until the process exits. Sizes whose
+ * gdn_chunk_fwd_workspace_size exceeds 8 MiB are rejected with
+ * GDN_ERR_WORKSPACE. The call allocates nothing. Its first call on a device
+ * (with that device current) looks up the array's device address once;
+ * make that first call before any stream capture. All calls on a device
+ * share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller. A malformed device cu_seqlens still makes the
+ * kernels write nothing, but this entry point offers no way to read the
+ * device error word: validate cu_seqlens with gdn_chunk_fwd +
+ * gdn_chunk_fwd_check when it is untrusted.
+ */
+gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                 const float *g, const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                                 int dtype, void *o, float *S_T, void *stream);
+
+/*
  * Synchronises `stream` and reads the device error word that the last
  * gdn_chunk_fwd on this workspace wrote: GDN_OK, GDN_ERR_SEQLENS or
  * GDN_ERR_TIMEOUT (a bounded inter-block wait gave up; outputs are then

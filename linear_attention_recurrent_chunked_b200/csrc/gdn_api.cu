@@ -118,6 +118,9 @@ cudaError_t launch_validate_seqlens(const int32_t *cu, int N, int T_tot, uint32_
     return cudaGetLastError();
 }
 
+// Sets the calling thread's last-error message (for entry points defined in other files).
+gdn_status record_error(gdn_status s, const char *msg) { return fail(s, "%s", msg); }
+
 }  // namespace gdn
 
 extern "C" {

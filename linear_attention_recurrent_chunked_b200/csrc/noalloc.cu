@@ -1,0 +1,77 @@
+// gdn_chunk_fwd_noalloc: the chunked forward with its scratch memory built into
+// the library, for callers that cannot allocate device memory themselves.
+//
+// Who needs it: code running under a memory manager that has already reserved
+// the GPU's memory (so a cudaMalloc would fail or fragment the pool), plugins
+// whose host application owns all device allocations, and latency-critical
+// paths that must not pay cudaMalloc / cudaFree's implicit synchronisation.
+// They still pass their own inputs and outputs; only the workspace that
+// gdn_chunk_fwd normally receives from the caller comes from here.
+//
+// The scratch is a file-scope __device__ array, so every GPU that loads the
+// library holds kNoallocScratchBytes of it until the process exits. In host
+// code the array's name is only a host-side stand-in, never a device address:
+// the device address is looked up once per device with cudaGetSymbolAddress
+// (on the first call made while that device is current) and cached. All calls
+// on a device share the one array; it keeps whatever the last call left in it,
+// and the forward path rewrites everything it reads (the error word included)
+// before use. Calls that overlap on the GPU (different streams, or threads
+// racing on one stream) race on the array and must be serialised by the caller.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace gdn {
+gdn_status record_error(gdn_status s, const char *msg);
+}
+
+namespace {
+
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_scratch_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once per device).
+cudaError_t scratch_for_current_device(void **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype);
+extern "C" gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                    const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk,
+                                    int dv, int dtype, void *o, float *S_T, void *workspace, size_t ws_bytes,
+                                    void *stream);
+
+extern "C" gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                                            const float *beta, const float *S0, const int32_t *cu_seqlens, int N,
+                                            int T_tot, int H, int dk, int dv, int dtype, void *o, float *S_T,
+                                            void *stream) {
+    const size_t need = gdn_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dtype);
+    if (need > kNoallocScratchBytes)
+        return gdn::record_error(GDN_ERR_WORKSPACE,
+                                 "these sizes need more scratch than the built-in 8 MiB; use gdn_chunk_fwd "
+                                 "with a caller-provided workspace");
+    void *ws = nullptr;
+    const cudaError_t e = scratch_for_current_device(&ws);
+    if (e != cudaSuccess) return gdn::record_error(GDN_ERR_CUDA, cudaGetErrorString(e));
+    return gdn_chunk_fwd(q, k, v, g, beta, S0, cu_seqlens, N, T_tot, H, dk, dv, dtype, o, S_T, ws,
+                         kNoallocScratchBytes, stream);
+}

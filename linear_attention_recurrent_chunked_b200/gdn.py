@@ -33,6 +33,7 @@ SIGNATURES = {
     "gdn_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_seq_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
     "gdn_diag_mma_tile": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "gdn_chunk_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
     "gdn_profile_enable": (None, [_I]),
     "gdn_profile_read": (_I, [ctypes.c_char_p, _SZ, _VP, _VP, _I]),
 }
@@ -127,6 +128,27 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = Non
                              N, T_tot, H, dk, dv, dt, _ptr(o), _ptr(S_T), _ptr(ws), ws.numel(), _stream()))
     if check:
         _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
+    return o, S_T
+
+
+def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = None, o=None, S_T=None):
+    """chunk_fwd without a workspace argument: the library's built-in scratch
+    array is used instead (see include/gdn.h). o and S_T are allocated here
+    only when the caller does not pass them."""
+    lib = load_library()
+    _need_cuda(q, k, v, g, beta, S0, cu_seqlens, o, S_T)
+    T_tot, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N = S0.shape[0] if S0 is not None else 1
+    if o is None:
+        o = torch.empty((T_tot, H, dv), dtype=q.dtype, device=q.device)
+    if S_T is None:
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device)
+    _check(lib.gdn_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                                     N, T_tot, H, dk, dv, _DTYPE.get(q.dtype, 99), _ptr(o), _ptr(S_T), _stream()))
     return o, S_T
 
 
