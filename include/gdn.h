@@ -189,6 +189,15 @@ gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, int M, int 
                              int a_mn, int b_mn, int variant, void *stream);
 
 /*
+ * Diagnostic (used by the tests): the chunked path's UT/WY solve on one
+ * matrix, T = (I + A)^{-1}, with A a 64 x 64 fp32 row-major device matrix
+ * that is zero on and above the diagonal and T its 64 x 64 fp32 result
+ * (page 2, "Resumen Tecnico", Metodologia, recurrent-layer item: the
+ * forward-substitution step of the chunked form). One CTA on `stream`.
+ */
+gdn_status gdn_diag_ut_solve(const float *A, float *T, void *stream);
+
+/*
  * Kernel timing (measurement support, off by default). While enabled, every
  * entry point records a CUDA event pair on its stream around each kernel it
  * launches. gdn_profile_read waits for those events, writes per kernel name

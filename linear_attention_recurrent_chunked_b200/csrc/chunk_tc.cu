@@ -14,27 +14,30 @@
 //
 //   X1 = [K;Q] K^T                  A_rs = beta_r exp(G_r-G_s) (KK^T)_rs, s<r
 //                                   P_rs = exp(G_r-G_s) (QK^T)_rs,      s<=r
-//   T  = (I + A)^{-1}               fp32 forward substitution, 16x16 blocks
+//   T  = (I + A)^{-1}               (ut_solve.cuh)
 //   W^T = K^T (T diag(beta gamma))^T,   U^T = V^T (T diag(beta))^T
 //   O1 = S Q^T,   Dl = U^T - S W^T  (= Delta^T),   Dt = Delta^T diag(e)
 //   O^T = O1 diag(gamma) + Dl P^T   (written to o)
 //   S  <- gamma_C S + Dt K          (the state entering the next chunk)
 //
-// Every product is one M = 128 tcgen05.mma group (D = A B^T): the rows of an
-// accumulator map 1:1 to TMEM lanes and to the CTA's 128 threads, so each
-// thread owns one row of every accumulator (a key row, a position row or a
-// value row of S) and writes it back in whichever shared-memory orientation
-// the next MMA wants. No operand is ever transposed through shared memory:
-// a tile written with 16-byte runs along one axis is read either K-major or
-// MN-major (see tc.cuh).
+// Every product is one M = 128 tcgen05.mma group (D = A B^T): accumulator row
+// m sits in TMEM lane m. The CTA has 8 warps; warp w reads TMEM lanes
+// 32*(w%4)..+31 and the two warpgroups split the columns, so each thread owns
+// half of one accumulator row (a key row, a position row or a value row of
+// S) and writes it back in whichever shared-memory orientation the next MMA
+// wants. No operand is ever transposed through shared memory: a tile written
+// with 16-byte runs along one axis is read either K-major or MN-major (see
+// tc.cuh). Outputs are staged through shared memory so that the stores to o
+// are whole 256-byte rows.
 //
-// One CTA (4 warps) per (sequence, head) walks its chunks in order; chunk
-// c+1's K, Q, V, g, beta are fetched with cp.async while chunk c computes.
-// Partial chunks are zero-filled (k = q = v = 0, g = 0, beta = 0), which
-// zeroes their rows of A, W, U, Delta and keeps G flat.
+// One CTA per (sequence, head) walks its chunks in order; chunk c+1's K, Q,
+// V, g, beta are fetched with cp.async while chunk c computes. Partial
+// chunks are zero-filled (k = q = v = 0, g = 0, beta = 0), which zeroes their
+// rows of A, W, U, Delta and keeps G flat.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
+#include "ut_solve.cuh"
 
 namespace gdn {
 namespace {
@@ -42,8 +45,9 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int C = 64;     // chunk length
 constexpr int D = 128;    // head size (dk = dv)
-constexpr int NT = 128;   // threads per CTA (one per TMEM lane)
+constexpr int NT = 256;   // threads per CTA (two threads per TMEM lane)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int AP = ut::AP;
 
 // ---- shared memory map (bytes). Tiles use 8x16-byte core matrices with
 // X-neighbouring core matrices adjacent (sx = 128) and sy = 16 * rows.
@@ -54,6 +58,7 @@ __device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 81920u : 655
 __device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 98816u : 98304u; }  // raw g[64], beta[64] (fp32)
 constexpr uint32_t T1 = 99328;                  // 64 r x 64 s, sy = 1024   (T diag(beta gamma))
 constexpr uint32_t T2 = 107520;                 // 64 r x 64 s               (T diag(beta))
+constexpr uint32_t OST = T1;                    // output staging o[r][v] bf16 (64 x 256 B), over T1+T2
 constexpr uint32_t P = 115712;                  // 64 r x 64 s
 constexpr uint32_t W = 123904;                  // 128 k x 64 r, sy = 2048 (runs along r)
 constexpr uint32_t S = 140288;                  // 128 v x 128 k, sy = 2048 (bf16 copy of the state)
@@ -65,7 +70,6 @@ constexpr uint32_t BAR = VEC + 1024;            // 4 mbarriers + TMEM slot
 constexpr uint32_t TOTAL = BAR + 64;
 constexpr uint32_t SCR = W;                     // fp32 scratch of the solve (W is free then)
 }  // namespace sm
-constexpr int AP = 65;  // pitch of the fp32 A / T matrices
 
 // TMEM columns (512 allocated): fp32 state S, state update, X1 then W^T, U^T,
 // Delta-part then O2, O1.
@@ -88,6 +92,12 @@ __device__ __forceinline__ void st_run8(uint32_t addr, const float *x) {
     st_shared_v4(addr, tc::pack_bf16x2(x[0], x[1]), tc::pack_bf16x2(x[2], x[3]), tc::pack_bf16x2(x[4], x[5]),
                  tc::pack_bf16x2(x[6], x[7]));
 }
+// 2^x on the MUFU unit (inputs here are <= 0; results below 2^-126 flush to zero).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Issue the cp.async copies of chunk [cs, cs + L) of head h into buffer b.
 __device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q, const bf16 *k, const bf16 *v,
@@ -95,7 +105,7 @@ __device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q,
     const int tid = threadIdx.x, lane = tid & 31;
     const uint32_t kq = sbase + sm::KQ(b), vt = sbase + sm::V(b);
 #pragma unroll
-    for (int it = 0; it < 8; ++it) {
+    for (int it = 0; it < 4; ++it) {
         const int idx = it * NT + tid;
         const int row = ((idx >> 5) & 7) * 8 + (lane >> 2);
         const int j = (idx >> 8) * 4 + (lane & 3);  // 16-byte run along d
@@ -106,67 +116,19 @@ __device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q,
         cp_async16(kq + tc::tile_off(64 + row, 8 * j, 128, 2048), q + off, nb);
         cp_async16(vt + tc::tile_off(row, 8 * j, 128, 1024), v + off, nb);
     }
-    if (tid < C) {
-        const bool ok = tid < L;
-        const size_t off = (size_t)(cs + (ok ? tid : 0)) * H + h;
-        cp_async4(sbase + sm::GB(b) + 4 * tid, g + off, ok ? 4u : 0u);
-        cp_async4(sbase + sm::GB(b) + 256 + 4 * tid, beta + off, ok ? 4u : 0u);
+    if (tid < 2 * C) {
+        const int r = tid & 63;
+        const bool ok = r < L;
+        const size_t off = (size_t)(cs + (ok ? r : 0)) * H + h;
+        if (tid < C)
+            cp_async4(sbase + sm::GB(b) + 4 * r, g + off, ok ? 4u : 0u);
+        else
+            cp_async4(sbase + sm::GB(b) + 256 + 4 * r, beta + off, ok ? 4u : 0u);
     }
     cp_async_commit();
 }
 
-// T = (I + A)^{-1} for the strictly lower-triangular 64x64 fp32 A (pitch AP):
-// the four diagonal 16x16 blocks by forward substitution (one warp each),
-// then off-diagonal blocks level by level, T_ij = -T_ii sum_{m=j}^{i-1} A_im T_mj.
-__device__ void ut_solve(const float *A, float *T, float *X) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // zero the strictly upper block triangle
-    for (int e = tid; e < 6 * 256; e += NT) {
-        const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
-        const int bi = (b < 3) ? 0 : (b < 5 ? 1 : 2);
-        const int bj = (b < 3) ? b + 1 : (b < 5 ? b - 1 : 3);
-        T[(16 * bi + ri) * AP + 16 * bj + cj] = 0.f;
-    }
-    if (lane < 16) {
-        const int j = lane, o = 16 * warp;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float acc = (i == j) ? 1.f : 0.f;
-#pragma unroll
-            for (int s = 0; s < i; ++s) acc = fmaf(-A[(o + i) * AP + o + s], x[s], acc);
-            x[i] = acc;
-        }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) T[(o + i) * AP + o + j] = x[i];
-    }
-    __syncthreads();
-    for (int lvl = 1; lvl < 4; ++lvl) {
-        const int nb = 4 - lvl;
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
-            const int bi = b + lvl, bj = b;
-            float acc = 0.f;
-            for (int m = bj; m < bi; ++m)
-#pragma unroll
-                for (int s = 0; s < 16; ++s)
-                    acc = fmaf(A[(16 * bi + ri) * AP + 16 * m + s], T[(16 * m + s) * AP + 16 * bj + cj], acc);
-            X[e] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < nb * 256; e += NT) {
-            const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
-            const int bi = b + lvl, bj = b;
-            float acc = 0.f;
-#pragma unroll
-            for (int s = 0; s < 16; ++s) acc = fmaf(T[(16 * bi + ri) * AP + 16 * bi + s], X[b * 256 + s * 16 + cj], acc);
-            T[(16 * bi + ri) * AP + 16 * bj + cj] = -acc;
-        }
-        __syncthreads();
-    }
-}
-
-// All threads agree whether the wait failed (bounded wait on the MMA barrier).
+// All threads agree whether the wait succeeded (bounded wait on the MMA barrier).
 __device__ __forceinline__ bool wait_all_ok(uint64_t *bar, uint32_t parity) {
     const bool ok = tc::mbar_wait(bar, parity);
     tc::fence_after_sync();
@@ -180,7 +142,9 @@ __global__ void __launch_bounds__(NT, 1)
                uint32_t *__restrict__ err) {
     extern __shared__ __align__(1024) uint8_t smem[];
     if (*err & ERRBIT_SEQLENS) return;  // malformed cu_seqlens: write nothing
-    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int row = tid & 127;   // the TMEM lane (accumulator row) this thread reads
+    const int half = tid >> 7;   // which half of the columns it handles
     int t0, t1;
     seq_bounds(cu, n, N, T_tot, t0, t1);
     const uint32_t sb = tc::smem_u32(smem);
@@ -198,23 +162,23 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = *tslot;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lane quarter
     const size_t sidx = ((size_t)n * H + h) * D * D;
 
-    // ---- initial state: thread v owns row v (fp32 in TMEM, bf16 copy in the S tile)
+    // ---- initial state: thread (v, half) owns columns [64 half, 64 half + 64) of row v
     {
-        const float *src = S0 ? S0 + sidx + (size_t)tid * D : nullptr;
+        const float *src = S0 ? S0 + sidx + (size_t)row * D : nullptr;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float r[16];
 #pragma unroll
             for (int i = 0; i < 16; i += 4) {
                 float4 x = src ? *reinterpret_cast<const float4 *>(src + c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
                 r[i] = x.x; r[i + 1] = x.y; r[i + 2] = x.z; r[i + 3] = x.w;
             }
-            tc::tmem_st16(tm + lane_off + TM_S + c0, r);
-            st_run8(sb + sm::S + tc::tile_off(tid, c0, 128, 2048), r);
-            st_run8(sb + sm::S + tc::tile_off(tid, c0 + 8, 128, 2048), r + 8);
+            tc::tmem_st16(tl + TM_S + c0, r);
+            st_run8(sb + sm::S + tc::tile_off(row, c0, 128, 2048), r);
+            st_run8(sb + sm::S + tc::tile_off(row, c0 + 8, 128, 2048), r + 8);
         }
         tc::tmem_st_wait();
     }
@@ -237,22 +201,21 @@ __global__ void __launch_bounds__(NT, 1)
         __syncthreads();
         // ---- G = cumsum(g) in log2 units (warp 0, two positions per lane), gamma, e, beta
         if (warp == 0) {
-            const int l = tid;
-            const float a = graw[2 * l] * kLog2e, b2 = a + graw[2 * l + 1] * kLog2e;
+            const float a = graw[2 * lane] * kLog2e, b2 = a + graw[2 * lane + 1] * kLog2e;
             float sc = b2;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, sc, off);
-                if (l >= off) sc += y;
+                if (lane >= off) sc += y;
             }
             const float base = sc - b2;
-            Gl[2 * l] = base + a;
-            Gl[2 * l + 1] = sc;
+            Gl[2 * lane] = base + a;
+            Gl[2 * lane + 1] = sc;
         }
         __syncthreads();
         if (tid < C) {
-            gam[tid] = exp2f(Gl[tid]);
-            dte[tid] = exp2f(Gl[C - 1] - Gl[tid]);
+            gam[tid] = ex2(Gl[tid]);
+            dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
             bet[tid] = graw[64 + tid];
         }
         // ---- MMA group 1: X1 = [K;Q] K^T and O1 = S Q^T
@@ -273,30 +236,40 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (c + 1 < nchunks) load_chunk(sb, b ^ 1, q, k, v, g, beta, cs + C, min(C, t1 - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
-        // ---- X1 epilogue: rows 0..63 -> A (fp32), rows 64..127 -> P (bf16 tile)
+        // ---- X1 epilogue: rows 0..63 -> A (fp32), rows 64..127 -> P (bf16 tile); columns [32 half, +32)
         {
             float *A = reinterpret_cast<float *>(smem + sm::AF);
-            const int r = tid & 63;
-            const float Gr = Gl[r];
+            const int r = row & 63, s0 = 32 * half;
+            const bool is_a = row < 64;
+            if (r < s0) {  // the whole column range lies above the diagonal (warp-uniform)
+                if (is_a) {
 #pragma unroll
-            for (int c0 = 0; c0 < C; c0 += 16) {
-                float x[16];
-                tc::tmem_ld16(tm + lane_off + TM_XW + c0, x);
-                if (tid < 64) {
+                    for (int i = 0; i < 32; ++i) A[r * AP + s0 + i] = 0.f;
+                } else {
+                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) st_run8(sb + sm::P + tc::tile_off(r, s0 + i, 128, 1024), z);
+                }
+            } else {
+                float x[32];
+                tc::tmem_ld16(tl + TM_XW + s0, *reinterpret_cast<float(*)[16]>(x));
+                tc::tmem_ld16(tl + TM_XW + s0 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+                const float Gr = Gl[r];
+                if (is_a) {
                     const float br = bet[r];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int s = c0 + i;
-                        A[r * AP + s] = (s < r) ? br * exp2f(Gr - Gl[s]) * x[i] : 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = s0 + i;
+                        A[r * AP + s] = (s < r) ? br * ex2(Gr - Gl[s]) * x[i] : 0.f;
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int s = c0 + i;
-                        x[i] = (s <= r) ? exp2f(Gr - Gl[s]) * x[i] : 0.f;
+                    for (int i = 0; i < 32; ++i) {
+                        const int s = s0 + i;
+                        x[i] = (s <= r) ? ex2(Gr - Gl[s]) * x[i] : 0.f;
                     }
-                    st_run8(sb + sm::P + tc::tile_off(r, c0, 128, 1024), x);
-                    st_run8(sb + sm::P + tc::tile_off(r, c0 + 8, 128, 1024), x + 8);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) st_run8(sb + sm::P + tc::tile_off(r, s0 + i, 128, 1024), x + i);
                 }
             }
         }
@@ -306,18 +279,19 @@ __global__ void __launch_bounds__(NT, 1)
         {
             const float *A = reinterpret_cast<const float *>(smem + sm::AF);
             float *T = reinterpret_cast<float *>(smem + sm::TF);
-            ut_solve(A, T, reinterpret_cast<float *>(smem + sm::SCR));
-            const int r = tid & 63;
-            const uint32_t dst = sb + (tid < 64 ? sm::T1 : sm::T2);
+            ut::solve64(A, T, reinterpret_cast<float *>(smem + sm::SCR));
+            const int task = tid & 127, r = task & 63, s0 = 32 * half;
+            const bool t1s = task < 64;
+            const uint32_t dst = sb + (t1s ? sm::T1 : sm::T2);
 #pragma unroll
-            for (int s0 = 0; s0 < C; s0 += 8) {
+            for (int i0 = 0; i0 < 32; i0 += 8) {
                 float x[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int s = s0 + i;
-                    x[i] = T[r * AP + s] * bet[s] * (tid < 64 ? gam[s] : 1.f);
+                    const int s = s0 + i0 + i;
+                    x[i] = T[r * AP + s] * bet[s] * (t1s ? gam[s] : 1.f);
                 }
-                st_run8(dst + tc::tile_off(r, s0, 128, 1024), x);
+                st_run8(dst + tc::tile_off(r, s0 + i0, 128, 1024), x);
             }
         }
         tc::fence_smem_to_async();
@@ -336,13 +310,13 @@ __global__ void __launch_bounds__(NT, 1)
             tc::mma_commit(&bars[1]);
         }
         if (!(ok = wait_all_ok(&bars[1], par))) break;
-        // ---- W epilogue: thread k writes W[., k] as a row of the W tile (runs along r)
+        // ---- W epilogue: thread (k, half) writes W[32 half .. +32][k] as part of row k of the W tile
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
+        for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
             float x[16];
-            tc::tmem_ld16(tm + lane_off + TM_XW + c0, x);
-            st_run8(sb + sm::W + tc::tile_off(tid, c0, 128, 2048), x);
-            st_run8(sb + sm::W + tc::tile_off(tid, c0 + 8, 128, 2048), x + 8);
+            tc::tmem_ld16(tl + TM_XW + c0, x);
+            st_run8(sb + sm::W + tc::tile_off(row, c0, 128, 2048), x);
+            st_run8(sb + sm::W + tc::tile_off(row, c0 + 8, 128, 2048), x + 8);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -359,18 +333,18 @@ __global__ void __launch_bounds__(NT, 1)
         if (!(ok = wait_all_ok(&bars[2], par))) break;
         // ---- Delta epilogue: Delta^T[v][s] = U^T[v][s] - (S W^T)[v][s]; Dl = Delta^T, Dt = Delta^T diag(e)
 #pragma unroll
-        for (int c0 = 0; c0 < C; c0 += 16) {
+        for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
             float u[16], d[16];
-            tc::tmem_ld16(tm + lane_off + TM_U + c0, u);
-            tc::tmem_ld16(tm + lane_off + TM_DD + c0, d);
+            tc::tmem_ld16(tl + TM_U + c0, u);
+            tc::tmem_ld16(tl + TM_DD + c0, d);
 #pragma unroll
             for (int i = 0; i < 16; ++i) u[i] -= d[i];
-            st_run8(sb + sm::DL + tc::tile_off(tid, c0, 128, 2048), u);
-            st_run8(sb + sm::DL + tc::tile_off(tid, c0 + 8, 128, 2048), u + 8);
+            st_run8(sb + sm::DL + tc::tile_off(row, c0, 128, 2048), u);
+            st_run8(sb + sm::DL + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
 #pragma unroll
             for (int i = 0; i < 16; ++i) u[i] *= dte[c0 + i];
-            st_run8(sb + sm::DT + tc::tile_off(tid, c0, 128, 2048), u);
-            st_run8(sb + sm::DT + tc::tile_off(tid, c0 + 8, 128, 2048), u + 8);
+            st_run8(sb + sm::DT + tc::tile_off(row, c0, 128, 2048), u);
+            st_run8(sb + sm::DT + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
@@ -388,32 +362,45 @@ __global__ void __launch_bounds__(NT, 1)
             tc::mma_commit(&bars[3]);
         }
         if (!(ok = wait_all_ok(&bars[3], par))) break;
-        // ---- outputs: o[cs + r][h][v] = gamma_r O1[v][r] + O2[v][r]  (thread v, r < L)
+        // ---- outputs: o[cs + r][h][v] = gamma_r O1[v][r] + O2[v][r], staged as rows o[r][.] in shared memory
         {
-            bf16 *orow = o + ((size_t)cs * H + h) * D + tid;
+            uint8_t *ost = smem + sm::OST;
 #pragma unroll
-            for (int c0 = 0; c0 < C; c0 += 16) {
+            for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
                 float a[16], d[16];
-                tc::tmem_ld16(tm + lane_off + TM_O1 + c0, a);
-                tc::tmem_ld16(tm + lane_off + TM_DD + c0, d);
+                tc::tmem_ld16(tl + TM_O1 + c0, a);
+                tc::tmem_ld16(tl + TM_DD + c0, d);
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
-                    if (c0 + i < L) orow[(size_t)(c0 + i) * H * D] = __float2bfloat16_rn(fmaf(gam[c0 + i], a[i], d[i]));
+                    *reinterpret_cast<bf16 *>(ost + (c0 + i) * 256 + 2 * row) =
+                        __float2bfloat16_rn(fmaf(gam[c0 + i], a[i], d[i]));
+            }
+        }
+        __syncthreads();
+        {
+            const uint8_t *ost = smem + sm::OST;
+#pragma unroll
+            for (int it = 0; it < 4; ++it) {
+                const int idx = it * NT + tid, r = idx >> 4, j = idx & 15;
+                if (r < L) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(ost + r * 256 + j * 16);
+                    *reinterpret_cast<uint4 *>(o + ((size_t)(cs + r) * H + h) * D + 8 * j) = val;
+                }
             }
         }
         // ---- state: S <- gamma_C S + SU (fp32 in TMEM), bf16 copy to the S tile
         {
             const float gC = gam[C - 1];
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
                 float s[16], u[16];
-                tc::tmem_ld16(tm + lane_off + TM_S + c0, s);
-                tc::tmem_ld16(tm + lane_off + TM_SU + c0, u);
+                tc::tmem_ld16(tl + TM_S + c0, s);
+                tc::tmem_ld16(tl + TM_SU + c0, u);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) s[i] = fmaf(gC, s[i], u[i]);
-                tc::tmem_st16(tm + lane_off + TM_S + c0, s);
-                st_run8(sb + sm::S + tc::tile_off(tid, c0, 128, 2048), s);
-                st_run8(sb + sm::S + tc::tile_off(tid, c0 + 8, 128, 2048), s + 8);
+                tc::tmem_st16(tl + TM_S + c0, s);
+                st_run8(sb + sm::S + tc::tile_off(row, c0, 128, 2048), s);
+                st_run8(sb + sm::S + tc::tile_off(row, c0 + 8, 128, 2048), s + 8);
             }
             tc::tmem_st_wait();
         }
@@ -426,11 +413,11 @@ __global__ void __launch_bounds__(NT, 1)
         if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
     } else {
         // ---- final state
-        float *dst = S_T + sidx + (size_t)tid * D;
+        float *dst = S_T + sidx + (size_t)row * D;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 16) {
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float r[16];
-            tc::tmem_ld16(tm + lane_off + TM_S + c0, r);
+            tc::tmem_ld16(tl + TM_S + c0, r);
 #pragma unroll
             for (int i = 0; i < 16; i += 4)
                 *reinterpret_cast<float4 *>(dst + c0 + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
@@ -439,6 +426,15 @@ __global__ void __launch_bounds__(NT, 1)
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+// Diagnostic wrapper of the solve: one 64 x 64 strictly lower fp32 matrix.
+__global__ void __launch_bounds__(NT) k_diag_ut_solve(const float *__restrict__ Ag, float *__restrict__ Tg) {
+    __shared__ float A[64 * AP], T[64 * AP], X[32 * ut::XP];
+    for (int e = threadIdx.x; e < 64 * 64; e += NT) A[(e >> 6) * AP + (e & 63)] = Ag[e];
+    __syncthreads();
+    ut::solve64(A, T, X);
+    for (int e = threadIdx.x; e < 64 * 64; e += NT) Tg[e] = T[(e >> 6) * AP + (e & 63)];
 }
 
 }  // namespace
@@ -452,6 +448,11 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
     if (e != cudaSuccess) return e;
     dim3 grid(H, N);
     k_chunk_tc<<<grid, NT, sm::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_diag_ut_solve(const float *A, float *T, cudaStream_t st) {
+    k_diag_ut_solve<<<1, NT, 0, st>>>(A, T);
     return cudaGetLastError();
 }
 

@@ -4,6 +4,7 @@
 // no-swizzle core-matrix tiles, two stride conventions) and the TMEM
 // accumulator layout against a CPU matmul, independently of the full path.
 #include "common.cuh"
+#include "kernels.h"
 #include "tc.cuh"
 
 namespace gdn {
@@ -88,4 +89,9 @@ extern "C" gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, 
     gdn::k_diag_mma<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16 *>(A), static_cast<const __nv_bfloat16 *>(B), D, M, N, K, a_mn, b_mn, variant);
     return cudaGetLastError() == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+extern "C" gdn_status gdn_diag_ut_solve(const float *A, float *T, void *stream) {
+    if (!A || !T) return GDN_ERR_NULL;
+    return gdn::launch_diag_ut_solve(A, T, static_cast<cudaStream_t>(stream)) == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }

@@ -26,6 +26,8 @@ cudaError_t launch_chunk_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, cons
                             const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
                             __nv_bfloat16 *o, float *S_T, uint32_t *err, cudaStream_t st);
 size_t chunk_tc_smem_bytes();
+// Diagnostic: T = (I + A)^{-1} for one strictly lower 64 x 64 fp32 matrix (row-major, device).
+cudaError_t launch_diag_ut_solve(const float *A, float *T, cudaStream_t st);
 
 // Writes the workspace error word: ERRBIT_SEQLENS if cu_seqlens (device, N+1
 // entries) is not 0 = c0 <= ... <= cN = T_tot, else 0. With cu == NULL it

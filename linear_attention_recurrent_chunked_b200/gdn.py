@@ -33,6 +33,7 @@ SIGNATURES = {
     "gdn_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_seq_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
     "gdn_diag_mma_tile": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
+    "gdn_diag_ut_solve": (_I, [_VP, _VP, _VP]),
     "gdn_chunk_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
     "gdn_profile_enable": (None, [_I]),
     "gdn_profile_read": (_I, [ctypes.c_char_p, _SZ, _VP, _VP, _I]),
@@ -212,3 +213,12 @@ def profile_read() -> dict:
     n = lib.gdn_profile_read(names, 8192, ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(cnt, ctypes.c_void_p), n_max)
     keys = names.value.decode().split("\n")[:n]
     return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(keys)}
+
+
+def diag_ut_solve(A):
+    """Diagnostic: the chunked path's (I + A)^{-1} for one strictly lower 64 x 64 fp32 matrix."""
+    lib = load_library()
+    _need_cuda(A)
+    T = torch.full((64, 64), float("nan"), dtype=torch.float32, device=A.device)
+    _check(lib.gdn_diag_ut_solve(_ptr(A), _ptr(T), _stream()))
+    return T

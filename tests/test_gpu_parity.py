@@ -210,3 +210,23 @@ def test_diag_mma_m64_lane_map():
     with open(os.path.join("gpurun_out", "m64_lane_map.txt"), "w") as f:
         f.write("M=64 accumulator row -> TMEM lane: %s\n" % lanes)
     assert all(x >= 0 for x in lanes), lanes
+
+
+@pytest.mark.parametrize("kind", ["workload", "stress", "ones"])
+def test_diag_ut_solve(kind):
+    """The chunk solve T = (I + A)^{-1} against numpy's inverse (fp64)."""
+    g = torch.Generator().manual_seed(5)
+    if kind == "ones":  # keys all equal, beta = 1, no decay: A = strictly lower ones
+        A = torch.tril(torch.ones(64, 64), -1)
+    else:
+        K = torch.nn.functional.normalize(torch.randn(64, 128, generator=g), dim=-1)
+        beta = torch.sigmoid(torch.randn(64, generator=g) + (3.0 if kind == "stress" else 0.0))
+        gl = -0.01 * torch.rand(64, generator=g) if kind == "stress" else -torch.nn.functional.softplus(
+            torch.randn(64, generator=g))
+        G = torch.cumsum(gl, 0)
+        A = torch.tril(beta[:, None] * torch.exp(G[:, None] - G[None, :]) * (K @ K.T), -1)
+    T = gdn.diag_ut_solve(A.cuda()).cpu().double()
+    ref = np.linalg.inv(np.eye(64) + A.double().numpy())
+    err = float(np.max(np.abs(T.numpy() - ref)) / np.max(np.abs(ref)))
+    assert err < 2e-3, err
+    assert torch.equal(torch.triu(T, 1), torch.zeros(64, 64, dtype=torch.float64))
