@@ -1,7 +1,7 @@
 // Chunked gated delta rule on the sm_100a tensor cores (bf16 inputs, d = 128,
 // chunk C = 64): tcgen05.mma with bf16 operands staged in shared memory and
-// fp32 accumulators in TMEM; the fp32 state lives in TMEM for the whole
-// sequence.
+// fp32 accumulators in TMEM; the fp32 state lives in TMEM while a CTA walks
+// its chunks.
 //
 // The pages give the shape of the method only: the token-by-token scan of
 // the recurrent layers becomes a chunk-wise delta-rule form with an
@@ -21,19 +21,31 @@
 //   S  <- gamma_C S + Dt K          (the state entering the next chunk)
 //
 // Every product is one M = 128 tcgen05.mma group (D = A B^T): accumulator row
-// m sits in TMEM lane m. The CTA has 8 warps; warp w reads TMEM lanes
+// m sits in TMEM lane m. A CTA has 8 warps; warp w reads TMEM lanes
 // 32*(w%4)..+31 and the two warpgroups split the columns, so each thread owns
-// half of one accumulator row (a key row, a position row or a value row of
-// S) and writes it back in whichever shared-memory orientation the next MMA
-// wants. No operand is ever transposed through shared memory: a tile written
-// with 16-byte runs along one axis is read either K-major or MN-major (see
-// tc.cuh). Outputs are staged through shared memory so that the stores to o
-// are whole 256-byte rows.
+// half of one accumulator row and writes it back in whichever shared-memory
+// orientation the next MMA wants. No operand is transposed through shared
+// memory: a tile written with 16-byte runs along one axis is read either
+// K-major or MN-major (see tc.cuh). Outputs are staged through shared memory
+// so that the stores to o are whole 256-byte rows.
 //
-// One CTA per (sequence, head) walks its chunks in order; chunk c+1's K, Q,
-// V, g, beta are fetched with cp.async while chunk c computes. Partial
-// chunks are zero-filled (k = q = v = 0, g = 0, beta = 0), which zeroes their
-// rows of A, W, U, Delta and keeps G flat.
+// Parallelism over time. A sequence's chunks may be split into segments that
+// run concurrently (the host picks the segment length so that the CTAs fill
+// the GPU when there are few (sequence, head) pairs). Per chunk the state
+// map is affine, S -> S M_c + N_c, so over a segment S_end = S_start Phi +
+// S_loc. Pass A (k_chunk_tc_trans) runs every segment but the last of each
+// sequence from S = 0 (giving S_loc) and, on a second set of 128 rows, from
+// X = I with the V-term dropped (giving Phi = X_end); it writes both to the
+// workspace. Pass B (k_chunk_tc) first folds the earlier segments,
+// S <- S Phi_j + S_loc_j starting from S0, then runs its own chunks with
+// outputs; the last segment writes S_T. Without segmentation pass B alone
+// runs, one CTA per (sequence, head).
+//
+// Chunk c+1's K, Q, V, g, beta are fetched with cp.async while chunk c
+// computes. Partial chunks are zero-filled (k = q = v = 0, g = 0, beta = 0),
+// which zeroes their rows of A, W, U, Delta and keeps G flat.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -48,14 +60,16 @@ constexpr int D = 128;    // head size (dk = dv)
 constexpr int NT = 256;   // threads per CTA (two threads per TMEM lane)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int AP = ut::AP;
+constexpr int CP = 132;   // pitch (floats) of the fp32 128 x 128 matrices of the segment fold
 
-// ---- shared memory map (bytes). Tiles use 8x16-byte core matrices with
+// ---- shared memory maps (bytes). Tiles use 8x16-byte core matrices with
 // X-neighbouring core matrices adjacent (sx = 128) and sy = 16 * rows.
-namespace sm {
-// double-buffered chunk inputs, buffer b in {0, 1}
-__device__ __forceinline__ constexpr uint32_t KQ(int b) { return b ? 32768u : 0u; }      // [K rows 0..63; Q rows 64..127] x 128 d, sy = 2048
+// Output pass: K and Q share one tile (K rows 0..63, Q rows 64..127, sy = 2048).
+namespace smo {
+__device__ __forceinline__ constexpr uint32_t KQ(int b) { return b ? 32768u : 0u; }
 __device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 81920u : 65536u; }   // 64 s x 128 d, sy = 1024
-__device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 98816u : 98304u; }  // raw g[64], beta[64] (fp32)
+__device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 98816u : 98304u; }  // raw g[64], beta[64]
+constexpr uint32_t KQ_SY = 2048;
 constexpr uint32_t T1 = 99328;                  // 64 r x 64 s, sy = 1024   (T diag(beta gamma))
 constexpr uint32_t T2 = 107520;                 // 64 r x 64 s               (T diag(beta))
 constexpr uint32_t OST = T1;                    // output staging o[r][v] bf16 (64 x 256 B), over T1+T2
@@ -69,11 +83,33 @@ constexpr uint32_t VEC = UNI + 33280;           // G (log2 units), gamma, e, bet
 constexpr uint32_t BAR = VEC + 1024;            // 4 mbarriers + TMEM slot
 constexpr uint32_t TOTAL = BAR + 64;
 constexpr uint32_t SCR = W;                     // fp32 scratch of the solve (W is free then)
-}  // namespace sm
+constexpr uint32_t FOLD_S = 0, FOLD_PHI = 67584;  // segment fold: two fp32 [128][CP] (before the chunk loop)
+}  // namespace smo
+// Transition pass: no Q, K has its own tile (sy = 1024); a second state (X) tile.
+namespace smt {
+__device__ __forceinline__ constexpr uint32_t K(int b) { return b ? 16384u : 0u; }
+__device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 49152u : 32768u; }
+__device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 66048u : 65536u; }
+constexpr uint32_t K_SY = 1024;
+constexpr uint32_t T1 = 67584;
+constexpr uint32_t T2 = 75776;
+constexpr uint32_t W = 83968;
+constexpr uint32_t S = 100352;                  // bf16 copy of S_loc
+constexpr uint32_t X = 133120;                  // bf16 copy of X
+constexpr uint32_t UNI = 165888;                // {Dt_S, Dt_X} bf16 | {A, T} fp32
+constexpr uint32_t DTS = UNI, DTX = UNI + 16384;
+constexpr uint32_t AF = UNI, TF = UNI + 16640;
+constexpr uint32_t VEC = UNI + 33280;
+constexpr uint32_t BAR = VEC + 1024;
+constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t SCR = W;
+}  // namespace smt
 
-// TMEM columns (512 allocated): fp32 state S, state update, X1 then W^T, U^T,
-// Delta-part then O2, O1.
+// TMEM columns (512 allocated per CTA).
+// Output pass: fp32 state S, state update, X1 then W^T, U^T, Delta-part then O2, O1.
 constexpr uint32_t TM_S = 0, TM_SU = 128, TM_XW = 256, TM_U = 320, TM_DD = 384, TM_O1 = 448;
+// Transition pass: S_loc, X (both updated in place), X1 then W^T, U^T, S W^T, X W^T.
+constexpr uint32_t TT_S = 0, TT_X = 128, TT_XW = 256, TT_U = 320, TT_DS = 384, TT_DX = 448;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -99,11 +135,13 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Issue the cp.async copies of chunk [cs, cs + L) of head h into buffer b.
-__device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q, const bf16 *k, const bf16 *v,
-                                           const float *g, const float *beta, int cs, int L, int H, int h) {
+// Issue the cp.async copies of chunk [cs, cs + L) of head h: K rows into
+// kq (+ tile_off(row, .)), Q rows (if with_q) at rows 64.. of the same tile,
+// V rows into vt, raw g / beta into gb.
+__device__ __forceinline__ void load_chunk(uint32_t kq, uint32_t kq_sy, bool with_q, uint32_t vt, uint32_t gb,
+                                           const bf16 *q, const bf16 *k, const bf16 *v, const float *g,
+                                           const float *beta, int cs, int L, int H, int h) {
     const int tid = threadIdx.x, lane = tid & 31;
-    const uint32_t kq = sbase + sm::KQ(b), vt = sbase + sm::V(b);
 #pragma unroll
     for (int it = 0; it < 4; ++it) {
         const int idx = it * NT + tid;
@@ -112,8 +150,8 @@ __device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q,
         const bool ok = row < L;
         const size_t off = ((size_t)(cs + (ok ? row : 0)) * H + h) * D + 8 * j;
         const uint32_t nb = ok ? 16u : 0u;
-        cp_async16(kq + tc::tile_off(row, 8 * j, 128, 2048), k + off, nb);
-        cp_async16(kq + tc::tile_off(64 + row, 8 * j, 128, 2048), q + off, nb);
+        cp_async16(kq + tc::tile_off(row, 8 * j, 128, kq_sy), k + off, nb);
+        if (with_q) cp_async16(kq + tc::tile_off(64 + row, 8 * j, 128, kq_sy), q + off, nb);
         cp_async16(vt + tc::tile_off(row, 8 * j, 128, 1024), v + off, nb);
     }
     if (tid < 2 * C) {
@@ -121,9 +159,9 @@ __device__ __forceinline__ void load_chunk(uint32_t sbase, int b, const bf16 *q,
         const bool ok = r < L;
         const size_t off = (size_t)(cs + (ok ? r : 0)) * H + h;
         if (tid < C)
-            cp_async4(sbase + sm::GB(b) + 4 * r, g + off, ok ? 4u : 0u);
+            cp_async4(gb + 4 * r, g + off, ok ? 4u : 0u);
         else
-            cp_async4(sbase + sm::GB(b) + 256 + 4 * r, beta + off, ok ? 4u : 0u);
+            cp_async4(gb + 256 + 4 * r, beta + off, ok ? 4u : 0u);
     }
     cp_async_commit();
 }
@@ -135,55 +173,253 @@ __device__ __forceinline__ bool wait_all_ok(uint64_t *bar, uint32_t parity) {
     return __syncthreads_and(ok) != 0;
 }
 
-__global__ void __launch_bounds__(NT, 1)
-    k_chunk_tc(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
-               const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
-               const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o, float *S_T,
-               uint32_t *__restrict__ err) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    if (*err & ERRBIT_SEQLENS) return;  // malformed cu_seqlens: write nothing
-    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int row = tid & 127;   // the TMEM lane (accumulator row) this thread reads
-    const int half = tid >> 7;   // which half of the columns it handles
-    int t0, t1;
-    seq_bounds(cu, n, N, T_tot, t0, t1);
-    const uint32_t sb = tc::smem_u32(smem);
-    float *Gl = reinterpret_cast<float *>(smem + sm::VEC);  // G * log2(e)
-    float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + sm::BAR);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + sm::BAR + 32);
+// G = cumsum(g) in log2 units (warp 0, two positions per lane), then gamma,
+// e = exp(G_C - G) and beta into the vector area. Ends with a barrier between
+// the cumsum and the derived vectors; the caller's next barrier publishes them.
+__device__ __forceinline__ void chunk_scalars(const float *graw, float *Gl, float *gam, float *dte, float *bet) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid < 32) {
+        const float a = graw[2 * lane] * kLog2e, b2 = a + graw[2 * lane + 1] * kLog2e;
+        float sc = b2;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, sc, off);
+            if (lane >= off) sc += y;
+        }
+        Gl[2 * lane] = sc - b2 + a;
+        Gl[2 * lane + 1] = sc;
+    }
+    __syncthreads();
+    if (tid < C) {
+        gam[tid] = ex2(Gl[tid]);
+        dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
+        bet[tid] = graw[64 + tid];
+    }
+}
 
-    if (warp == 0) tc::tmem_alloc(tslot, 512);
-    if (tid == 0) {
+// X1 epilogue: accumulator rows 0..63 -> A (fp32, pitch AP), rows 64..127 ->
+// P (bf16 tile at p_tile, if p_tile != 0); this thread's columns [32 half, +32).
+__device__ __forceinline__ void x1_epilogue(float *A, uint32_t p_tile, uint32_t tl_x1, const float *Gl,
+                                            const float *bet, int row, int half) {
+    const int r = row & 63, s0 = 32 * half;
+    const bool is_a = row < 64;
+    if (!is_a && !p_tile) return;
+    if (r < s0) {  // the whole column range lies above the diagonal (warp-uniform)
+        if (is_a) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) A[r * AP + s0 + i] = 0.f;
+        } else {
+            const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) st_run8(p_tile + tc::tile_off(r, s0 + i, 128, 1024), z);
+        }
+        return;
+    }
+    float x[32];
+    tc::tmem_ld16(tl_x1 + s0, *reinterpret_cast<float(*)[16]>(x));
+    tc::tmem_ld16(tl_x1 + s0 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+    const float Gr = Gl[r];
+    if (is_a) {
+        const float br = bet[r];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int s = s0 + i;
+            A[r * AP + s] = (s < r) ? br * ex2(Gr - Gl[s]) * x[i] : 0.f;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int s = s0 + i;
+            x[i] = (s <= r) ? ex2(Gr - Gl[s]) * x[i] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) st_run8(p_tile + tc::tile_off(r, s0 + i, 128, 1024), x + i);
+    }
+}
+
+// T = (I + A)^{-1}, then T1 = T diag(beta gamma) and T2 = T diag(beta) as bf16 tiles.
+__device__ __forceinline__ void solve_and_scale(const float *A, float *T, float *scratch, uint32_t t1, uint32_t t2,
+                                                const float *gam, const float *bet, int half) {
+    ut::solve64(A, T, scratch);
+    const int task = threadIdx.x & 127, r = task & 63, s0 = 32 * half;
+    const bool first = task < 64;
+    const uint32_t dst = first ? t1 : t2;
+#pragma unroll
+    for (int i0 = 0; i0 < 32; i0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int s = s0 + i0 + i;
+            x[i] = T[r * AP + s] * bet[s] * (first ? gam[s] : 1.f);
+        }
+        st_run8(dst + tc::tile_off(r, s0 + i0, 128, 1024), x);
+    }
+}
+
+// W epilogue: thread (k, half) writes W[32 half .. +32][k] into row k of the W tile (runs along r).
+__device__ __forceinline__ void w_epilogue(uint32_t w_tile, uint32_t tl_w, int row, int half) {
+#pragma unroll
+    for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
+        float x[16];
+        tc::tmem_ld16(tl_w + c0, x);
+        st_run8(w_tile + tc::tile_off(row, c0, 128, 2048), x);
+        st_run8(w_tile + tc::tile_off(row, c0 + 8, 128, 2048), x + 8);
+    }
+}
+
+// Generic-proxy smem writes and TMEM accesses done; make them visible to the tensor core and sync.
+__device__ __forceinline__ void handoff_to_mma() {
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+}
+
+// Segment of global index gseg: sequence n, index s within it, count ns, token range [a, b).
+struct Segment {
+    int n, s, ns, a, b, seq_end;
+};
+__device__ __forceinline__ bool find_segment(const int32_t *seg_off, const int32_t *cu, int N, int T_tot, int gseg,
+                                             int seg_tokens, Segment &sg) {
+    if (!seg_off) {  // one segment per sequence
+        sg.n = gseg;
+        sg.s = 0;
+        sg.ns = 1;
+    } else {
+        if (gseg >= seg_off[N]) return false;
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {  // largest n with seg_off[n] <= gseg
+            const int mid = (lo + hi + 1) >> 1;
+            if (seg_off[mid] <= gseg) lo = mid; else hi = mid - 1;
+        }
+        sg.n = lo;
+        sg.s = gseg - seg_off[lo];
+        sg.ns = seg_off[lo + 1] - seg_off[lo];
+    }
+    int t0, t1;
+    seq_bounds(cu, sg.n, N, T_tot, t0, t1);
+    sg.seq_end = t1;
+    if (sg.ns == 1) {
+        sg.a = t0;
+        sg.b = t1;
+    } else {
+        sg.a = min(t1, t0 + sg.s * seg_tokens);
+        sg.b = min(t1, sg.a + seg_tokens);
+    }
+    return true;
+}
+
+__device__ __forceinline__ void tmem_setup(uint32_t *tslot, uint64_t *bars) {
+    if ((threadIdx.x >> 5) == 0) tc::tmem_alloc(tslot, 512);
+    if (threadIdx.x == 0) {
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tm = *tslot;
-    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lane quarter
-    const size_t sidx = ((size_t)n * H + h) * D * D;
+}
 
-    // ---- initial state: thread (v, half) owns columns [64 half, 64 half + 64) of row v
+// Segment fold (tf32 mma.sync, fp32 accumulation): Ss <- Ss * Phi + S_loc for
+// one workspace slot (S_loc then Phi, fp32 128 x 128 each); Ss and the staged
+// Phi are fp32 [128][CP] in shared memory. Each warp owns 16 rows of Ss (its
+// own A operand rows), so the update is in place.
+__device__ void segment_fold(float *Ss, float *Ph, const float *slot) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int r0 = 16 * warp;
     {
-        const float *src = S0 ? S0 + sidx + (size_t)row * D : nullptr;
+        const float *Sloc = slot;
+        const float *Phi = slot + D * D;
+        for (int e = tid * 4; e < D * D; e += NT * 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(Phi + e);
+            float *dst = Ph + (e >> 7) * CP + (e & 127);
+            dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
+        }
+        __syncthreads();
+        float acc[16][4];
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll 2
+        for (int k = 0; k < D; k += 8) {
+            const uint32_t a[4] = {ut::tf32(Ss[(r0 + g) * CP + k + t]), ut::tf32(Ss[(r0 + g + 8) * CP + k + t]),
+                                   ut::tf32(Ss[(r0 + g) * CP + k + t + 4]), ut::tf32(Ss[(r0 + g + 8) * CP + k + t + 4])};
+#pragma unroll
+            for (int nt = 0; nt < 16; ++nt) {
+                const uint32_t b[2] = {ut::tf32(Ph[(k + t) * CP + 8 * nt + g]), ut::tf32(Ph[(k + t + 4) * CP + 8 * nt + g])};
+                ut::mma_tf32(acc[nt], a, b);
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+            const int c = 8 * nt + 2 * t;
+            const float2 s0 = *reinterpret_cast<const float2 *>(Sloc + (size_t)(r0 + g) * D + c);
+            const float2 s1 = *reinterpret_cast<const float2 *>(Sloc + (size_t)(r0 + g + 8) * D + c);
+            Ss[(r0 + g) * CP + c] = acc[nt][0] + s0.x;
+            Ss[(r0 + g) * CP + c + 1] = acc[nt][1] + s0.y;
+            Ss[(r0 + g + 8) * CP + c] = acc[nt][2] + s1.x;
+            Ss[(r0 + g + 8) * CP + c + 1] = acc[nt][3] + s1.y;
+        }
+        __syncthreads();
+    }
+}
+
+// ============================================================================ output pass
+__global__ void __launch_bounds__(NT, 1)
+    k_chunk_tc(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
+               const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
+               const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o, float *S_T,
+               uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off, int seg_tokens,
+               const float *__restrict__ slots) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;  // malformed cu_seqlens: write nothing
+    Segment sg;
+    const int h = blockIdx.x;
+    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_tokens, sg)) return;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127;   // the TMEM lane (accumulator row) this thread reads
+    const int half = tid >> 7;   // which half of the columns it handles
+    const uint32_t sb = tc::smem_u32(smem);
+    float *Gl = reinterpret_cast<float *>(smem + smo::VEC);  // G * log2(e)
+    float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smo::BAR);
+    tmem_setup(reinterpret_cast<uint32_t *>(smem + smo::BAR + 32), bars);
+    const uint32_t tm = *reinterpret_cast<uint32_t *>(smem + smo::BAR + 32);
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lane quarter
+    const size_t sidx = ((size_t)sg.n * H + h) * D * D;
+
+    // ---- initial state of this segment: S0 (first segment) or the fold of the earlier segments
+    const float *init = S0 ? S0 + sidx : nullptr;
+    int init_pitch = D;
+    if (sg.s > 0) {
+        float *Ss = reinterpret_cast<float *>(smem + smo::FOLD_S);
+        for (int e = tid; e < D * D; e += NT) Ss[(e >> 7) * CP + (e & 127)] = init ? init[e] : 0.f;
+        __syncthreads();
+        // slots are laid out [gseg][h][S_loc, Phi]; segment j of this sequence is gseg = seg_off[n] + j
+        for (int j = 0; j < sg.s; ++j)
+            segment_fold(Ss, reinterpret_cast<float *>(smem + smo::FOLD_PHI),
+                         slots + ((size_t)(seg_off[sg.n] + j) * H + h) * 2 * D * D);
+        init = Ss;
+        init_pitch = CP;
+    }
+    // thread (v, half) owns columns [64 half, 64 half + 64) of row v
+    {
+        const float *src = init ? init + (size_t)row * init_pitch : nullptr;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float r[16];
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-                r[i] = x.x; r[i + 1] = x.y; r[i + 2] = x.z; r[i + 3] = x.w;
-            }
+            for (int i = 0; i < 16; ++i) r[i] = src ? src[c0 + i] : 0.f;
             tc::tmem_st16(tl + TM_S + c0, r);
-            st_run8(sb + sm::S + tc::tile_off(row, c0, 128, 2048), r);
-            st_run8(sb + sm::S + tc::tile_off(row, c0 + 8, 128, 2048), r + 8);
+            st_run8(sb + smo::S + tc::tile_off(row, c0, 128, 2048), r);
+            st_run8(sb + smo::S + tc::tile_off(row, c0 + 8, 128, 2048), r + 8);
         }
         tc::tmem_st_wait();
     }
-    const int nchunks = (t1 - t0 + C - 1) / C;
-    if (nchunks > 0) load_chunk(sb, 0, q, k, v, g, beta, t0, min(C, t1 - t0), H, h);
+    __syncthreads();  // the fold area is reused by the chunk buffers below
+    const int nchunks = (sg.b - sg.a + C - 1) / C;
+    if (nchunks > 0)
+        load_chunk(sb + smo::KQ(0), smo::KQ_SY, true, sb + smo::V(0), sb + smo::GB(0), q, k, v, g, beta, sg.a,
+                   min(C, sg.b - sg.a), H, h);
 
     const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
     const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
@@ -192,32 +428,13 @@ __global__ void __launch_bounds__(NT, 1)
     bool ok = true;
 
     for (int c = 0; c < nchunks; ++c) {
-        const int cs = t0 + c * C, L = min(C, t1 - cs), b = c & 1;
+        const int cs = sg.a + c * C, L = min(C, sg.b - cs), b = c & 1;
         const uint32_t par = (uint32_t)(c & 1);
-        const uint32_t kq = sb + sm::KQ(b), vt = sb + sm::V(b);
-        const float *graw = reinterpret_cast<const float *>(smem + sm::GB(b));
+        const uint32_t kq = sb + smo::KQ(b), vt = sb + smo::V(b);
         cp_async_wait_all();
         tc::fence_smem_to_async();
         __syncthreads();
-        // ---- G = cumsum(g) in log2 units (warp 0, two positions per lane), gamma, e, beta
-        if (warp == 0) {
-            const float a = graw[2 * lane] * kLog2e, b2 = a + graw[2 * lane + 1] * kLog2e;
-            float sc = b2;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, sc, off);
-                if (lane >= off) sc += y;
-            }
-            const float base = sc - b2;
-            Gl[2 * lane] = base + a;
-            Gl[2 * lane + 1] = sc;
-        }
-        __syncthreads();
-        if (tid < C) {
-            gam[tid] = ex2(Gl[tid]);
-            dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
-            bet[tid] = graw[64 + tid];
-        }
+        chunk_scalars(reinterpret_cast<const float *>(smem + smo::GB(b)), Gl, gam, dte, bet);
         // ---- MMA group 1: X1 = [K;Q] K^T and O1 = S Q^T
         if (tid == 0) {
             tc::fence_after_sync();
@@ -228,106 +445,44 @@ __global__ void __launch_bounds__(NT, 1)
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t a = tc::make_desc(sb + sm::S + kk * 4096, 2048, 128);
+                const uint64_t a = tc::make_desc(sb + smo::S + kk * 4096, 2048, 128);
                 const uint64_t bq = tc::make_desc(kq + 1024 + kk * 4096, 2048, 128);
                 tc::mma_bf16(tm + TM_O1, a, bq, id_kk64, kk > 0);
             }
             tc::mma_commit(&bars[0]);
         }
-        if (c + 1 < nchunks) load_chunk(sb, b ^ 1, q, k, v, g, beta, cs + C, min(C, t1 - cs - C), H, h);
+        if (c + 1 < nchunks)
+            load_chunk(sb + smo::KQ(b ^ 1), smo::KQ_SY, true, sb + smo::V(b ^ 1), sb + smo::GB(b ^ 1), q, k, v, g,
+                       beta, cs + C, min(C, sg.b - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
-        // ---- X1 epilogue: rows 0..63 -> A (fp32), rows 64..127 -> P (bf16 tile); columns [32 half, +32)
-        {
-            float *A = reinterpret_cast<float *>(smem + sm::AF);
-            const int r = row & 63, s0 = 32 * half;
-            const bool is_a = row < 64;
-            if (r < s0) {  // the whole column range lies above the diagonal (warp-uniform)
-                if (is_a) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) A[r * AP + s0 + i] = 0.f;
-                } else {
-                    const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) st_run8(sb + sm::P + tc::tile_off(r, s0 + i, 128, 1024), z);
-                }
-            } else {
-                float x[32];
-                tc::tmem_ld16(tl + TM_XW + s0, *reinterpret_cast<float(*)[16]>(x));
-                tc::tmem_ld16(tl + TM_XW + s0 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
-                const float Gr = Gl[r];
-                if (is_a) {
-                    const float br = bet[r];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = s0 + i;
-                        A[r * AP + s] = (s < r) ? br * ex2(Gr - Gl[s]) * x[i] : 0.f;
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = s0 + i;
-                        x[i] = (s <= r) ? ex2(Gr - Gl[s]) * x[i] : 0.f;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) st_run8(sb + sm::P + tc::tile_off(r, s0 + i, 128, 1024), x + i);
-                }
-            }
-        }
+        x1_epilogue(reinterpret_cast<float *>(smem + smo::AF), sb + smo::P, tl + TM_XW, Gl, bet, row, half);
         tc::fence_before_sync();
         __syncthreads();
-        // ---- T = (I + A)^{-1}; T1 = T diag(beta gamma), T2 = T diag(beta) as bf16 tiles
-        {
-            const float *A = reinterpret_cast<const float *>(smem + sm::AF);
-            float *T = reinterpret_cast<float *>(smem + sm::TF);
-            ut::solve64(A, T, reinterpret_cast<float *>(smem + sm::SCR));
-            const int task = tid & 127, r = task & 63, s0 = 32 * half;
-            const bool t1s = task < 64;
-            const uint32_t dst = sb + (t1s ? sm::T1 : sm::T2);
-#pragma unroll
-            for (int i0 = 0; i0 < 32; i0 += 8) {
-                float x[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int s = s0 + i0 + i;
-                    x[i] = T[r * AP + s] * bet[s] * (t1s ? gam[s] : 1.f);
-                }
-                st_run8(dst + tc::tile_off(r, s0 + i0, 128, 1024), x);
-            }
-        }
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        __syncthreads();
+        solve_and_scale(reinterpret_cast<const float *>(smem + smo::AF), reinterpret_cast<float *>(smem + smo::TF),
+                        reinterpret_cast<float *>(smem + smo::SCR), sb + smo::T1, sb + smo::T2, gam, bet, half);
+        handoff_to_mma();
         // ---- MMA group 2: W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views)
         if (tid == 0) {
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
                 tc::mma_bf16(tm + TM_XW, tc::make_desc(kq + kk * 256, 128, 2048),
-                             tc::make_desc(sb + sm::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                             tc::make_desc(sb + smo::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
                 tc::mma_bf16(tm + TM_U, tc::make_desc(vt + kk * 256, 128, 1024),
-                             tc::make_desc(sb + sm::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                             tc::make_desc(sb + smo::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
             }
             tc::mma_commit(&bars[1]);
         }
         if (!(ok = wait_all_ok(&bars[1], par))) break;
-        // ---- W epilogue: thread (k, half) writes W[32 half .. +32][k] as part of row k of the W tile
-#pragma unroll
-        for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
-            float x[16];
-            tc::tmem_ld16(tl + TM_XW + c0, x);
-            st_run8(sb + sm::W + tc::tile_off(row, c0, 128, 2048), x);
-            st_run8(sb + sm::W + tc::tile_off(row, c0 + 8, 128, 2048), x + 8);
-        }
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        __syncthreads();
+        w_epilogue(sb + smo::W, tl + TM_XW, row, half);
+        handoff_to_mma();
         // ---- MMA group 3: S W^T (B operand: MN-major view of the W tile)
         if (tid == 0) {
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk)
-                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + sm::S + kk * 4096, 2048, 128),
-                             tc::make_desc(sb + sm::W + kk * 256, 128, 2048), id_km64, kk > 0);
+                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + smo::S + kk * 4096, 2048, 128),
+                             tc::make_desc(sb + smo::W + kk * 256, 128, 2048), id_km64, kk > 0);
             tc::mma_commit(&bars[2]);
         }
         if (!(ok = wait_all_ok(&bars[2], par))) break;
@@ -339,24 +494,22 @@ __global__ void __launch_bounds__(NT, 1)
             tc::tmem_ld16(tl + TM_DD + c0, d);
 #pragma unroll
             for (int i = 0; i < 16; ++i) u[i] -= d[i];
-            st_run8(sb + sm::DL + tc::tile_off(row, c0, 128, 2048), u);
-            st_run8(sb + sm::DL + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
+            st_run8(sb + smo::DL + tc::tile_off(row, c0, 128, 2048), u);
+            st_run8(sb + smo::DL + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
 #pragma unroll
             for (int i = 0; i < 16; ++i) u[i] *= dte[c0 + i];
-            st_run8(sb + sm::DT + tc::tile_off(row, c0, 128, 2048), u);
-            st_run8(sb + sm::DT + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
+            st_run8(sb + smo::DT + tc::tile_off(row, c0, 128, 2048), u);
+            st_run8(sb + smo::DT + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
         }
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        __syncthreads();
+        handoff_to_mma();
         // ---- MMA group 4: O2 = Dl P^T (into the Delta-part columns), SU = Dt K (B: MN-major view of K)
         if (tid == 0) {
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + sm::DL + kk * 4096, 2048, 128),
-                             tc::make_desc(sb + sm::P + kk * 2048, 1024, 128), id_kk64, kk > 0);
-                tc::mma_bf16(tm + TM_SU, tc::make_desc(sb + sm::DT + kk * 4096, 2048, 128),
+                tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + smo::DL + kk * 4096, 2048, 128),
+                             tc::make_desc(sb + smo::P + kk * 2048, 1024, 128), id_kk64, kk > 0);
+                tc::mma_bf16(tm + TM_SU, tc::make_desc(sb + smo::DT + kk * 4096, 2048, 128),
                              tc::make_desc(kq + kk * 256, 128, 2048), id_km128, kk > 0);
             }
             tc::mma_commit(&bars[3]);
@@ -364,7 +517,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!(ok = wait_all_ok(&bars[3], par))) break;
         // ---- outputs: o[cs + r][h][v] = gamma_r O1[v][r] + O2[v][r], staged as rows o[r][.] in shared memory
         {
-            uint8_t *ost = smem + sm::OST;
+            uint8_t *ost = smem + smo::OST;
 #pragma unroll
             for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
                 float a[16], d[16];
@@ -378,7 +531,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
         __syncthreads();
         {
-            const uint8_t *ost = smem + sm::OST;
+            const uint8_t *ost = smem + smo::OST;
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
                 const int idx = it * NT + tid, r = idx >> 4, j = idx & 15;
@@ -399,20 +552,18 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) s[i] = fmaf(gC, s[i], u[i]);
                 tc::tmem_st16(tl + TM_S + c0, s);
-                st_run8(sb + sm::S + tc::tile_off(row, c0, 128, 2048), s);
-                st_run8(sb + sm::S + tc::tile_off(row, c0 + 8, 128, 2048), s + 8);
+                st_run8(sb + smo::S + tc::tile_off(row, c0, 128, 2048), s);
+                st_run8(sb + smo::S + tc::tile_off(row, c0 + 8, 128, 2048), s + 8);
             }
             tc::tmem_st_wait();
         }
-        tc::fence_smem_to_async();
-        tc::fence_before_sync();
-        __syncthreads();
+        handoff_to_mma();
     }
     cp_async_wait_all();
     if (!ok) {
         if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
-    } else {
-        // ---- final state
+    } else if (sg.s == sg.ns - 1) {
+        // ---- final state (last segment of the sequence)
         float *dst = S_T + sidx + (size_t)row * D;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
@@ -428,6 +579,240 @@ __global__ void __launch_bounds__(NT, 1)
     if (warp == 0) tc::tmem_dealloc(tm, 512);
 }
 
+// ============================================================================ transition pass
+// For every segment except the last of its sequence: S_loc (from S = 0, with
+// the V-term) and Phi (from X = I, without it), written to the workspace slot
+// [gseg][h] as two fp32 128 x 128 matrices.
+__global__ void __launch_bounds__(NT, 1)
+    k_chunk_tc_trans(const bf16 *__restrict__ k, const bf16 *__restrict__ v, const float *__restrict__ g,
+                     const float *__restrict__ beta, const int32_t *__restrict__ cu, int N, int T_tot, int H,
+                     uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off, int seg_tokens,
+                     float *__restrict__ slots) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;
+    Segment sg;
+    const int h = blockIdx.x;
+    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_tokens, sg)) return;
+    if (sg.s == sg.ns - 1) return;  // the last segment's transition is never needed
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127, half = tid >> 7;
+    const uint32_t sb = tc::smem_u32(smem);
+    float *Gl = reinterpret_cast<float *>(smem + smt::VEC);
+    float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smt::BAR);
+    tmem_setup(reinterpret_cast<uint32_t *>(smem + smt::BAR + 32), bars);
+    const uint32_t tm = *reinterpret_cast<uint32_t *>(smem + smt::BAR + 32);
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
+
+    // ---- S_loc = 0, X = I (fp32 in TMEM, bf16 copies in the S / X tiles)
+#pragma unroll 1
+    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+        float z[16], x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            z[i] = 0.f;
+            x[i] = (c0 + i == row) ? 1.f : 0.f;
+        }
+        tc::tmem_st16(tl + TT_S + c0, z);
+        tc::tmem_st16(tl + TT_X + c0, x);
+        st_run8(sb + smt::S + tc::tile_off(row, c0, 128, 2048), z);
+        st_run8(sb + smt::S + tc::tile_off(row, c0 + 8, 128, 2048), z + 8);
+        st_run8(sb + smt::X + tc::tile_off(row, c0, 128, 2048), x);
+        st_run8(sb + smt::X + tc::tile_off(row, c0 + 8, 128, 2048), x + 8);
+    }
+    tc::tmem_st_wait();
+    const int nchunks = (sg.b - sg.a + C - 1) / C;
+    if (nchunks > 0)
+        load_chunk(sb + smt::K(0), smt::K_SY, false, sb + smt::V(0), sb + smt::GB(0), nullptr, k, v, g, beta, sg.a,
+                   min(C, sg.b - sg.a), H, h);
+
+    // X1's A operand covers 128 rows; rows 64..127 read unrelated shared memory
+    // (no Q here) and land in accumulator rows this pass never reads.
+    const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
+    const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+    const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
+    const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+    bool ok = true;
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int cs = sg.a + c * C, b = c & 1;
+        const uint32_t par = (uint32_t)(c & 1);
+        const uint32_t kt = sb + smt::K(b), vt = sb + smt::V(b);
+        cp_async_wait_all();
+        tc::fence_smem_to_async();
+        __syncthreads();
+        chunk_scalars(reinterpret_cast<const float *>(smem + smt::GB(b)), Gl, gam, dte, bet);
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::make_desc(kt + kk * 2048, 1024, 128);
+                tc::mma_bf16(tm + TT_XW, a, a, id_kk64, kk > 0);
+            }
+            tc::mma_commit(&bars[0]);
+        }
+        if (c + 1 < nchunks)
+            load_chunk(sb + smt::K(b ^ 1), smt::K_SY, false, sb + smt::V(b ^ 1), sb + smt::GB(b ^ 1), nullptr, k, v,
+                       g, beta, cs + C, min(C, sg.b - cs - C), H, h);
+        if (!(ok = wait_all_ok(&bars[0], par))) break;
+        x1_epilogue(reinterpret_cast<float *>(smem + smt::AF), 0, tl + TT_XW, Gl, bet, row, half);
+        tc::fence_before_sync();
+        __syncthreads();
+        solve_and_scale(reinterpret_cast<const float *>(smem + smt::AF), reinterpret_cast<float *>(smem + smt::TF),
+                        reinterpret_cast<float *>(smem + smt::SCR), sb + smt::T1, sb + smt::T2, gam, bet, half);
+        handoff_to_mma();
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                tc::mma_bf16(tm + TT_XW, tc::make_desc(kt + kk * 256, 128, 1024),
+                             tc::make_desc(sb + smt::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                tc::mma_bf16(tm + TT_U, tc::make_desc(vt + kk * 256, 128, 1024),
+                             tc::make_desc(sb + smt::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+            }
+            tc::mma_commit(&bars[1]);
+        }
+        if (!(ok = wait_all_ok(&bars[1], par))) break;
+        w_epilogue(sb + smt::W, tl + TT_XW, row, half);
+        handoff_to_mma();
+        // ---- S W^T and X W^T
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t bw = tc::make_desc(sb + smt::W + kk * 256, 128, 2048);
+                tc::mma_bf16(tm + TT_DS, tc::make_desc(sb + smt::S + kk * 4096, 2048, 128), bw, id_km64, kk > 0);
+                tc::mma_bf16(tm + TT_DX, tc::make_desc(sb + smt::X + kk * 4096, 2048, 128), bw, id_km64, kk > 0);
+            }
+            tc::mma_commit(&bars[2]);
+        }
+        if (!(ok = wait_all_ok(&bars[2], par))) break;
+        // ---- Dt_S = (U^T - S W^T) diag(e), Dt_X = -(X W^T) diag(e); states scaled by gamma_C in place
+#pragma unroll
+        for (int c0 = 32 * half; c0 < 32 * half + 32; c0 += 16) {
+            float u[16], d[16];
+            tc::tmem_ld16(tl + TT_U + c0, u);
+            tc::tmem_ld16(tl + TT_DS + c0, d);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) u[i] = (u[i] - d[i]) * dte[c0 + i];
+            st_run8(sb + smt::DTS + tc::tile_off(row, c0, 128, 2048), u);
+            st_run8(sb + smt::DTS + tc::tile_off(row, c0 + 8, 128, 2048), u + 8);
+            tc::tmem_ld16(tl + TT_DX + c0, d);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) d[i] = -d[i] * dte[c0 + i];
+            st_run8(sb + smt::DTX + tc::tile_off(row, c0, 128, 2048), d);
+            st_run8(sb + smt::DTX + tc::tile_off(row, c0 + 8, 128, 2048), d + 8);
+        }
+        {
+            const float gC = gam[C - 1];
+#pragma unroll 1
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+                float s[16], x[16];
+                tc::tmem_ld16(tl + TT_S + c0, s);
+                tc::tmem_ld16(tl + TT_X + c0, x);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    s[i] *= gC;
+                    x[i] *= gC;
+                }
+                tc::tmem_st16(tl + TT_S + c0, s);
+                tc::tmem_st16(tl + TT_X + c0, x);
+            }
+            tc::tmem_st_wait();
+        }
+        handoff_to_mma();
+        // ---- S += Dt_S K, X += Dt_X K (accumulating into the scaled states)
+        if (tid == 0) {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < C / 16; ++kk) {
+                const uint64_t bk = tc::make_desc(kt + kk * 256, 128, 1024);
+                tc::mma_bf16(tm + TT_S, tc::make_desc(sb + smt::DTS + kk * 4096, 2048, 128), bk, id_km128, 1);
+                tc::mma_bf16(tm + TT_X, tc::make_desc(sb + smt::DTX + kk * 4096, 2048, 128), bk, id_km128, 1);
+            }
+            tc::mma_commit(&bars[3]);
+        }
+        if (!(ok = wait_all_ok(&bars[3], par))) break;
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+            float s[16], x[16];
+            tc::tmem_ld16(tl + TT_S + c0, s);
+            tc::tmem_ld16(tl + TT_X + c0, x);
+            st_run8(sb + smt::S + tc::tile_off(row, c0, 128, 2048), s);
+            st_run8(sb + smt::S + tc::tile_off(row, c0 + 8, 128, 2048), s + 8);
+            st_run8(sb + smt::X + tc::tile_off(row, c0, 128, 2048), x);
+            st_run8(sb + smt::X + tc::tile_off(row, c0 + 8, 128, 2048), x + 8);
+        }
+        handoff_to_mma();
+    }
+    cp_async_wait_all();
+    if (!ok) {
+        if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
+    } else {
+        float *slot = slots + ((size_t)blockIdx.y * H + h) * 2 * D * D;
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+            float s[16], x[16];
+            tc::tmem_ld16(tl + TT_S + c0, s);
+            tc::tmem_ld16(tl + TT_X + c0, x);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                *reinterpret_cast<float4 *>(slot + (size_t)row * D + c0 + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
+                *reinterpret_cast<float4 *>(slot + D * D + (size_t)row * D + c0 + i) =
+                    make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+// Segment plan: validates cu_seqlens (error word) and writes seg_off[0..N],
+// the exclusive prefix of max(1, ceil(ceil(L_n / C) / seg_chunks)).
+__global__ void __launch_bounds__(256) k_plan(const int32_t *__restrict__ cu, int N, int T_tot, int seg_chunks,
+                                              uint32_t *__restrict__ err, int32_t *__restrict__ seg_off) {
+    __shared__ int part[256];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = 0;
+    __syncthreads();
+    const int per = (N + 255) / 256;
+    const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
+    auto nseg = [&](int n) {
+        int L = cu ? cu[n + 1] - cu[n] : T_tot / N;
+        L = max(L, 0);
+        const int nc = (L + C - 1) / C;
+        return max(1, (nc + seg_chunks - 1) / seg_chunks);
+    };
+    int sum = 0;
+    bool b = false;
+    for (int n = n0; n < n1; ++n) {
+        if (cu) b |= cu[n + 1] < cu[n];
+        sum += nseg(n);
+    }
+    if (tid == 0 && cu) b |= (cu[0] != 0) || (cu[N] != T_tot);
+    if (b) atomicOr(&bad, 1);
+    part[tid] = sum;
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int i = 0; i < 256; ++i) {
+            const int x = part[i];
+            part[i] = acc;
+            acc += x;
+        }
+        seg_off[N] = acc;
+        *err = bad ? ERRBIT_SEQLENS : 0u;
+    }
+    __syncthreads();
+    int acc = part[tid];
+    for (int n = n0; n < n1; ++n) {
+        seg_off[n] = acc;
+        acc += nseg(n);
+    }
+}
+
 // Diagnostic wrapper of the solve: one 64 x 64 strictly lower fp32 matrix.
 __global__ void __launch_bounds__(NT) k_diag_ut_solve(const float *__restrict__ Ag, float *__restrict__ Tg) {
     __shared__ float A[64 * AP], T[64 * AP], X[32 * ut::XP];
@@ -439,15 +824,78 @@ __global__ void __launch_bounds__(NT) k_diag_ut_solve(const float *__restrict__ 
 
 }  // namespace
 
-size_t chunk_tc_smem_bytes() { return sm::TOTAL; }
+// ---- host side
+int chunk_tc_seg_chunks(int N, int T_tot, int H) {
+    const long pairs = (long)N * H;
+    const long nc_avg = ((long)T_tot / N + C - 1) / C;
+    if (pairs >= 96 || nc_avg < 8) return 0;
+    const long segs = 144 / pairs;
+    if (segs < 2) return 0;
+    return (int)std::max<long>(2, (nc_avg + segs - 1) / segs);
+}
+
+size_t chunk_tc_seg_slots(int N, int T_tot, int seg_chunks) {
+    const long nc_total = ((long)T_tot + C - 1) / C;
+    return (size_t)((nc_total + N) / seg_chunks + N + 1);
+}
+
+size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks) {
+    if (seg_chunks <= 0) return 256;
+    const size_t off = 256 + ((size_t)(N + 1) * 4 + 255) / 256 * 256;
+    return off + chunk_tc_seg_slots(N, T_tot, seg_chunks) * H * 2 * D * D * sizeof(float);
+}
 
 cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
                             const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
-                            uint32_t *err, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm::TOTAL);
+                            void *workspace, size_t ws_bytes, cudaStream_t st, const char **stage) {
+    uint32_t *err = static_cast<uint32_t *>(workspace);
+    // Largest segmentation that fits the workspace (none at all needs only the error word).
+    int seg_chunks = chunk_tc_seg_chunks(N, T_tot, H);
+    while (seg_chunks > 0 && chunk_tc_workspace(N, T_tot, H, seg_chunks) > ws_bytes) {
+        const long nc_avg = ((long)T_tot / N + C - 1) / C;
+        seg_chunks = (seg_chunks * 2 >= nc_avg) ? 0 : seg_chunks * 2;
+    }
+    cudaError_t e;
+    if (seg_chunks == 0) {
+        *stage = "validate_seqlens";
+        void *pv = prof_start("validate_seqlens", st);
+        e = launch_validate_seqlens(cu, N, T_tot, err, st);
+        prof_stop(pv);
+        if (e != cudaSuccess) return e;
+        *stage = "chunk_tc";
+        e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
+        if (e != cudaSuccess) return e;
+        void *pr = prof_start("chunk_tc", st);
+        k_chunk_tc<<<dim3(H, N), NT, smo::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err, nullptr,
+                                                         0, nullptr);
+        prof_stop(pr);
+        return cudaGetLastError();
+    }
+    int32_t *seg_off = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(workspace) + 256);
+    float *slots = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + 256 +
+                                             ((size_t)(N + 1) * 4 + 255) / 256 * 256);
+    const int nslots = (int)chunk_tc_seg_slots(N, T_tot, seg_chunks);
+    const int seg_tokens = seg_chunks * C;
+    *stage = "plan";
+    void *pr = prof_start("plan", st);
+    k_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off);
+    prof_stop(pr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    *stage = "chunk_tc_trans";
+    e = cudaFuncSetAttribute(k_chunk_tc_trans, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smt::TOTAL);
     if (e != cudaSuccess) return e;
-    dim3 grid(H, N);
-    k_chunk_tc<<<grid, NT, sm::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err);
+    pr = prof_start("chunk_tc_trans", st);
+    k_chunk_tc_trans<<<dim3(H, nslots), NT, smt::TOTAL, st>>>(k, v, g, beta, cu, N, T_tot, H, err, seg_off,
+                                                               seg_tokens, slots);
+    prof_stop(pr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    *stage = "chunk_tc";
+    e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
+    if (e != cudaSuccess) return e;
+    pr = prof_start("chunk_tc", st);
+    k_chunk_tc<<<dim3(H, nslots), NT, smo::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err, seg_off,
+                                                         seg_tokens, slots);
+    prof_stop(pr);
     return cudaGetLastError();
 }
 

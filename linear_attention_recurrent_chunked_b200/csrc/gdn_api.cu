@@ -5,6 +5,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -118,6 +119,30 @@ cudaError_t launch_validate_seqlens(const int32_t *cu, int N, int T_tot, uint32_
     return cudaGetLastError();
 }
 
+struct ProfHandle {
+    const char *name;
+    cudaStream_t st;
+    cudaEvent_t start;
+};
+
+void *prof_start(const char *name, cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    if (!g_prof.on) return nullptr;
+    ProfHandle *hd = new ProfHandle{name, st, prof_event()};
+    cudaEventRecord(hd->start, st);
+    return hd;
+}
+
+void prof_stop(void *handle) {
+    if (!handle) return;
+    ProfHandle *hd = static_cast<ProfHandle *>(handle);
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    cudaEvent_t stop = prof_event();
+    cudaEventRecord(stop, hd->st);
+    g_prof.recs.push_back({hd->name, hd->start, stop});
+    delete hd;
+}
+
 // Sets the calling thread's last-error message (for entry points defined in other files).
 gdn_status record_error(gdn_status s, const char *msg) { return fail(s, "%s", msg); }
 
@@ -130,7 +155,8 @@ int gdn_version(void) { return 100; }
 const char *gdn_last_error(void) { return g_msg; }
 
 size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype) {
-    (void)N; (void)T_tot; (void)H; (void)dk; (void)dv; (void)dtype;
+    if (dtype == GDN_BF16 && dk == 128 && dv == 128 && N >= 1 && H >= 1 && T_tot >= 0)
+        return std::max(kErrWordBytes, gdn::chunk_tc_workspace(N, T_tot, H, gdn::chunk_tc_seg_chunks(N, T_tot, H)));
     return kErrWordBytes;
 }
 
@@ -154,20 +180,19 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint32_t *err = static_cast<uint32_t *>(workspace);
     cudaError_t e;
+    if (dtype == GDN_BF16 && dk == 128) {
+        const char *stage = "";
+        e = gdn::launch_chunk_tc(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+                                 static_cast<const __nv_bfloat16 *>(v), g, beta, S0, cu_seqlens, N, T_tot, H,
+                                 static_cast<__nv_bfloat16 *>(o), S_T, workspace, ws_bytes, st, &stage);
+        if (e != cudaSuccess) return cuda_fail(e, stage);
+        return ok();
+    }
     {
         ProfScope ps("validate_seqlens", st);
         e = gdn::launch_validate_seqlens(cu_seqlens, N, T_tot, err, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens validation launch");
-
-    if (dtype == GDN_BF16 && dk == 128) {
-        ProfScope ps("chunk_tc", st);
-        e = gdn::launch_chunk_tc(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
-                                 static_cast<const __nv_bfloat16 *>(v), g, beta, S0, cu_seqlens, N, T_tot, H,
-                                 static_cast<__nv_bfloat16 *>(o), S_T, err, st);
-        if (e != cudaSuccess) return cuda_fail(e, "chunked forward (tensor-core) launch");
-        return ok();
-    }
     ProfScope ps("chunk_simt", st);
     if (dtype == GDN_F32) {
         const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),

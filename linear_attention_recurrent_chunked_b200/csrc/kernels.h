@@ -21,11 +21,23 @@ cudaError_t launch_chunk_simt(const T *q, const T *k, const T *v, const float *g
                               const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, const uint32_t *err,
                               cudaStream_t st);
 
-// Tensor-core chunked forward, bf16 inputs, dk = dv = 128 (one CTA per (sequence, head)).
+// Tensor-core chunked forward, bf16 inputs, dk = dv = 128. Launches the
+// validation / plan, the optional transition pass and the output pass;
+// *stage names the launch that failed when an error is returned. The
+// workspace holds the error word, the segment offsets and the per-segment
+// transition slots (chunk_tc_workspace bytes for the preferred plan; a
+// smaller workspace selects a coarser segmentation or none).
 cudaError_t launch_chunk_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const float *g,
                             const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
-                            __nv_bfloat16 *o, float *S_T, uint32_t *err, cudaStream_t st);
-size_t chunk_tc_smem_bytes();
+                            __nv_bfloat16 *o, float *S_T, void *workspace, size_t ws_bytes, cudaStream_t st,
+                            const char **stage);
+int chunk_tc_seg_chunks(int N, int T_tot, int H);
+size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks);
+
+// Kernel timing hooks (no-ops unless gdn_profile_enable(1)): an event pair
+// around the launches between prof_start and prof_stop, recorded on st.
+void *prof_start(const char *name, cudaStream_t st);
+void prof_stop(void *handle);
 // Diagnostic: T = (I + A)^{-1} for one strictly lower 64 x 64 fp32 matrix (row-major, device).
 cudaError_t launch_diag_ut_solve(const float *A, float *T, cudaStream_t st);
 

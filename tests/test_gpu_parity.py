@@ -230,3 +230,36 @@ def test_diag_ut_solve(kind):
     err = float(np.max(np.abs(T.numpy() - ref)) / np.max(np.abs(ref)))
     assert err < 2e-3, err
     assert torch.equal(torch.triu(T, 1), torch.zeros(64, 64, dtype=torch.float64))
+
+
+# ------------------------------------------------------------------ segment-parallel prefill (few sequence-head pairs)
+
+def test_segmented_varlen_mixed_segment_counts():
+    """Few (sequence, head) pairs: the sequences are split into segments run in
+    parallel (here 6, 1, 12 and 1 segments, one of them an empty sequence)."""
+    w = make_prefill("varlen", seqlens=[700, 100, 1500, 0], H=2, d=128, s0=True, seed=21)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "segmented varlen")
+    assert torch.equal(S_T[3].cpu(), w["S0"][3])
+
+
+def test_segmented_slow_decay_stress():
+    """Segment transitions matter when the state is remembered across segments."""
+    w = make_prefill("prefill_2k", seqlens=[3000], H=1, s0=True, stress=True, seed=22)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "segmented stress")
+
+
+def test_small_workspace_selects_coarser_plan():
+    """A workspace too small for the preferred segmentation gives the same results."""
+    w = make_prefill("prefill_2k", seqlens=[1200], H=2, s0=True, seed=23)
+    dw = to_dev(w)
+    o_big, S_big = chunk(dw)
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")  # error word only: no segmentation
+    o_small, S_small = chunk(dw, workspace=small)
+    assert gdn.chunk_fwd_workspace_size(1, 1200, 2, 128, 128, torch.bfloat16) > 256
+    o_ref, S_ref = run_oracle(w)
+    check(o_small, S_small, o_ref, S_ref, "bf16", "unsegmented")
+    check(o_big, S_big, o_ref, S_ref, "bf16", "segmented")
