@@ -69,10 +69,14 @@ int gdn_version(void);
 const char *gdn_last_error(void);
 
 /*
- * Workspace bytes gdn_chunk_fwd needs for these sizes (0 is never returned:
- * the workspace always holds at least the device error word). The workspace
- * is scratch owned by the caller: its contents on entry are ignored and on
- * exit are meaningless except for the error word read by gdn_chunk_fwd_check.
+ * Workspace bytes with which gdn_chunk_fwd runs its fastest plan for these
+ * sizes (always >= 256). Any workspace of at least 256 bytes (the device
+ * error word) is accepted: when there are few (sequence, head) pairs the
+ * bf16 path splits each sequence into segments that run in parallel and
+ * keeps two fp32 d x d matrices per (segment, head) in the workspace; a
+ * smaller workspace selects fewer segments, down to none. The workspace is
+ * scratch owned by the caller: its contents on entry are ignored and on exit
+ * are meaningless except for the error word read by gdn_chunk_fwd_check.
  * Two calls that overlap on the GPU must not share a workspace.
  */
 size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype);
@@ -94,8 +98,8 @@ size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int
  *             an empty sequence gives S_T = S0 (or 0).
  *   o         [T_tot][H][dv] dtype  (output; must not alias any input)
  *   S_T       [N][H][dv][dk] fp32   (output: state after each sequence)
- *   workspace, ws_bytes: >= gdn_chunk_fwd_workspace_size(...) bytes of device
- *             memory, 256-byte aligned.
+ *   workspace, ws_bytes: device memory, 256-byte aligned, ws_bytes >= 256
+ *             (gdn_chunk_fwd_workspace_size(...) bytes for the fastest plan).
  *
  * A device-side cu_seqlens is validated on the device (the host cannot read
  * it without a synchronisation): if it is malformed, the kernels write
@@ -120,9 +124,12 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
  *
  * Arguments, results and dtype dispatch are those of gdn_chunk_fwd; the
  * workspace comes from an 8 MiB array built into the library, which every
- * GPU that loads the library holds until the process exits. Sizes whose
- * gdn_chunk_fwd_workspace_size exceeds 8 MiB are rejected with
- * GDN_ERR_WORKSPACE. The call allocates nothing. Its first call on a device
+ * GPU that loads the library holds until the process exits. When the sizes'
+ * preferred workspace (gdn_chunk_fwd_workspace_size) exceeds 8 MiB, the
+ * forward runs with the coarser time segmentation that fits in it (the
+ * results are the same up to rounding); GDN_ERR_WORKSPACE is returned only
+ * if the array could not hold gdn_chunk_fwd's 256-byte minimum. The call
+ * allocates nothing. Its first call on a device
  * (with that device current) looks up the array's device address once;
  * make that first call before any stream capture. All calls on a device
  * share the array: calls that overlap on the GPU race and must be

@@ -834,9 +834,12 @@ int chunk_tc_seg_chunks(int N, int T_tot, int H) {
     return (int)std::max<long>(2, (nc_avg + segs - 1) / segs);
 }
 
+// Upper bound of sum_n max(1, ceil(ceil(L_n / C) / seg)) over any lengths with
+// sum L_n = T_tot: each term is at most ceil(L_n / C) / seg + 1, and
+// sum ceil(L_n / C) <= (T_tot + (C - 1) N) / C.
 size_t chunk_tc_seg_slots(int N, int T_tot, int seg_chunks) {
-    const long nc_total = ((long)T_tot + C - 1) / C;
-    return (size_t)((nc_total + N) / seg_chunks + N + 1);
+    const long nc_bound = ((long)T_tot + (long)(C - 1) * N) / C;
+    return (size_t)(nc_bound / seg_chunks + N);
 }
 
 size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks) {

@@ -171,9 +171,9 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
         return fail(GDN_ERR_ALIGN, "S0, S_T and cu_seqlens must be 16-byte aligned");
     if (!cu_seqlens && T_tot % N != 0)
         return fail(GDN_ERR_SEQLENS, "cu_seqlens is NULL and T_tot=%d is not a multiple of N=%d", T_tot, N);
-    const size_t need = gdn_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dtype);
-    if (!workspace || ws_bytes < need)
-        return fail(GDN_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace ? ws_bytes : 0, need);
+    if (!workspace || ws_bytes < kErrWordBytes)
+        return fail(GDN_ERR_WORKSPACE, "workspace of %zu bytes given, at least %zu needed", workspace ? ws_bytes : 0,
+                    kErrWordBytes);
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return fail(GDN_ERR_ALIGN, "workspace must be 256-byte aligned");
 

@@ -9,7 +9,9 @@
 // gdn_chunk_fwd normally receives from the caller comes from here.
 //
 // The scratch is a file-scope __device__ array, so every GPU that loads the
-// library holds kNoallocScratchBytes of it until the process exits. In host
+// library holds kNoallocScratchBytes of it until the process exits. When a
+// call's preferred workspace (gdn_chunk_fwd_workspace_size) is larger than the
+// array, the forward runs with the coarser time segmentation that fits. In host
 // code the array's name is only a host-side stand-in, never a device address:
 // the device address is looked up once per device with cudaGetSymbolAddress
 // (on the first call made while that device is current) and cached. All calls
@@ -28,6 +30,7 @@ gdn_status record_error(gdn_status s, const char *msg);
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(8) << 20;  // 8 MiB per device
+constexpr size_t kMinWorkspaceBytes = 256;                   // gdn_chunk_fwd's minimum (the error word)
 constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
@@ -64,10 +67,12 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const 
                                             const float *beta, const float *S0, const int32_t *cu_seqlens, int N,
                                             int T_tot, int H, int dk, int dv, int dtype, void *o, float *S_T,
                                             void *stream) {
-    const size_t need = gdn_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dtype);
-    if (need > kNoallocScratchBytes)
+    // gdn_chunk_fwd needs at least its 256-byte error word and uses whatever
+    // more it gets to split long sequences into segments; the built-in array
+    // must at least hold that minimum.
+    if (kNoallocScratchBytes < kMinWorkspaceBytes)
         return gdn::record_error(GDN_ERR_WORKSPACE,
-                                 "these sizes need more scratch than the built-in 8 MiB; use gdn_chunk_fwd "
+                                 "the built-in scratch is smaller than the minimum workspace; use gdn_chunk_fwd "
                                  "with a caller-provided workspace");
     void *ws = nullptr;
     const cudaError_t e = scratch_for_current_device(&ws);

@@ -75,6 +75,7 @@ def chunk_args(**over):
     (dict(N=3, T=128), 5),                # equal split impossible
     (dict(ws=None), 6),
     (dict(ws_bytes=8), 6),
+    (dict(ws_bytes=255), 6),
     (dict(ws=ctypes.c_void_p((1 << 20) + 16)), 4),  # workspace must be 256-byte aligned
 ])
 def test_chunk_fwd_rejects_bad_arguments(lib, over, status):

@@ -21,19 +21,23 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-@pytest.mark.parametrize("dtype,d,seqlens", [("bf16", 128, [130, 64, 1, 0]), ("f32", 64, [100, 29])])
-def test_noalloc_matches_workspace_entry_twice(dtype, d, seqlens):
+@pytest.mark.parametrize("dtype,d,seqlens,H", [
+    ("bf16", 128, [130, 64, 1, 0], 3),
+    ("f32", 64, [100, 29], 3),
+    ("bf16", 128, [2048], 16),  # preferred workspace above the 8 MiB array: a coarser plan is used
+])
+def test_noalloc_matches_workspace_entry_twice(dtype, d, seqlens, H):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     lib = gdn.load_library()
     for call, seed in enumerate((11, 12)):  # two calls in a row, different inputs
-        w = make_prefill("varlen", seqlens=seqlens, H=3, d=d, dtype=dtype, s0=True, seed=seed)
+        w = make_prefill("varlen", seqlens=seqlens, H=H, d=d, dtype=dtype, s0=True, seed=seed)
         t = {k: (v.cuda() if hasattr(v, "cuda") else v) for k, v in w.items()}
         o_ref, S_ref = gdn.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], t["cu_seqlens"],
                                      check=True)
         o = torch.full_like(o_ref, float("nan"))
         S_T = torch.full_like(S_ref, float("nan"))
-        N, H = len(seqlens), 3
+        N = len(seqlens)
         st = lib.gdn_chunk_fwd_noalloc(_p(t["q"]), _p(t["k"]), _p(t["v"]), _p(t["g"]), _p(t["beta"]), _p(t["S0"]),
                                        _p(t["cu_seqlens"]), N, w["T_tot"], H, d, d,
                                        1 if dtype == "bf16" else 0, _p(o), _p(S_T),
