@@ -44,7 +44,11 @@
 // Chunk c+1's K, Q, V, g, beta are fetched with cp.async while chunk c
 // computes. Partial chunks are zero-filled (k = q = v = 0, g = 0, beta = 0),
 // which zeroes their rows of A, W, U, Delta and keeps G flat.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -135,24 +139,29 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// Issue the cp.async copies of chunk [cs, cs + L) of head h: K rows into
-// kq (+ tile_off(row, .)), Q rows (if with_q) at rows 64.. of the same tile,
-// V rows into vt, raw g / beta into gb.
+// Fetch chunk [cs, cs + L) of head h into one buffer. K, Q (if with_q) and V
+// arrive by TMA, one 64-row x 16-byte box per 16-byte column run j, which
+// lands exactly as one column of core matrices of the tile (K at
+// kq + j*kq_sy, Q at kq + 1024 + j*kq_sy, V at vt + j*1024); thread 32
+// issues them and arms the buffer's mbarrier with the byte count. Rows past
+// the end of the tensor are zero-filled by TMA; rows past the end of the
+// sequence (the next sequence's tokens in a packed batch) do arrive, and are
+// neutralised by their zero g and beta (below): they only reach rows and
+// columns of A, P, W, U and Delta that are multiplied by beta = 0 or never
+// written out. g and beta come by cp.async (4-byte copies), zero-filled past L.
 __device__ __forceinline__ void load_chunk(uint32_t kq, uint32_t kq_sy, bool with_q, uint32_t vt, uint32_t gb,
-                                           const bf16 *q, const bf16 *k, const bf16 *v, const float *g,
-                                           const float *beta, int cs, int L, int H, int h) {
-    const int tid = threadIdx.x, lane = tid & 31;
-#pragma unroll
-    for (int it = 0; it < 4; ++it) {
-        const int idx = it * NT + tid;
-        const int row = ((idx >> 5) & 7) * 8 + (lane >> 2);
-        const int j = (idx >> 8) * 4 + (lane & 3);  // 16-byte run along d
-        const bool ok = row < L;
-        const size_t off = ((size_t)(cs + (ok ? row : 0)) * H + h) * D + 8 * j;
-        const uint32_t nb = ok ? 16u : 0u;
-        cp_async16(kq + tc::tile_off(row, 8 * j, 128, kq_sy), k + off, nb);
-        if (with_q) cp_async16(kq + tc::tile_off(64 + row, 8 * j, 128, kq_sy), q + off, nb);
-        cp_async16(vt + tc::tile_off(row, 8 * j, 128, 1024), v + off, nb);
+                                           uint64_t *lbar, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                           const CUtensorMap *tm_v, const float *g, const float *beta, int cs,
+                                           int L, int H, int h) {
+    const int tid = threadIdx.x;
+    if (tid == 32) {
+        tc::mbar_arrive_expect_tx(lbar, (with_q ? 3u : 2u) * 16384u);
+#pragma unroll 4
+        for (int j = 0; j < 16; ++j) {
+            tc::tma_load_3d(kq + j * kq_sy, tm_k, lbar, 8 * j, h, cs);
+            if (with_q) tc::tma_load_3d(kq + 1024 + j * kq_sy, tm_q, lbar, 8 * j, h, cs);
+            tc::tma_load_3d(vt + j * 1024, tm_v, lbar, 8 * j, h, cs);
+        }
     }
     if (tid < 2 * C) {
         const int r = tid & 63;
@@ -308,10 +317,13 @@ __device__ __forceinline__ bool find_segment(const int32_t *seg_off, const int32
     return true;
 }
 
+// bars[0..3]: MMA completion; the TMEM slot at byte 32 (bars[4]); bars[5..6]: TMA loads.
 __device__ __forceinline__ void tmem_setup(uint32_t *tslot, uint64_t *bars) {
     if ((threadIdx.x >> 5) == 0) tc::tmem_alloc(tslot, 512);
     if (threadIdx.x == 0) {
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
+        tc::mbar_init(&bars[5], 1);
+        tc::mbar_init(&bars[6], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc::fence_before_sync();
@@ -365,8 +377,9 @@ __device__ void segment_fold(float *Ss, float *Ph, const float *slot) {
 
 // ============================================================================ output pass
 __global__ void __launch_bounds__(NT, 1)
-    k_chunk_tc(const bf16 *__restrict__ q, const bf16 *__restrict__ k, const bf16 *__restrict__ v,
-               const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
+    k_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, const float *__restrict__ beta,
+               const float *S0,
                const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o, float *S_T,
                uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off, int seg_tokens,
                const float *__restrict__ slots) {
@@ -382,6 +395,7 @@ __global__ void __launch_bounds__(NT, 1)
     float *Gl = reinterpret_cast<float *>(smem + smo::VEC);  // G * log2(e)
     float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smo::BAR);
+    uint64_t *lbar = bars + 5;  // one TMA barrier per input buffer
     tmem_setup(reinterpret_cast<uint32_t *>(smem + smo::BAR + 32), bars);
     const uint32_t tm = *reinterpret_cast<uint32_t *>(smem + smo::BAR + 32);
     const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);  // this warp's TMEM lane quarter
@@ -415,11 +429,12 @@ __global__ void __launch_bounds__(NT, 1)
         }
         tc::tmem_st_wait();
     }
-    __syncthreads();  // the fold area is reused by the chunk buffers below
+    tc::fence_smem_to_async();  // the fold area is rewritten by TMA below
+    __syncthreads();
     const int nchunks = (sg.b - sg.a + C - 1) / C;
     if (nchunks > 0)
-        load_chunk(sb + smo::KQ(0), smo::KQ_SY, true, sb + smo::V(0), sb + smo::GB(0), q, k, v, g, beta, sg.a,
-                   min(C, sg.b - sg.a), H, h);
+        load_chunk(sb + smo::KQ(0), smo::KQ_SY, true, sb + smo::V(0), sb + smo::GB(0), &lbar[0], &tm_q, &tm_k,
+                   &tm_v, g, beta, sg.a, min(C, sg.b - sg.a), H, h);
 
     const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
     const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
@@ -435,9 +450,10 @@ __global__ void __launch_bounds__(NT, 1)
         tc::fence_smem_to_async();
         __syncthreads();
         chunk_scalars(reinterpret_cast<const float *>(smem + smo::GB(b)), Gl, gam, dte, bet);
-        // ---- MMA group 1: X1 = [K;Q] K^T and O1 = S Q^T
+        // ---- MMA group 1: X1 = [K;Q] K^T and O1 = S Q^T (after this buffer's TMA bytes landed)
         if (tid == 0) {
             tc::fence_after_sync();
+            if (!tc::mbar_wait(&lbar[b], (uint32_t)((c >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint64_t a = tc::make_desc(kq + kk * 4096, 2048, 128);
@@ -452,8 +468,8 @@ __global__ void __launch_bounds__(NT, 1)
             tc::mma_commit(&bars[0]);
         }
         if (c + 1 < nchunks)
-            load_chunk(sb + smo::KQ(b ^ 1), smo::KQ_SY, true, sb + smo::V(b ^ 1), sb + smo::GB(b ^ 1), q, k, v, g,
-                       beta, cs + C, min(C, sg.b - cs - C), H, h);
+            load_chunk(sb + smo::KQ(b ^ 1), smo::KQ_SY, true, sb + smo::V(b ^ 1), sb + smo::GB(b ^ 1), &lbar[b ^ 1],
+                       &tm_q, &tm_k, &tm_v, g, beta, cs + C, min(C, sg.b - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
         x1_epilogue(reinterpret_cast<float *>(smem + smo::AF), sb + smo::P, tl + TM_XW, Gl, bet, row, half);
         tc::fence_before_sync();
@@ -584,8 +600,9 @@ __global__ void __launch_bounds__(NT, 1)
 // the V-term) and Phi (from X = I, without it), written to the workspace slot
 // [gseg][h] as two fp32 128 x 128 matrices.
 __global__ void __launch_bounds__(NT, 1)
-    k_chunk_tc_trans(const bf16 *__restrict__ k, const bf16 *__restrict__ v, const float *__restrict__ g,
-                     const float *__restrict__ beta, const int32_t *__restrict__ cu, int N, int T_tot, int H,
+    k_chunk_tc_trans(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const float *__restrict__ g, const float *__restrict__ beta, const int32_t *__restrict__ cu,
+                     int N, int T_tot, int H,
                      uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off, int seg_tokens,
                      float *__restrict__ slots) {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -600,6 +617,7 @@ __global__ void __launch_bounds__(NT, 1)
     float *Gl = reinterpret_cast<float *>(smem + smt::VEC);
     float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smt::BAR);
+    uint64_t *lbar = bars + 5;
     tmem_setup(reinterpret_cast<uint32_t *>(smem + smt::BAR + 32), bars);
     const uint32_t tm = *reinterpret_cast<uint32_t *>(smem + smt::BAR + 32);
     const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
@@ -623,8 +641,8 @@ __global__ void __launch_bounds__(NT, 1)
     tc::tmem_st_wait();
     const int nchunks = (sg.b - sg.a + C - 1) / C;
     if (nchunks > 0)
-        load_chunk(sb + smt::K(0), smt::K_SY, false, sb + smt::V(0), sb + smt::GB(0), nullptr, k, v, g, beta, sg.a,
-                   min(C, sg.b - sg.a), H, h);
+        load_chunk(sb + smt::K(0), smt::K_SY, false, sb + smt::V(0), sb + smt::GB(0), &lbar[0], nullptr, &tm_k,
+                   &tm_v, g, beta, sg.a, min(C, sg.b - sg.a), H, h);
 
     // X1's A operand covers 128 rows; rows 64..127 read unrelated shared memory
     // (no Q here) and land in accumulator rows this pass never reads.
@@ -644,6 +662,7 @@ __global__ void __launch_bounds__(NT, 1)
         chunk_scalars(reinterpret_cast<const float *>(smem + smt::GB(b)), Gl, gam, dte, bet);
         if (tid == 0) {
             tc::fence_after_sync();
+            if (!tc::mbar_wait(&lbar[b], (uint32_t)((c >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint64_t a = tc::make_desc(kt + kk * 2048, 1024, 128);
@@ -652,8 +671,8 @@ __global__ void __launch_bounds__(NT, 1)
             tc::mma_commit(&bars[0]);
         }
         if (c + 1 < nchunks)
-            load_chunk(sb + smt::K(b ^ 1), smt::K_SY, false, sb + smt::V(b ^ 1), sb + smt::GB(b ^ 1), nullptr, k, v,
-                       g, beta, cs + C, min(C, sg.b - cs - C), H, h);
+            load_chunk(sb + smt::K(b ^ 1), smt::K_SY, false, sb + smt::V(b ^ 1), sb + smt::GB(b ^ 1), &lbar[b ^ 1],
+                       nullptr, &tm_k, &tm_v, g, beta, cs + C, min(C, sg.b - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
         x1_epilogue(reinterpret_cast<float *>(smem + smt::AF), 0, tl + TT_XW, Gl, bet, row, half);
         tc::fence_before_sync();
@@ -848,17 +867,49 @@ size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks) {
     return off + chunk_tc_seg_slots(N, T_tot, seg_chunks) * H * 2 * D * D * sizeof(float);
 }
 
+namespace {
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+// TMA descriptor of a token-major bf16 tensor [T][H][128]: boxes of 8 elements
+// (16 bytes) x 1 head x 64 tokens; out-of-range tokens read as zero.
+cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T) {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!g_encode) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)std::max(T, 1)};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    const cuuint32_t box[3] = {8, 1, 64};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<bf16 *>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+}  // namespace
+
 cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
                             const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
                             void *workspace, size_t ws_bytes, cudaStream_t st, const char **stage) {
     uint32_t *err = static_cast<uint32_t *>(workspace);
+    CUtensorMap tm_q, tm_k, tm_v;
+    cudaError_t e;
+    *stage = "TMA descriptor encoding";
+    if ((e = make_row_map(&tm_q, q, H, T_tot)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tm_k, k, H, T_tot)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tm_v, v, H, T_tot)) != cudaSuccess) return e;
     // Largest segmentation that fits the workspace (none at all needs only the error word).
     int seg_chunks = chunk_tc_seg_chunks(N, T_tot, H);
     while (seg_chunks > 0 && chunk_tc_workspace(N, T_tot, H, seg_chunks) > ws_bytes) {
         const long nc_avg = ((long)T_tot / N + C - 1) / C;
         seg_chunks = (seg_chunks * 2 >= nc_avg) ? 0 : seg_chunks * 2;
     }
-    cudaError_t e;
     if (seg_chunks == 0) {
         *stage = "validate_seqlens";
         void *pv = prof_start("validate_seqlens", st);
@@ -869,8 +920,8 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
         e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
         if (e != cudaSuccess) return e;
         void *pr = prof_start("chunk_tc", st);
-        k_chunk_tc<<<dim3(H, N), NT, smo::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err, nullptr,
-                                                         0, nullptr);
+        k_chunk_tc<<<dim3(H, N), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
+                                                         nullptr, 0, nullptr);
         prof_stop(pr);
         return cudaGetLastError();
     }
@@ -888,7 +939,7 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
     e = cudaFuncSetAttribute(k_chunk_tc_trans, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smt::TOTAL);
     if (e != cudaSuccess) return e;
     pr = prof_start("chunk_tc_trans", st);
-    k_chunk_tc_trans<<<dim3(H, nslots), NT, smt::TOTAL, st>>>(k, v, g, beta, cu, N, T_tot, H, err, seg_off,
+    k_chunk_tc_trans<<<dim3(H, nslots), NT, smt::TOTAL, st>>>(tm_k, tm_v, g, beta, cu, N, T_tot, H, err, seg_off,
                                                                seg_tokens, slots);
     prof_stop(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -896,8 +947,8 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
     e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
     if (e != cudaSuccess) return e;
     pr = prof_start("chunk_tc", st);
-    k_chunk_tc<<<dim3(H, nslots), NT, smo::TOTAL, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err, seg_off,
-                                                         seg_tokens, slots);
+    k_chunk_tc<<<dim3(H, nslots), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
+                                                         seg_off, seg_tokens, slots);
     prof_stop(pr);
     return cudaGetLastError();
 }

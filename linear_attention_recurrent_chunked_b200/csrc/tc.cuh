@@ -137,6 +137,20 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) 
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// ---- TMA (bulk tensor copies global -> shared, completion counted on an mbarrier) ----
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(mbar)), "r"(bytes)
+                 : "memory");
+}
+// One box of a 3-D tensor map (coordinates innermost first) into shared memory at dst.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint64_t *mbar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(mbar))
+        : "memory");
+}
+
 // TMEM address of (lane, column) relative to the allocation base.
 __device__ __forceinline__ uint32_t taddr(uint32_t base, uint32_t lane, uint32_t col) {
     return base + (lane << 16) + col;
