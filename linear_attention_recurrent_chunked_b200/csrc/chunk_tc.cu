@@ -64,7 +64,6 @@ constexpr int D = 128;    // head size (dk = dv)
 constexpr int NT = 256;   // threads per CTA (two threads per TMEM lane)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int AP = ut::AP;
-constexpr int CP = 132;   // pitch (floats) of the fp32 128 x 128 matrices of the segment fold
 
 // ---- shared memory maps (bytes). Tiles use 8x16-byte core matrices with
 // X-neighbouring core matrices adjacent (sx = 128) and sy = 16 * rows.
@@ -80,14 +79,15 @@ constexpr uint32_t OST = T1;                    // output staging o[r][v] bf16 (
 constexpr uint32_t P = 115712;                  // 64 r x 64 s
 constexpr uint32_t W = 123904;                  // 128 k x 64 r, sy = 2048 (runs along r)
 constexpr uint32_t S = 140288;                  // 128 v x 128 k, sy = 2048 (bf16 copy of the state)
-constexpr uint32_t UNI = 173056;                // union: {Dl, Dt} bf16  |  {A, T} fp32 [64][65]
+constexpr uint32_t UNI = 173056;                // union: {Dl, Dt} bf16  |  {A, T} fp32 [64][AP]
 constexpr uint32_t DL = UNI, DT = UNI + 16384;  // 128 v x 64 s, sy = 2048
-constexpr uint32_t AF = UNI, TF = UNI + 16640;
-constexpr uint32_t VEC = UNI + 33280;           // G (log2 units), gamma, e, beta: 4 x 64 fp32
-constexpr uint32_t BAR = VEC + 1024;            // 4 mbarriers + TMEM slot
-constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t AF = UNI, TF = UNI + 64 * ut::AP * 4;
+constexpr uint32_t VEC = UNI + 2 * 64 * ut::AP * 4;  // G (log2 units), gamma, e, beta: 4 x 64 fp32
+constexpr uint32_t BAR = VEC + 1024;            // mbarriers + TMEM slot (see tmem_setup)
+constexpr uint32_t TOTAL = BAR + 128;
 constexpr uint32_t SCR = W;                     // fp32 scratch of the solve (W is free then)
-constexpr uint32_t FOLD_S = 0, FOLD_PHI = 67584;  // segment fold: two fp32 [128][CP] (before the chunk loop)
+// segment fold (before the chunk loop): two buffers of {Phi_hi, Phi_lo} bf16 tiles; S_hi is the S tile, S_lo sits in UNI
+constexpr uint32_t FOLD_PHI0 = 0, FOLD_PHI1 = 65536, FOLD_SLO = UNI;
 }  // namespace smo
 // Transition pass: no Q, K has its own tile (sy = 1024); a second state (X) tile.
 namespace smt {
@@ -102,10 +102,10 @@ constexpr uint32_t S = 100352;                  // bf16 copy of S_loc
 constexpr uint32_t X = 133120;                  // bf16 copy of X
 constexpr uint32_t UNI = 165888;                // {Dt_S, Dt_X} bf16 | {A, T} fp32
 constexpr uint32_t DTS = UNI, DTX = UNI + 16384;
-constexpr uint32_t AF = UNI, TF = UNI + 16640;
-constexpr uint32_t VEC = UNI + 33280;
+constexpr uint32_t AF = UNI, TF = UNI + 64 * ut::AP * 4;
+constexpr uint32_t VEC = UNI + 2 * 64 * ut::AP * 4;
 constexpr uint32_t BAR = VEC + 1024;
-constexpr uint32_t TOTAL = BAR + 64;
+constexpr uint32_t TOTAL = BAR + 128;
 constexpr uint32_t SCR = W;
 }  // namespace smt
 
@@ -216,7 +216,7 @@ __device__ __forceinline__ void x1_epilogue(float *A, uint32_t p_tile, uint32_t 
     if (r < s0) {  // the whole column range lies above the diagonal (warp-uniform)
         if (is_a) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) A[r * AP + s0 + i] = 0.f;
+            for (int i = 0; i < 32; i += 4) *reinterpret_cast<float4 *>(A + r * AP + s0 + i) = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
             const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -231,9 +231,13 @@ __device__ __forceinline__ void x1_epilogue(float *A, uint32_t p_tile, uint32_t 
     if (is_a) {
         const float br = bet[r];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int s = s0 + i;
-            A[r * AP + s] = (s < r) ? br * ex2(Gr - Gl[s]) * x[i] : 0.f;
+        for (int i = 0; i < 32; i += 4) {
+            float4 a;
+            a.x = (s0 + i < r) ? br * ex2(Gr - Gl[s0 + i]) * x[i] : 0.f;
+            a.y = (s0 + i + 1 < r) ? br * ex2(Gr - Gl[s0 + i + 1]) * x[i + 1] : 0.f;
+            a.z = (s0 + i + 2 < r) ? br * ex2(Gr - Gl[s0 + i + 2]) * x[i + 2] : 0.f;
+            a.w = (s0 + i + 3 < r) ? br * ex2(Gr - Gl[s0 + i + 3]) * x[i + 3] : 0.f;
+            *reinterpret_cast<float4 *>(A + r * AP + s0 + i) = a;
         }
     } else {
 #pragma unroll
@@ -255,11 +259,13 @@ __device__ __forceinline__ void solve_and_scale(const float *A, float *T, float 
     const uint32_t dst = first ? t1 : t2;
 #pragma unroll
     for (int i0 = 0; i0 < 32; i0 += 8) {
-        float x[8];
+        const float4 t0 = *reinterpret_cast<const float4 *>(T + r * AP + s0 + i0);
+        const float4 t1 = *reinterpret_cast<const float4 *>(T + r * AP + s0 + i0 + 4);
+        float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int s = s0 + i0 + i;
-            x[i] = T[r * AP + s] * bet[s] * (first ? gam[s] : 1.f);
+            x[i] *= bet[s] * (first ? gam[s] : 1.f);
         }
         st_run8(dst + tc::tile_off(r, s0 + i0, 128, 1024), x);
     }
@@ -317,13 +323,13 @@ __device__ __forceinline__ bool find_segment(const int32_t *seg_off, const int32
     return true;
 }
 
-// bars[0..3]: MMA completion; the TMEM slot at byte 32 (bars[4]); bars[5..6]: TMA loads.
+// bars[0..3]: MMA completion per chunk; the TMEM slot at byte 32 (bars[4]);
+// bars[5..6]: TMA loads; bars[7]: segment-fold MMAs; bars[8..9]: fold inputs.
 __device__ __forceinline__ void tmem_setup(uint32_t *tslot, uint64_t *bars) {
     if ((threadIdx.x >> 5) == 0) tc::tmem_alloc(tslot, 512);
     if (threadIdx.x == 0) {
         for (int i = 0; i < 4; ++i) tc::mbar_init(&bars[i], 1);
-        tc::mbar_init(&bars[5], 1);
-        tc::mbar_init(&bars[6], 1);
+        for (int i = 5; i < 10; ++i) tc::mbar_init(&bars[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc::fence_before_sync();
@@ -331,48 +337,100 @@ __device__ __forceinline__ void tmem_setup(uint32_t *tslot, uint64_t *bars) {
     tc::fence_after_sync();
 }
 
-// Segment fold (tf32 mma.sync, fp32 accumulation): Ss <- Ss * Phi + S_loc for
-// one workspace slot (S_loc then Phi, fp32 128 x 128 each); Ss and the staged
-// Phi are fp32 [128][CP] in shared memory. Each warp owns 16 rows of Ss (its
-// own A operand rows), so the update is in place.
-__device__ void segment_fold(float *Ss, float *Ph, const float *slot) {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int r0 = 16 * warp;
-    {
-        const float *Sloc = slot;
-        const float *Phi = slot + D * D;
-        for (int e = tid * 4; e < D * D; e += NT * 4) {
-            const float4 x = *reinterpret_cast<const float4 *>(Phi + e);
-            float *dst = Ph + (e >> 7) * CP + (e & 127);
-            dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
+// Split a row run into bf16 hi / lo parts (x = hi + lo + O(2^-16 |x|)) and store both.
+__device__ __forceinline__ void st_run8_split(uint32_t hi_addr, uint32_t lo_addr, const float *x) {
+    float hi[8], lo[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+        lo[i] = x[i] - hi[i];
+    }
+    st_run8(hi_addr, hi);
+    st_run8(lo_addr, lo);
+}
+
+// Segment fold on the tensor cores: S <- S Phi_j + S_loc_j for the sequence's
+// segments j = 0..count-1, starting from S0 (or zero). S and each Phi are
+// split into bf16 hi + lo parts and S Phi = S_hi Phi_hi + S_hi Phi_lo +
+// S_lo Phi_hi (fp32 accumulation in TMEM; the dropped S_lo Phi_lo term is
+// ~2^-16 relative). Phi_hi / Phi_lo arrive as ready-made operand tiles
+// (written by the transition pass) by bulk copy, double-buffered. The
+// result lands as the fp32 state in TMEM (TM_S) and its bf16 copy in the S tile.
+// Returns false (all threads agreeing) if a bounded wait gave up; the error bit is then set in err.
+__device__ bool segment_fold(uint32_t sb, uint32_t tm, uint32_t tl, uint64_t *bars, uint32_t *err,
+                             const float *S0row, const float *slots, size_t slot0, size_t slot_step, int count,
+                             int row, int half) {
+    const int tid = threadIdx.x;
+    const uint32_t shi = sb + smo::S, slo = sb + smo::FOLD_SLO;
+    const uint32_t phbuf[2] = {sb + smo::FOLD_PHI0, sb + smo::FOLD_PHI1};
+    const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+    // S_hi / S_lo from S0 (thread (v, half): columns [64 half, +64) of row v)
+#pragma unroll 1
+    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = S0row ? S0row[c0 + i] : 0.f;
+        st_run8_split(shi + tc::tile_off(row, c0, 128, 2048), slo + tc::tile_off(row, c0, 128, 2048), x);
+    }
+    if (tid == 32) {
+        tc::mbar_arrive_expect_tx(&bars[8], 65536u);
+        tc::bulk_load(phbuf[0], slots + slot0 + D * D, 65536u, &bars[8]);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    for (int j = 0; j < count; ++j) {
+        const int b = j & 1;
+        if (tid == 32 && j + 1 < count) {  // prefetch the next transition's tiles
+            tc::mbar_arrive_expect_tx(&bars[8 + (b ^ 1)], 65536u);
+            tc::bulk_load(phbuf[b ^ 1], slots + slot0 + (j + 1) * slot_step + D * D, 65536u, &bars[8 + (b ^ 1)]);
         }
-        __syncthreads();
-        float acc[16][4];
+        if (tid == 0) {
+            tc::fence_after_sync();
+            if (!tc::mbar_wait(&bars[8 + b], (uint32_t)((j >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-#pragma unroll 2
-        for (int k = 0; k < D; k += 8) {
-            const uint32_t a[4] = {ut::tf32(Ss[(r0 + g) * CP + k + t]), ut::tf32(Ss[(r0 + g + 8) * CP + k + t]),
-                                   ut::tf32(Ss[(r0 + g) * CP + k + t + 4]), ut::tf32(Ss[(r0 + g + 8) * CP + k + t + 4])};
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t ah = tc::make_desc(shi + kk * 4096, 2048, 128);
+                const uint64_t al = tc::make_desc(slo + kk * 4096, 2048, 128);
+                const uint64_t bh = tc::make_desc(phbuf[b] + kk * 256, 128, 2048);
+                const uint64_t bl = tc::make_desc(phbuf[b] + 32768 + kk * 256, 128, 2048);
+                tc::mma_bf16(tm + TM_SU, ah, bh, id_km128, kk > 0);
+                tc::mma_bf16(tm + TM_SU, ah, bl, id_km128, 1);
+                tc::mma_bf16(tm + TM_SU, al, bh, id_km128, 1);
+            }
+            tc::mma_commit(&bars[7]);
+        }
+        if (!wait_all_ok(&bars[7], (uint32_t)(j & 1))) {
+            if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
+            return false;
+        }
+        const float *Sloc = slots + slot0 + j * slot_step + (size_t)row * D;
+        const bool last = j + 1 == count;
+#pragma unroll 1
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+            float d[16];
+            tc::tmem_ld16(tl + TM_SU + c0, d);
 #pragma unroll
-            for (int nt = 0; nt < 16; ++nt) {
-                const uint32_t b[2] = {ut::tf32(Ph[(k + t) * CP + 8 * nt + g]), ut::tf32(Ph[(k + t + 4) * CP + 8 * nt + g])};
-                ut::mma_tf32(acc[nt], a, b);
+            for (int i = 0; i < 16; i += 4) {
+                const float4 sl = *reinterpret_cast<const float4 *>(Sloc + c0 + i);
+                d[i] += sl.x; d[i + 1] += sl.y; d[i + 2] += sl.z; d[i + 3] += sl.w;
+            }
+            if (last) {
+                tc::tmem_st16(tl + TM_S + c0, d);
+                st_run8(shi + tc::tile_off(row, c0, 128, 2048), d);
+                st_run8(shi + tc::tile_off(row, c0 + 8, 128, 2048), d + 8);
+            } else {
+                st_run8_split(shi + tc::tile_off(row, c0, 128, 2048), slo + tc::tile_off(row, c0, 128, 2048), d);
+                st_run8_split(shi + tc::tile_off(row, c0 + 8, 128, 2048), slo + tc::tile_off(row, c0 + 8, 128, 2048),
+                              d + 8);
             }
         }
-        __syncwarp();
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int c = 8 * nt + 2 * t;
-            const float2 s0 = *reinterpret_cast<const float2 *>(Sloc + (size_t)(r0 + g) * D + c);
-            const float2 s1 = *reinterpret_cast<const float2 *>(Sloc + (size_t)(r0 + g + 8) * D + c);
-            Ss[(r0 + g) * CP + c] = acc[nt][0] + s0.x;
-            Ss[(r0 + g) * CP + c + 1] = acc[nt][1] + s0.y;
-            Ss[(r0 + g + 8) * CP + c] = acc[nt][2] + s1.x;
-            Ss[(r0 + g + 8) * CP + c + 1] = acc[nt][3] + s1.y;
-        }
+        tc::tmem_st_wait();
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
         __syncthreads();
     }
+    return true;
 }
 
 // ============================================================================ output pass
@@ -402,37 +460,33 @@ __global__ void __launch_bounds__(NT, 1)
     const size_t sidx = ((size_t)sg.n * H + h) * D * D;
 
     // ---- initial state of this segment: S0 (first segment) or the fold of the earlier segments
-    const float *init = S0 ? S0 + sidx : nullptr;
-    int init_pitch = D;
+    bool ok = true;
     if (sg.s > 0) {
-        float *Ss = reinterpret_cast<float *>(smem + smo::FOLD_S);
-        for (int e = tid; e < D * D; e += NT) Ss[(e >> 7) * CP + (e & 127)] = init ? init[e] : 0.f;
-        __syncthreads();
-        // slots are laid out [gseg][h][S_loc, Phi]; segment j of this sequence is gseg = seg_off[n] + j
-        for (int j = 0; j < sg.s; ++j)
-            segment_fold(Ss, reinterpret_cast<float *>(smem + smo::FOLD_PHI),
-                         slots + ((size_t)(seg_off[sg.n] + j) * H + h) * 2 * D * D);
-        init = Ss;
-        init_pitch = CP;
-    }
-    // thread (v, half) owns columns [64 half, 64 half + 64) of row v
-    {
-        const float *src = init ? init + (size_t)row * init_pitch : nullptr;
+        // slots are laid out [gseg][h][S_loc fp32, Phi_hi tile, Phi_lo tile]; segment j of this sequence is gseg = seg_off[n] + j
+        ok = segment_fold(sb, tm, tl, bars, err, S0 ? S0 + sidx + (size_t)row * D : nullptr, slots,
+                          ((size_t)seg_off[sg.n] * H + h) * 2 * D * D, (size_t)H * 2 * D * D, sg.s, row, half);
+    } else {
+        // thread (v, half) owns columns [64 half, 64 half + 64) of row v
+        const float *src = S0 ? S0 + sidx + (size_t)row * D : nullptr;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float r[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = src ? src[c0 + i] : 0.f;
+            for (int i = 0; i < 16; i += 4) {
+                const float4 x = src ? *reinterpret_cast<const float4 *>(src + c0 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                r[i] = x.x; r[i + 1] = x.y; r[i + 2] = x.z; r[i + 3] = x.w;
+            }
             tc::tmem_st16(tl + TM_S + c0, r);
             st_run8(sb + smo::S + tc::tile_off(row, c0, 128, 2048), r);
             st_run8(sb + smo::S + tc::tile_off(row, c0 + 8, 128, 2048), r + 8);
         }
         tc::tmem_st_wait();
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        __syncthreads();
     }
-    tc::fence_smem_to_async();  // the fold area is rewritten by TMA below
-    __syncthreads();
     const int nchunks = (sg.b - sg.a + C - 1) / C;
-    if (nchunks > 0)
+    if (ok && nchunks > 0)
         load_chunk(sb + smo::KQ(0), smo::KQ_SY, true, sb + smo::V(0), sb + smo::GB(0), &lbar[0], &tm_q, &tm_k,
                    &tm_v, g, beta, sg.a, min(C, sg.b - sg.a), H, h);
 
@@ -440,9 +494,8 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
     const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
     const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
-    bool ok = true;
 
-    for (int c = 0; c < nchunks; ++c) {
+    for (int c = 0; ok && c < nchunks; ++c) {
         const int cs = sg.a + c * C, L = min(C, sg.b - cs), b = c & 1;
         const uint32_t par = (uint32_t)(c & 1);
         const uint32_t kq = sb + smo::KQ(b), vt = sb + smo::V(b);
@@ -768,17 +821,32 @@ __global__ void __launch_bounds__(NT, 1)
     if (!ok) {
         if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
     } else {
+        // slot: S_loc (fp32 row-major), then Phi as bf16 hi and lo operand tiles
+        // (rows k, 16-byte runs along k', sx = 128, sy = 2048), byte for byte the
+        // shared-memory layout the output pass's fold reads them in.
         float *slot = slots + ((size_t)blockIdx.y * H + h) * 2 * D * D;
+        uint8_t *phi_hi = reinterpret_cast<uint8_t *>(slot + D * D), *phi_lo = phi_hi + 32768;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
             float s[16], x[16];
             tc::tmem_ld16(tl + TT_S + c0, s);
             tc::tmem_ld16(tl + TT_X + c0, x);
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
+            for (int i = 0; i < 16; i += 4)
                 *reinterpret_cast<float4 *>(slot + (size_t)row * D + c0 + i) = make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
-                *reinterpret_cast<float4 *>(slot + D * D + (size_t)row * D + c0 + i) =
-                    make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+#pragma unroll
+            for (int r8 = 0; r8 < 16; r8 += 8) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) {
+                    const float h0 = __bfloat162float(__float2bfloat16_rn(x[r8 + i]));
+                    const float h1 = __bfloat162float(__float2bfloat16_rn(x[r8 + i + 1]));
+                    hi[i / 2] = tc::pack_bf16x2(h0, h1);
+                    lo[i / 2] = tc::pack_bf16x2(x[r8 + i] - h0, x[r8 + i + 1] - h1);
+                }
+                const uint32_t off = tc::tile_off(row, c0 + r8, 128, 2048);
+                *reinterpret_cast<uint4 *>(phi_hi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(phi_lo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
         }
     }

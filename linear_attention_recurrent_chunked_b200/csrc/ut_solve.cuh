@@ -22,7 +22,8 @@
 namespace gdn {
 namespace ut {
 
-constexpr int AP = 65;   // pitch of A and T (odd: row-parallel accesses hit distinct banks)
+constexpr int AP = 68;   // pitch of A and T: rows 16-byte aligned; 8 consecutive rows' 16-byte chunks and the
+                         // mma fragment patterns (4 g + t) hit distinct banks
 constexpr int XP = 40;   // pitch of the product scratch
 
 __device__ __forceinline__ uint32_t tf32(float x) {
