@@ -188,9 +188,11 @@ gdn_status gdn_seq_scan(const void *q, const void *k, const void *v,
  *   D [128][N] fp32 (device): every TMEM lane is dumped, so for M = 64 the
  *     rows the hardware leaves unused are visible as well.
  *   a_mn / b_mn: 1 = stage that operand as an MN-major tile, 0 = K-major.
- *   variant: 0 or 1, the two core-matrix stride conventions of the kernels.
+ *   variant: 0 or 1, the two no-swizzle core-matrix stride conventions of
+ *     the kernels; 2, the 128-byte-swizzled tiles that TMA writes.
  * Limits: M in {64, 128}; 16 <= N <= 256 (multiple of 16 for M = 128, of 8
- * for M = 64); 16 <= K <= 128, multiple of 16. Launches one CTA on `stream`.
+ * for M = 64; N <= 128 for variant 2); 16 <= K <= 128, multiple of 16.
+ * Launches one CTA on `stream`.
  */
 gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, int M, int N, int K,
                              int a_mn, int b_mn, int variant, void *stream);

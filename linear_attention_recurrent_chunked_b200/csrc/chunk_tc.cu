@@ -67,12 +67,12 @@ constexpr int AP = ut::AP;
 
 // ---- shared memory maps (bytes). Tiles use 8x16-byte core matrices with
 // X-neighbouring core matrices adjacent (sx = 128) and sy = 16 * rows.
-// Output pass: K and Q share one tile (K rows 0..63, Q rows 64..127, sy = 2048).
+// Output pass: K and Q share one buffer ([K;Q] is one 128-row operand per column half).
 namespace smo {
 __device__ __forceinline__ constexpr uint32_t KQ(int b) { return b ? 32768u : 0u; }
-__device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 81920u : 65536u; }   // 64 s x 128 d, sy = 1024
+__device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 81920u : 65536u; }   // [V_lo | V_hi], 128-byte swizzled
 __device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 98816u : 98304u; }  // raw g[64], beta[64]
-constexpr uint32_t KQ_SY = 2048;
+constexpr uint32_t KQ_HALF = 16384;  // [K_lo | Q_lo | K_hi | Q_hi], 8 KB each, 128-byte swizzled
 constexpr uint32_t T1 = 99328;                  // 64 r x 64 s, sy = 1024   (T diag(beta gamma))
 constexpr uint32_t T2 = 107520;                 // 64 r x 64 s               (T diag(beta))
 constexpr uint32_t OST = T1;                    // output staging o[r][v] bf16 (64 x 256 B), over T1+T2
@@ -89,12 +89,12 @@ constexpr uint32_t SCR = W;                     // fp32 scratch of the solve (W 
 // segment fold (before the chunk loop): two buffers of {Phi_hi, Phi_lo} bf16 tiles; S_hi is the S tile, S_lo sits in UNI
 constexpr uint32_t FOLD_PHI0 = 0, FOLD_PHI1 = 65536, FOLD_SLO = UNI;
 }  // namespace smo
-// Transition pass: no Q, K has its own tile (sy = 1024); a second state (X) tile.
+// Transition pass: no Q; a second state (X) tile.
 namespace smt {
 __device__ __forceinline__ constexpr uint32_t K(int b) { return b ? 16384u : 0u; }
 __device__ __forceinline__ constexpr uint32_t V(int b) { return b ? 49152u : 32768u; }
 __device__ __forceinline__ constexpr uint32_t GB(int b) { return b ? 66048u : 65536u; }
-constexpr uint32_t K_SY = 1024;
+constexpr uint32_t K_HALF = 8192;    // [K_lo | K_hi], 128-byte swizzled
 constexpr uint32_t T1 = 67584;
 constexpr uint32_t T2 = 75776;
 constexpr uint32_t W = 83968;
@@ -140,27 +140,28 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // Fetch chunk [cs, cs + L) of head h into one buffer. K, Q (if with_q) and V
-// arrive by TMA, one 64-row x 16-byte box per 16-byte column run j, which
-// lands exactly as one column of core matrices of the tile (K at
-// kq + j*kq_sy, Q at kq + 1024 + j*kq_sy, V at vt + j*1024); thread 32
-// issues them and arms the buffer's mbarrier with the byte count. Rows past
-// the end of the tensor are zero-filled by TMA; rows past the end of the
-// sequence (the next sequence's tokens in a packed batch) do arrive, and are
-// neutralised by their zero g and beta (below): they only reach rows and
-// columns of A, P, W, U and Delta that are multiplied by beta = 0 or never
-// written out. g and beta come by cp.async (4-byte copies), zero-filled past L.
-__device__ __forceinline__ void load_chunk(uint32_t kq, uint32_t kq_sy, bool with_q, uint32_t vt, uint32_t gb,
+// arrive by TMA as 128-byte-swizzled tiles (SWIZZLE_128B boxes of 64 tokens x
+// 64 columns), two column halves per matrix: K halves at kq and kq + k_half,
+// Q halves 8 KB after each K half (so that [K; Q] forms one 128-row operand
+// per column half), V halves at vt and vt + 8192. Thread 32 issues them and
+// arms the buffer's mbarrier with the byte count. Rows past the end of the
+// tensor are zero-filled by TMA; rows past the end of the sequence (the next
+// sequence's tokens in a packed batch) do arrive, and are neutralised by
+// their zero g and beta (below): they only reach rows and columns of A, P,
+// W, U and Delta that are multiplied by beta = 0 or never written out.
+// g and beta come by cp.async (4-byte copies), zero-filled past L.
+__device__ __forceinline__ void load_chunk(uint32_t kq, uint32_t k_half, bool with_q, uint32_t vt, uint32_t gb,
                                            uint64_t *lbar, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                            const CUtensorMap *tm_v, const float *g, const float *beta, int cs,
                                            int L, int H, int h) {
     const int tid = threadIdx.x;
     if (tid == 32) {
-        tc::mbar_arrive_expect_tx(lbar, (with_q ? 3u : 2u) * 16384u);
-#pragma unroll 4
-        for (int j = 0; j < 16; ++j) {
-            tc::tma_load_3d(kq + j * kq_sy, tm_k, lbar, 8 * j, h, cs);
-            if (with_q) tc::tma_load_3d(kq + 1024 + j * kq_sy, tm_q, lbar, 8 * j, h, cs);
-            tc::tma_load_3d(vt + j * 1024, tm_v, lbar, 8 * j, h, cs);
+        tc::mbar_arrive_expect_tx(lbar, (with_q ? 6u : 4u) * 8192u);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            tc::tma_load_3d(kq + hf * k_half, tm_k, lbar, 64 * hf, h, cs);
+            if (with_q) tc::tma_load_3d(kq + hf * k_half + 8192, tm_q, lbar, 64 * hf, h, cs);
+            tc::tma_load_3d(vt + hf * 8192, tm_v, lbar, 64 * hf, h, cs);
         }
     }
     if (tid < 2 * C) {
@@ -400,20 +401,28 @@ __device__ bool segment_fold(uint32_t sb, uint32_t tm, uint32_t tl, uint64_t *ba
             }
             tc::mma_commit(&bars[7]);
         }
+        // this thread's half row of S_loc, fetched while the MMAs run
+        float4 sl[16];
+        {
+            const float4 *Sloc = reinterpret_cast<const float4 *>(slots + slot0 + j * slot_step + (size_t)row * D +
+                                                                  64 * half);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sl[i] = Sloc[i];
+        }
         if (!wait_all_ok(&bars[7], (uint32_t)(j & 1))) {
             if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
             return false;
         }
-        const float *Sloc = slots + slot0 + j * slot_step + (size_t)row * D;
         const bool last = j + 1 == count;
-#pragma unroll 1
-        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+            const int c0 = 64 * half + 16 * blk;
             float d[16];
             tc::tmem_ld16(tl + TM_SU + c0, d);
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                const float4 sl = *reinterpret_cast<const float4 *>(Sloc + c0 + i);
-                d[i] += sl.x; d[i + 1] += sl.y; d[i + 2] += sl.z; d[i + 3] += sl.w;
+            for (int i = 0; i < 4; ++i) {
+                d[4 * i] += sl[4 * blk + i].x; d[4 * i + 1] += sl[4 * blk + i].y;
+                d[4 * i + 2] += sl[4 * blk + i].z; d[4 * i + 3] += sl[4 * blk + i].w;
             }
             if (last) {
                 tc::tmem_st16(tl + TM_S + c0, d);
@@ -450,6 +459,10 @@ __global__ void __launch_bounds__(NT, 1)
     const int row = tid & 127;   // the TMEM lane (accumulator row) this thread reads
     const int half = tid >> 7;   // which half of the columns it handles
     const uint32_t sb = tc::smem_u32(smem);
+    if (sb & 1023u) {  // swizzled tiles need a 1024-byte aligned shared-memory base
+        if (threadIdx.x == 0) atomicOr(err, ERRBIT_INTERNAL);
+        return;
+    }
     float *Gl = reinterpret_cast<float *>(smem + smo::VEC);  // G * log2(e)
     float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smo::BAR);
@@ -487,7 +500,7 @@ __global__ void __launch_bounds__(NT, 1)
     }
     const int nchunks = (sg.b - sg.a + C - 1) / C;
     if (ok && nchunks > 0)
-        load_chunk(sb + smo::KQ(0), smo::KQ_SY, true, sb + smo::V(0), sb + smo::GB(0), &lbar[0], &tm_q, &tm_k,
+        load_chunk(sb + smo::KQ(0), smo::KQ_HALF, true, sb + smo::V(0), sb + smo::GB(0), &lbar[0], &tm_q, &tm_k,
                    &tm_v, g, beta, sg.a, min(C, sg.b - sg.a), H, h);
 
     const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
@@ -507,21 +520,24 @@ __global__ void __launch_bounds__(NT, 1)
         if (tid == 0) {
             tc::fence_after_sync();
             if (!tc::mbar_wait(&lbar[b], (uint32_t)((c >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
+            // swizzled K-major: a K=16 step is 32 bytes within the 128-byte row; columns 64.. in the next half
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t a = tc::make_desc(kq + kk * 4096, 2048, 128);
-                tc::mma_bf16(tm + TM_XW, a, a, id_kk64, kk > 0);  // B = first 64 rows of the same tile (K)
+                const uint32_t off = (kk >> 2) * smo::KQ_HALF + (kk & 3) * 32;
+                const uint64_t a = tc::make_desc_sw128(kq + off, 16, 1024);
+                tc::mma_bf16(tm + TM_XW, a, a, id_kk64, kk > 0);  // B = first 64 rows of the same operand (K)
             }
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint64_t a = tc::make_desc(sb + smo::S + kk * 4096, 2048, 128);
-                const uint64_t bq = tc::make_desc(kq + 1024 + kk * 4096, 2048, 128);
+                const uint64_t bq =
+                    tc::make_desc_sw128(kq + (kk >> 2) * smo::KQ_HALF + (kk & 3) * 32 + 8192, 16, 1024);
                 tc::mma_bf16(tm + TM_O1, a, bq, id_kk64, kk > 0);
             }
             tc::mma_commit(&bars[0]);
         }
         if (c + 1 < nchunks)
-            load_chunk(sb + smo::KQ(b ^ 1), smo::KQ_SY, true, sb + smo::V(b ^ 1), sb + smo::GB(b ^ 1), &lbar[b ^ 1],
+            load_chunk(sb + smo::KQ(b ^ 1), smo::KQ_HALF, true, sb + smo::V(b ^ 1), sb + smo::GB(b ^ 1), &lbar[b ^ 1],
                        &tm_q, &tm_k, &tm_v, g, beta, cs + C, min(C, sg.b - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
         x1_epilogue(reinterpret_cast<float *>(smem + smo::AF), sb + smo::P, tl + TM_XW, Gl, bet, row, half);
@@ -535,9 +551,10 @@ __global__ void __launch_bounds__(NT, 1)
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                tc::mma_bf16(tm + TM_XW, tc::make_desc(kq + kk * 256, 128, 2048),
+                // swizzled MN-major views: 16 token rows = 2048 bytes; LBO = distance of the column halves
+                tc::mma_bf16(tm + TM_XW, tc::make_desc_sw128(kq + kk * 2048, smo::KQ_HALF, 1024),
                              tc::make_desc(sb + smo::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                tc::mma_bf16(tm + TM_U, tc::make_desc(vt + kk * 256, 128, 1024),
+                tc::mma_bf16(tm + TM_U, tc::make_desc_sw128(vt + kk * 2048, 8192, 1024),
                              tc::make_desc(sb + smo::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
             }
             tc::mma_commit(&bars[1]);
@@ -579,7 +596,7 @@ __global__ void __launch_bounds__(NT, 1)
                 tc::mma_bf16(tm + TM_DD, tc::make_desc(sb + smo::DL + kk * 4096, 2048, 128),
                              tc::make_desc(sb + smo::P + kk * 2048, 1024, 128), id_kk64, kk > 0);
                 tc::mma_bf16(tm + TM_SU, tc::make_desc(sb + smo::DT + kk * 4096, 2048, 128),
-                             tc::make_desc(kq + kk * 256, 128, 2048), id_km128, kk > 0);
+                             tc::make_desc_sw128(kq + kk * 2048, smo::KQ_HALF, 1024), id_km128, kk > 0);
             }
             tc::mma_commit(&bars[3]);
         }
@@ -667,6 +684,10 @@ __global__ void __launch_bounds__(NT, 1)
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, half = tid >> 7;
     const uint32_t sb = tc::smem_u32(smem);
+    if (sb & 1023u) {
+        if (threadIdx.x == 0) atomicOr(err, ERRBIT_INTERNAL);
+        return;
+    }
     float *Gl = reinterpret_cast<float *>(smem + smt::VEC);
     float *gam = Gl + 64, *dte = Gl + 128, *bet = Gl + 192;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + smt::BAR);
@@ -694,7 +715,7 @@ __global__ void __launch_bounds__(NT, 1)
     tc::tmem_st_wait();
     const int nchunks = (sg.b - sg.a + C - 1) / C;
     if (nchunks > 0)
-        load_chunk(sb + smt::K(0), smt::K_SY, false, sb + smt::V(0), sb + smt::GB(0), &lbar[0], nullptr, &tm_k,
+        load_chunk(sb + smt::K(0), smt::K_HALF, false, sb + smt::V(0), sb + smt::GB(0), &lbar[0], nullptr, &tm_k,
                    &tm_v, g, beta, sg.a, min(C, sg.b - sg.a), H, h);
 
     // X1's A operand covers 128 rows; rows 64..127 read unrelated shared memory
@@ -718,13 +739,13 @@ __global__ void __launch_bounds__(NT, 1)
             if (!tc::mbar_wait(&lbar[b], (uint32_t)((c >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t a = tc::make_desc(kt + kk * 2048, 1024, 128);
+                const uint64_t a = tc::make_desc_sw128(kt + (kk >> 2) * smt::K_HALF + (kk & 3) * 32, 16, 1024);
                 tc::mma_bf16(tm + TT_XW, a, a, id_kk64, kk > 0);
             }
             tc::mma_commit(&bars[0]);
         }
         if (c + 1 < nchunks)
-            load_chunk(sb + smt::K(b ^ 1), smt::K_SY, false, sb + smt::V(b ^ 1), sb + smt::GB(b ^ 1), &lbar[b ^ 1],
+            load_chunk(sb + smt::K(b ^ 1), smt::K_HALF, false, sb + smt::V(b ^ 1), sb + smt::GB(b ^ 1), &lbar[b ^ 1],
                        nullptr, &tm_k, &tm_v, g, beta, cs + C, min(C, sg.b - cs - C), H, h);
         if (!(ok = wait_all_ok(&bars[0], par))) break;
         x1_epilogue(reinterpret_cast<float *>(smem + smt::AF), 0, tl + TT_XW, Gl, bet, row, half);
@@ -737,9 +758,9 @@ __global__ void __launch_bounds__(NT, 1)
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                tc::mma_bf16(tm + TT_XW, tc::make_desc(kt + kk * 256, 128, 1024),
+                tc::mma_bf16(tm + TT_XW, tc::make_desc_sw128(kt + kk * 2048, smt::K_HALF, 1024),
                              tc::make_desc(sb + smt::T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                tc::mma_bf16(tm + TT_U, tc::make_desc(vt + kk * 256, 128, 1024),
+                tc::mma_bf16(tm + TT_U, tc::make_desc_sw128(vt + kk * 2048, 8192, 1024),
                              tc::make_desc(sb + smt::T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
             }
             tc::mma_commit(&bars[1]);
@@ -798,7 +819,7 @@ __global__ void __launch_bounds__(NT, 1)
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk) {
-                const uint64_t bk = tc::make_desc(kt + kk * 256, 128, 1024);
+                const uint64_t bk = tc::make_desc_sw128(kt + kk * 2048, smt::K_HALF, 1024);
                 tc::mma_bf16(tm + TT_S, tc::make_desc(sb + smt::DTS + kk * 4096, 2048, 128), bk, id_km128, 1);
                 tc::mma_bf16(tm + TT_X, tc::make_desc(sb + smt::DTX + kk * 4096, 2048, 128), bk, id_km128, 1);
             }
@@ -939,8 +960,9 @@ namespace {
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
-// TMA descriptor of a token-major bf16 tensor [T][H][128]: boxes of 8 elements
-// (16 bytes) x 1 head x 64 tokens; out-of-range tokens read as zero.
+// TMA descriptor of a token-major bf16 tensor [T][H][128]: boxes of 64
+// columns (128 bytes) x 1 head x 64 tokens, written to shared memory with the
+// 128-byte swizzle; out-of-range tokens read as zero.
 cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
@@ -953,10 +975,10 @@ cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T) {
     if (!g_encode) return cudaErrorNotSupported;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)std::max(T, 1)};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    const cuuint32_t box[3] = {8, 1, 64};
+    const cuuint32_t box[3] = {64, 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<bf16 *>(base), dims, strides, box,
-                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }

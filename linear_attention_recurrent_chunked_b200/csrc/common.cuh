@@ -10,7 +10,7 @@
 namespace gdn {
 
 // Device error word layout (first 4 bytes of the chunk workspace).
-enum : uint32_t { ERRBIT_SEQLENS = 1u, ERRBIT_TIMEOUT = 2u };
+enum : uint32_t { ERRBIT_SEQLENS = 1u, ERRBIT_TIMEOUT = 2u, ERRBIT_INTERNAL = 4u };
 
 template <typename T> struct Elem;
 template <> struct Elem<float> {

@@ -26,15 +26,32 @@ __device__ void stage(uint8_t *dst, const __nv_bfloat16 *src, int rows, int cols
     }
 }
 
+// 128-byte-swizzled staging (variant 2): K-major tiles have rows = MN and
+// 128-byte rows along K; MN-major tiles have rows = K and 128-byte rows along MN.
+__device__ void stage_sw128(uint8_t *dst, const __nv_bfloat16 *src, int rows, int cols, int mn_major) {
+    const int R = mn_major ? cols : rows;  // tile rows
+    for (int idx = threadIdx.x; idx < rows * cols; idx += blockDim.x) {
+        const int r = idx / cols, c = idx % cols;
+        const int tr = mn_major ? c : r, tc_ = mn_major ? r : c;
+        *reinterpret_cast<__nv_bfloat16 *>(dst + tc::sw128_off(tr, tc_, R)) = src[idx];
+    }
+}
+
 __global__ void __launch_bounds__(128) k_diag_mma(const __nv_bfloat16 *A, const __nv_bfloat16 *B, float *D, int M,
                                                   int N, int K, int a_mn, int b_mn, int variant) {
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t mbar;
     __shared__ uint32_t tslot;
-    uint8_t *sA = smem, *sB = smem + (size_t)M * K * 2;
-    uint32_t axs, ays, bxs, bys;
-    stage(sA, A, M, K, a_mn, variant, axs, ays);
-    stage(sB, B, N, K, b_mn, variant, bxs, bys);
+    uint8_t *smem = smem_raw + ((1024u - (tc::smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-byte aligned base
+    uint8_t *sA = smem, *sB = smem + 65536;
+    uint32_t axs = 0, ays = 0, bxs = 0, bys = 0;
+    if (variant == 2) {
+        stage_sw128(sA, A, M, K, a_mn);
+        stage_sw128(sB, B, N, K, b_mn);
+    } else {
+        stage(sA, A, M, K, a_mn, variant, axs, ays);
+        stage(sB, B, N, K, b_mn, variant, bxs, bys);
+    }
     tc::fence_smem_to_async();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == 0) tc::tmem_alloc(&tslot, 256);
@@ -47,15 +64,29 @@ __global__ void __launch_bounds__(128) k_diag_mma(const __nv_bfloat16 *A, const 
     tc::fence_after_sync();
     const uint32_t tmem = tslot;
     if (threadIdx.x == 0) {
-        // K-major: SBO = X stride (MN), LBO = Y stride (K); one K=16 step = 2 core matrices along Y.
-        // MN-major: SBO = Y stride (MN), LBO = X stride (K); one K=16 step = 2 core matrices along X.
-        const uint32_t a_sbo = a_mn ? ays : axs, a_lbo = a_mn ? axs : ays, a_step = 2 * (a_mn ? axs : ays);
-        const uint32_t b_sbo = b_mn ? bys : bxs, b_lbo = b_mn ? bxs : bys, b_step = 2 * (b_mn ? bxs : bys);
         const uint32_t idesc = tc::make_idesc_bf16(M, N, a_mn, b_mn);
-        for (int kk = 0; kk < K / 16; ++kk) {
-            const uint64_t ad = tc::make_desc(tc::smem_u32(sA) + kk * a_step, a_lbo, a_sbo);
-            const uint64_t bd = tc::make_desc(tc::smem_u32(sB) + kk * b_step, b_lbo, b_sbo);
-            tc::mma_bf16(tmem, ad, bd, idesc, kk > 0);
+        if (variant == 2) {
+            // K-major: rows = MN, SBO = 1024 (8-row groups); a K=16 step moves 32 bytes inside
+            // the 128-byte row, and K >= 64 continues in the second column half (R x 128 bytes on).
+            // MN-major: rows = K, SBO = 1024 (8-row K groups), LBO = K x 128 (next 64-wide MN half);
+            // a K=16 step is 16 rows = 2048 bytes.
+            for (int kk = 0; kk < K / 16; ++kk) {
+                const uint32_t a_off = a_mn ? kk * 2048u : (uint32_t)((kk >> 2) * M * 128 + (kk & 3) * 32);
+                const uint32_t b_off = b_mn ? kk * 2048u : (uint32_t)((kk >> 2) * N * 128 + (kk & 3) * 32);
+                const uint64_t ad = tc::make_desc_sw128(tc::smem_u32(sA) + a_off, a_mn ? (uint32_t)K * 128 : 16, 1024);
+                const uint64_t bd = tc::make_desc_sw128(tc::smem_u32(sB) + b_off, b_mn ? (uint32_t)K * 128 : 16, 1024);
+                tc::mma_bf16(tmem, ad, bd, idesc, kk > 0);
+            }
+        } else {
+            // K-major: SBO = X stride (MN), LBO = Y stride (K); one K=16 step = 2 core matrices along Y.
+            // MN-major: SBO = Y stride (MN), LBO = X stride (K); one K=16 step = 2 core matrices along X.
+            const uint32_t a_sbo = a_mn ? ays : axs, a_lbo = a_mn ? axs : ays, a_step = 2 * (a_mn ? axs : ays);
+            const uint32_t b_sbo = b_mn ? bys : bxs, b_lbo = b_mn ? bxs : bys, b_step = 2 * (b_mn ? bxs : bys);
+            for (int kk = 0; kk < K / 16; ++kk) {
+                const uint64_t ad = tc::make_desc(tc::smem_u32(sA) + kk * a_step, a_lbo, a_sbo);
+                const uint64_t bd = tc::make_desc(tc::smem_u32(sB) + kk * b_step, b_lbo, b_sbo);
+                tc::mma_bf16(tmem, ad, bd, idesc, kk > 0);
+            }
         }
         tc::mma_commit(&mbar);
     }
@@ -80,10 +111,12 @@ extern "C" gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, 
                                         int b_mn, int variant, void *stream) {
     if (!A || !B || !D) return GDN_ERR_NULL;
     const bool n_ok = (M == 128) ? (N % 16 == 0) : (N % 8 == 0);
-    if ((M != 64 && M != 128) || N < 16 || N > 256 || !n_ok || K < 16 || K > 128 || K % 16 || (variant & ~1) ||
-        (a_mn & ~1) || (b_mn & ~1))
+    if ((M != 64 && M != 128) || N < 16 || N > 256 || !n_ok || K < 16 || K > 128 || K % 16 || variant < 0 ||
+        variant > 2 || (a_mn & ~1) || (b_mn & ~1))
         return GDN_ERR_SHAPE;
-    const int smem = (M + N) * K * 2;
+    if (variant == 2 && (N > 128 || (a_mn && K < 64 && M > 64) || (b_mn && K < 64 && N > 64)))
+        return GDN_ERR_SHAPE;  // swizzled tiles: N <= 128; an MN-major tile wider than 64 needs K >= 64 rows per half
+    const int smem = 1024 + 65536 + 65536;
     cudaError_t e = cudaFuncSetAttribute(gdn::k_diag_mma, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
     gdn::k_diag_mma<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(

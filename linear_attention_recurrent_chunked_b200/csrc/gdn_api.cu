@@ -221,6 +221,7 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
     if (word & gdn::ERRBIT_SEQLENS) return fail(GDN_ERR_SEQLENS, "cu_seqlens is not 0 = c0 <= c1 <= ... <= cN = T_tot");
     if (word & gdn::ERRBIT_TIMEOUT) return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    if (word & gdn::ERRBIT_INTERNAL) return fail(GDN_ERR_CUDA, "internal: misaligned shared-memory base, nothing written");
     return ok();
 }
 

@@ -34,6 +34,21 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t smem_addr, uint32_t lbo, 
     return d;
 }
 
+// 128-byte-swizzled operand tiles (the layout TMA writes with SWIZZLE_128B):
+// rows of 128 bytes (64 bf16), 8-row atoms of 1024 bytes, the 16-byte chunk
+// index within a row XORed with (row % 8). A tile of R rows and 128 columns
+// holds two such column halves of R x 128 bytes each. Byte offset of
+// element (row, col) in a tile of R rows (tile base 1024-byte aligned):
+__host__ __device__ __forceinline__ uint32_t sw128_off(int row, int col, int R) {
+    const uint32_t half = (uint32_t)(col >> 6), c = (uint32_t)(col & 63);
+    const uint32_t lin = (uint32_t)row * 128u + c * 2u;
+    return half * (uint32_t)R * 128u + (lin ^ (((lin >> 7) & 7u) << 4));
+}
+// SWIZZLE_128B descriptor (layout type 2 in bits 61-63).
+__device__ __forceinline__ uint64_t make_desc_sw128(uint32_t smem_addr, uint32_t lbo, uint32_t sbo) {
+    return make_desc(smem_addr, lbo, sbo) | ((uint64_t)2u << 61);
+}
+
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, dense.
 // a_mn / b_mn: 1 if that operand is MN-major (0 = K-major).
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, int a_mn, int b_mn) {

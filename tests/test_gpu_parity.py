@@ -195,6 +195,18 @@ def test_diag_mma_m128(variant, a_mn, b_mn, N, K):
     assert torch.allclose(D, ref, atol=1e-3, rtol=1e-3), (D - ref).abs().max()
 
 
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (1, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (128, 128)])
+def test_diag_mma_m128_swizzled(a_mn, b_mn, N, K):
+    """128-byte-swizzled operand tiles (the layout TMA writes with SWIZZLE_128B)."""
+    g = torch.Generator().manual_seed(3 * N + K)
+    A = torch.randn(128, K, generator=g).bfloat16()
+    B = torch.randn(N, K, generator=g).bfloat16()
+    D = gdn.diag_mma_tile(A.cuda(), B.cuda(), a_mn, b_mn, 2).cpu()
+    ref = A.float() @ B.float().T
+    assert torch.allclose(D, ref, atol=1e-3, rtol=1e-3), (D - ref).abs().max()
+
+
 def test_diag_mma_m64_lane_map():
     """Where the rows of an M=64 accumulator land in TMEM (recorded for the kernels)."""
     g = torch.Generator().manual_seed(64)
