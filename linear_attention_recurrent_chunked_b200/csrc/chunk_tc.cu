@@ -445,8 +445,8 @@ __device__ bool segment_fold(uint32_t sb, uint32_t tm, uint32_t tl, uint64_t *ba
 // ============================================================================ output pass
 __global__ void __launch_bounds__(NT, 1)
     k_chunk_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const float *__restrict__ g, const float *__restrict__ beta,
-               const float *S0,
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const float *__restrict__ g, const float *__restrict__ beta, const float *S0,
                const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o, float *S_T,
                uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off, int seg_tokens,
                const float *__restrict__ slots) {
@@ -512,6 +512,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int cs = sg.a + c * C, L = min(C, sg.b - cs), b = c & 1;
         const uint32_t par = (uint32_t)(c & 1);
         const uint32_t kq = sb + smo::KQ(b), vt = sb + smo::V(b);
+        if (tid == 64) tc::bulk_wait_read();  // the previous chunk's output store has left the staging rows
         cp_async_wait_all();
         tc::fence_smem_to_async();
         __syncthreads();
@@ -615,8 +616,15 @@ __global__ void __launch_bounds__(NT, 1)
                         __float2bfloat16_rn(fmaf(gam[c0 + i], a[i], d[i]));
             }
         }
-        __syncthreads();
-        {
+        // A whole chunk, or a partial one that ends the tensor (TMA clips the rows past it), goes out
+        // as one bulk tensor store; a partial chunk followed by another sequence's tokens is copied
+        // row by row so that those tokens' outputs are not overwritten.
+        if (L == C || cs + L >= T_tot) {
+            tc::fence_smem_to_async();
+            __syncthreads();
+            if (tid == 64) tc::tma_store_3d(&tm_o, sb + smo::OST, 0, h, cs);
+        } else {
+            __syncthreads();
             const uint8_t *ost = smem + smo::OST;
 #pragma unroll
             for (int it = 0; it < 4; ++it) {
@@ -646,6 +654,7 @@ __global__ void __launch_bounds__(NT, 1)
         handoff_to_mma();
     }
     cp_async_wait_all();
+    if (tid == 64) tc::bulk_wait_all();
     if (!ok) {
         if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
     } else if (sg.s == sg.ns - 1) {
@@ -962,8 +971,9 @@ std::once_flag g_encode_once;
 
 // TMA descriptor of a token-major bf16 tensor [T][H][128]: boxes of 64
 // columns (128 bytes) x 1 head x 64 tokens, written to shared memory with the
-// 128-byte swizzle; out-of-range tokens read as zero.
-cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T) {
+// 128-byte swizzle, out-of-range tokens reading as zero; or (whole_rows) boxes
+// of whole 256-byte rows x 64 tokens without swizzle, for the output store.
+cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T, bool whole_rows = false) {
     std::call_once(g_encode_once, [] {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -975,10 +985,11 @@ cudaError_t make_row_map(CUtensorMap *map, const bf16 *base, int H, int T) {
     if (!g_encode) return cudaErrorNotSupported;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)std::max(T, 1)};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    const cuuint32_t box[3] = {64, 1, 64};
+    const cuuint32_t box[3] = {whole_rows ? 128u : 64u, 1, 64};
     const cuuint32_t estr[3] = {1, 1, 1};
     const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<bf16 *>(base), dims, strides, box,
-                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                whole_rows ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
@@ -988,9 +999,10 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
                             const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
                             void *workspace, size_t ws_bytes, cudaStream_t st, const char **stage) {
     uint32_t *err = static_cast<uint32_t *>(workspace);
-    CUtensorMap tm_q, tm_k, tm_v;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o;
     cudaError_t e;
     *stage = "TMA descriptor encoding";
+    if ((e = make_row_map(&tm_o, o, H, T_tot, true)) != cudaSuccess) return e;
     if ((e = make_row_map(&tm_q, q, H, T_tot)) != cudaSuccess) return e;
     if ((e = make_row_map(&tm_k, k, H, T_tot)) != cudaSuccess) return e;
     if ((e = make_row_map(&tm_v, v, H, T_tot)) != cudaSuccess) return e;
@@ -1010,7 +1022,7 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
         e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
         if (e != cudaSuccess) return e;
         void *pr = prof_start("chunk_tc", st);
-        k_chunk_tc<<<dim3(H, N), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
+        k_chunk_tc<<<dim3(H, N), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, tm_o, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
                                                          nullptr, 0, nullptr);
         prof_stop(pr);
         return cudaGetLastError();
@@ -1037,7 +1049,7 @@ cudaError_t launch_chunk_tc(const bf16 *q, const bf16 *k, const bf16 *v, const f
     e = cudaFuncSetAttribute(k_chunk_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smo::TOTAL);
     if (e != cudaSuccess) return e;
     pr = prof_start("chunk_tc", st);
-    k_chunk_tc<<<dim3(H, nslots), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
+    k_chunk_tc<<<dim3(H, nslots), NT, smo::TOTAL, st>>>(tm_q, tm_k, tm_v, tm_o, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
                                                          seg_off, seg_tokens, slots);
     prof_stop(pr);
     return cudaGetLastError();
