@@ -55,6 +55,34 @@ def decode_bytes(B, H, d) -> int:
     return B * H * (2 * d * d * 4 + 3 * d * 2 + 8 + d * 2)
 
 
+def kernel_source_digest() -> str:
+    """Digest of the CUDA sources and the C header: ties an ncu traffic figure to the kernels it was taken on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "linear_attention_recurrent_chunked_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh")) +
+                    glob.glob(os.path.join(pkg, "*.h")) + [os.path.join(ROOT, "include", "gdn.h")]):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of `kernel` on
+    `workload` from the committed ncu capture in profiles/traffic.json, or None if that capture
+    was taken on different kernel sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("source_digest") != kernel_source_digest():
+        return None
+    v = t.get("bytes_per_launch", {}).get("%s@%s" % (kernel, workload))
+    return float(v) if v is not None else None
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -241,7 +269,8 @@ def gpu_arm(args):
                         for k, v in kt.items()},
             "top_kernel": top[0],
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": None, "peak_source": pk["src"],
+                         "frac": gbs / pk["hbm"], "traffic": measured_traffic(top[0], name),
+                         "peak_source": pk["src"], "kernel": top[0],
                          "tensor_tflops": nflops / (top_ms * 1e-3) / 1e12},
             "launches_per_step": sum(v[1] for v in kt.values()) // max(3, min(steps, 10)),
         }
