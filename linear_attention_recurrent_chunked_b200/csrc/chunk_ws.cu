@@ -1,0 +1,1237 @@
+// Chunked gated delta rule on the sm_100a tensor cores with warp-specialised
+// pipelining (bf16 inputs, d = 128, chunk C = 64). The arithmetic is the
+// chunked rewrite of the recurrence (page 1, abstract, result (i); page 2,
+// "Resumen Tecnico", Metodologia, recurrent-layer item: intra-chunk part,
+// inter-chunk state pass and a forward-substitution solve). Per chunk of one
+// (sequence, head), S the d_v x d_k state entering it, G_r = sum_{s<=r} g_s,
+// gamma_r = exp(G_r), e_s = exp(G_C - G_s):
+//
+//   T  = (I + A)^{-1},  A_rs = beta_r exp(G_r - G_s) (k_r . k_s), s < r
+//   T1 = T diag(beta gamma),  T2 = T diag(beta)
+//   W^T = K^T T1^T,  U^T = V^T T2^T
+//   Delta^T = U^T - S W^T
+//   O^T = S (diag(gamma) Q)^T + Delta^T P^T,  P_rs = exp(G_r - G_s)(q_r . k_s), s <= r
+//   S  <- gamma_C S + Delta^T (diag(e) K)
+//
+// Work is split three ways:
+//  1. k_ws_prep, over every (chunk, head) in parallel (several CTAs per SM):
+//     the state-independent scalars and the UT solve. One 9 KB record per
+//     (chunk, head): T2 as a ready bf16 operand tile, then G (log2 units),
+//     gamma, e and beta.
+//  2. k_ws_trans, one CTA per segment except the last of its sequence (only
+//     when a sequence is split into segments that run concurrently): runs the
+//     segment from S = 0 (S_loc) and, on a second state, from X = I with the
+//     V-term dropped (Phi = X_end), since over a segment the state map is
+//     affine, S_end = S_in Phi + S_loc. It then waits for the previous
+//     segment's published end state S_in, forms S_end on the tensor cores
+//     (bf16 hi/lo split operands, fp32 accumulation) and publishes it. The
+//     first segment starts from S0 and needs no Phi.
+//  3. k_ws_out, one CTA per segment: starts from S0 or the published end
+//     state of the previous segment and writes the outputs (and S_T).
+//
+// In 2 and 3 the warps have fixed roles and pass tiles to each other through
+// mbarriers, so that the next chunk's loads and operand preparation overlap
+// the current chunk's dependent state step:
+//   loader (1 thread)  K, Q, V by TMA (128-byte swizzle), the record by bulk copy
+//   MMA    (1 thread)  every tcgen05.mma, in an order that keeps the chain first
+//   prep   (4 warps)   T1 from T2; P from X1 = Q K^T; Q <- diag(gamma) Q and
+//                      K <- diag(e) K in place; -W from W^T
+//   state  (4 warps)   Delta^T (accumulated on top of U^T in TMEM) -> bf16 tile;
+//                      S -> bf16 tile, and S <- gamma_C' S in TMEM so that the
+//                      next update accumulates onto it
+//   output (4 warps)   O^T -> bf16 rows -> TMA store  (k_ws_out)
+//   X-state (4 warps)  the Phi chain                   (k_ws_trans)
+// Every wait is bounded in time; a timeout sets the error word and makes all
+// roles of the CTA leave their loops.
+#include "chunk_common.cuh"
+#include "kernels.h"
+#include "ut_solve.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace chunk;
+using bf16 = __nv_bfloat16;
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int AP = ut::AP;
+constexpr uint64_t kWaitNs = 1000000000ull;  // bound of any single wait (1 s)
+
+// ---- per-(chunk, head) record written by k_ws_prep
+constexpr uint32_t REC_T2 = 0;      // T2 bf16 tile: rows r, 16-byte runs along s (sx = 128, sy = 1024)
+constexpr uint32_t REC_VEC = 8192;  // G (log2 units), gamma, e, beta: 4 x 64 fp32
+constexpr uint32_t REC_BYTES = 9216;
+// ---- published segment end state: bf16 hi and lo tiles, rows v, runs along k (sx = 128, sy = 2048)
+constexpr uint32_t LINK_BYTES = 65536;
+constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
+
+// Warp roles of the pipelined kernels (448 threads).
+constexpr int NT_WS = 448;
+constexpr int W_LOAD = 12, W_MMA = 13;
+
+struct Ctl {
+    uint32_t tmem;   // TMEM base written by tcgen05.alloc
+    uint32_t abort;  // set by the first role that gives up
+};
+
+// Bounded wait for the phase `parity` of an mbarrier. Gives up when another
+// role has aborted, or after kWaitNs (then it records the timeout and aborts).
+__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = tc::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) == 0) {
+            if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
+            if (tc::globaltimer() - t0 > kWaitNs) {
+                atomicOr(err, ERRBIT_TIMEOUT);
+                *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+                return false;
+            }
+        }
+    }
+}
+// Time-bounded wait that ignores the abort flag (used to drain copies in flight before exit).
+__device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = tc::globaltimer();
+    while (!tc::mbar_try_wait(bar, parity))
+        if (tc::globaltimer() - t0 > kWaitNs) return;
+}
+
+__device__ __forceinline__ uint32_t lane_base(uint32_t tm, int warp) { return tm + ((uint32_t)((warp & 3) * 32) << 16); }
+
+// Scale the 64 rows of a 128-byte-swizzled 64 x 128 bf16 tile (two 8 KB column
+// halves) by f[row], in place. The swizzle only permutes 16-byte chunks within
+// a row, so a chunk's row is its offset within the half / 128. 128 threads.
+__device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, int t128) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int idx = t128 + 128 * i, row = (idx & 511) >> 3;
+        uint4 *p = reinterpret_cast<uint4 *>(tile + 16 * idx);
+        uint4 x = *p;
+        const float s = f[row];
+        uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[j]));
+            w[j] = tc::pack_bf16x2(a.x * s, a.y * s);
+        }
+        *p = x;
+    }
+}
+
+// T1 = T2 diag(gamma) between two 64 x 64 bf16 tiles (rows r, runs along s; sy = 1024). 128 threads.
+__device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t128) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int idx = t128 + 128 * i, s0 = 8 * (idx >> 6);
+        uint4 x = *reinterpret_cast<const uint4 *>(t2 + 16 * idx);
+        uint32_t *w = reinterpret_cast<uint32_t *>(&x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[j]));
+            w[j] = tc::pack_bf16x2(a.x * gam[s0 + 2 * j], a.y * gam[s0 + 2 * j + 1]);
+        }
+        *reinterpret_cast<uint4 *>(t1 + 16 * idx) = x;
+    }
+}
+
+// -W tile (rows k, runs along r; sx = 128, sy = 2048) from this thread's TMEM lane k of W^T (64 columns).
+__device__ __forceinline__ void neg_w_epilogue(uint32_t w_tile, uint32_t tl_wt, int k) {
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        float x[32];
+        tc::tmem_ld32(tl_wt + c0, x);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = -x[i];
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) st_run8(w_tile + tc::tile_off(k, c0 + i, 128, 2048), x + i);
+    }
+}
+
+// bf16 tile (rows v, runs along the 64 columns; sx = 128, sy = 2048) from this thread's TMEM lane v.
+__device__ __forceinline__ void tile64_epilogue(uint32_t tile, uint32_t tl, int v) {
+#pragma unroll
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+        float x[32];
+        tc::tmem_ld32(tl + c0, x);
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) st_run8(tile + tc::tile_off(v, c0 + i, 128, 2048), x + i);
+    }
+}
+
+// The state step after the update MMA: read row v of S (fp32, 128 columns) from
+// TMEM, write its bf16 copy to the S tile and S * g_next back to TMEM (the
+// next update accumulates onto gamma_C S). With last set, nothing is written
+// back and the row goes to dst_row (fp32, global) if given.
+__device__ __forceinline__ void state_epilogue(uint32_t s_tile, uint32_t tl_s, int v, float g_next, bool last,
+                                               float *dst_row) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+        float x[32];
+        tc::tmem_ld32(tl_s + c0, x);
+        if (!last) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) st_run8(s_tile + tc::tile_off(v, c0 + i, 128, 2048), x + i);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] *= g_next;
+            tc::tmem_st16(tl_s + c0, *reinterpret_cast<float(*)[16]>(x));
+            tc::tmem_st16(tl_s + c0 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+        } else if (dst_row) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                *reinterpret_cast<float4 *>(dst_row + c0 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        }
+    }
+    if (!last) tc::tmem_st_wait();
+}
+
+// Initial state row v: fp32 values from src_f32 (row-major, may be null: zeros),
+// or from a published hi/lo tile pair (link, may be null), or the identity row.
+// Written as g0 * S to TMEM and as bf16 to the tile.
+__device__ __forceinline__ void state_init(uint32_t s_tile, uint32_t tl_s, int v, float g0, const float *src_f32,
+                                           const uint8_t *link, bool identity) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 16) {
+        float x[16];
+        if (link) {
+#pragma unroll
+            for (int h8 = 0; h8 < 16; h8 += 8) {
+                const uint32_t off = tc::tile_off(v, c0 + h8, 128, 2048);
+                uint4 hi = *reinterpret_cast<const uint4 *>(link + off);
+                uint4 lo = *reinterpret_cast<const uint4 *>(link + 32768 + off);
+                const uint32_t *wh = reinterpret_cast<const uint32_t *>(&hi);
+                const uint32_t *wl = reinterpret_cast<const uint32_t *>(&lo);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wh[j]));
+                    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wl[j]));
+                    x[h8 + 2 * j] = a.x + b.x;
+                    x[h8 + 2 * j + 1] = a.y + b.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (src_f32) a = *reinterpret_cast<const float4 *>(src_f32 + c0 + i);
+                x[i] = a.x; x[i + 1] = a.y; x[i + 2] = a.z; x[i + 3] = a.w;
+            }
+            if (identity)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) x[i] = (c0 + i == v) ? 1.f : 0.f;
+        }
+        st_run8(s_tile + tc::tile_off(v, c0, 128, 2048), x);
+        st_run8(s_tile + tc::tile_off(v, c0 + 8, 128, 2048), x + 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] *= g0;
+        tc::tmem_st16(tl_s + c0, x);
+    }
+    tc::tmem_st_wait();
+}
+
+// Signal an mbarrier after this thread's shared-memory writes (for the tensor
+// core) and TMEM accesses are complete.
+__device__ __forceinline__ void handoff(uint64_t *bar) {
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    tc::mbar_arrive(bar);
+}
+
+// Index of the (chunk, head) record; the segment's first chunk is chunk_off[n] + s * seg_chunks.
+__device__ __forceinline__ size_t rec_index(const int32_t *chunk_off, const Segment &sg, int seg_chunks, int c, int H,
+                                            int h) {
+    return ((size_t)chunk_off[sg.n] + (size_t)sg.s * seg_chunks + c) * H + h;
+}
+
+// ============================================================================ prep
+namespace pp {
+constexpr uint32_t K0 = 0;                          // two K tiles (128-byte swizzle), 16 KB each
+constexpr uint32_t AT = 32768;                      // A, then T in place: fp32 [64][AP]
+constexpr uint32_t XS = AT + 64 * AP * 4;           // solve scratch, 32 x XP fp32
+constexpr uint32_t REC = XS + 32 * ut::XP * 4;      // record staging (bulk-stored)
+constexpr uint32_t RAW = REC + REC_BYTES;           // raw g, beta of two items: 2 x 512 B
+constexpr uint32_t BAR = RAW + 1024;                // full[2], mma, TMEM slot
+constexpr uint32_t TOTAL = BAR + 64;
+}  // namespace pp
+
+// Persistent: CTA b handles items b, b + gridDim.x, ... where item = gc * H + h
+// (gc = global chunk index, prefix chunk_off over sequences). The next item's
+// K tile (TMA) and g, beta (cp.async) are fetched while the current one runs.
+__global__ void __launch_bounds__(256, 3)
+    k_ws_prep(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ g, const float *__restrict__ beta,
+              const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
+              const int32_t *__restrict__ chunk_off, uint8_t *__restrict__ rec) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;
+    const int items = chunk_off[N] * H;
+    if ((int)blockIdx.x >= items) return;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t sb = tc::smem_u32(smem);
+    if (sb & 1023u) {
+        if (tid == 0) atomicOr(err, ERRBIT_INTERNAL);
+        return;
+    }
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + pp::BAR);  // [0,1] full, [2] mma
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + pp::BAR + 32);
+    if (warp == 0) tc::tmem_alloc(tslot, 64);
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) tc::mbar_init(&bars[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = *tslot;
+    float *AT = reinterpret_cast<float *>(smem + pp::AT);
+    float *vec = reinterpret_cast<float *>(smem + pp::REC + REC_VEC);
+    float *Gl = vec, *gam = vec + 64, *dte = vec + 128, *bet = vec + 192;
+
+    // where item w lives: sequence n, chunk start cs, valid length L
+    auto locate = [&](int w, int &h, int &cs, int &L, int &gc) {
+        gc = w / H;
+        h = w - gc * H;
+        int lo = 0, hi = N - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+        }
+        int t0, t1;
+        seq_bounds(cu, lo, N, T_tot, t0, t1);
+        cs = t0 + (gc - chunk_off[lo]) * C;
+        L = min(C, t1 - cs);
+    };
+    auto issue = [&](int w, int b) {
+        int h, cs, L, gc;
+        locate(w, h, cs, L, gc);
+        if (tid == 32) {
+            tc::mbar_arrive_expect_tx(&bars[b], 16384u);
+            tc::tma_load_3d(sb + pp::K0 + b * 16384u, &tm_k, &bars[b], 0, h, cs);
+            tc::tma_load_3d(sb + pp::K0 + b * 16384u + 8192u, &tm_k, &bars[b], 64, h, cs);
+        }
+        if (tid < 2 * C) {
+            const int r = tid & 63;
+            const bool ok = r < L;
+            const size_t off = (size_t)(cs + (ok ? r : 0)) * H + h;
+            cp_async4(sb + pp::RAW + b * 512u + (tid < C ? 0u : 256u) + 4u * r, (tid < C ? g : beta) + off,
+                      ok ? 4u : 0u);
+        }
+        cp_async_commit();
+    };
+
+    const uint32_t id_m64 = tc::make_idesc_bf16(64, 64, 0, 0);
+    const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
+    bool ok = true;
+    issue(blockIdx.x, 0);
+    int it = 0;
+    for (int w = blockIdx.x; w < items; w += gridDim.x, ++it) {
+        const int b = it & 1;
+        const int wn = w + gridDim.x;
+        if (wn < items) {
+            issue(wn, b ^ 1);
+            cp_async_wait_1();
+        } else {
+            cp_async_wait_all();
+        }
+        if (tid == 0) tc::bulk_wait_read();  // the previous record has left the staging area
+        __syncthreads();
+        // ---- scalars: G = cumsum(g) (log2 units), gamma, e, beta
+        const float *graw = reinterpret_cast<const float *>(smem + pp::RAW + b * 512u);
+        if (tid < 32) {
+            const float a = graw[2 * tid] * kLog2e, b2 = a + graw[2 * tid + 1] * kLog2e;
+            float sc = b2;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, sc, off);
+                if (tid >= off) sc += y;
+            }
+            Gl[2 * tid] = sc - b2 + a;
+            Gl[2 * tid + 1] = sc;
+        }
+        __syncthreads();
+        if (tid < C) {
+            gam[tid] = ex2(Gl[tid]);
+            dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
+            bet[tid] = graw[64 + tid];
+        }
+        // ---- X1 = K K^T (M = 64: accumulator row i in TMEM lane (i % 16) + 32 (i / 16))
+        if (tid == 0) {
+            if (!tc::mbar_wait(&bars[b], (uint32_t)((it >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
+            tc::fence_after_sync();
+            const uint32_t kt = sb + pp::K0 + b * 16384u;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::make_desc_sw128(kt + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                tc::mma_bf16(tm, a, a, id_m64, kk > 0);
+            }
+            tc::mma_commit(&bars[2]);
+        }
+        ok = tc::mbar_wait(&bars[2], (uint32_t)(it & 1));
+        tc::fence_after_sync();
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
+            break;
+        }
+        // ---- A_rs = beta_r exp(G_r - G_s) X1_rs for s < r (warp w: rows 16 (w%4) + lane, columns 32 (w/4) ..)
+        {
+            const int lane = tid & 31, r = 16 * (warp & 3) + (lane & 15), s0 = 32 * (warp >> 2);
+            float x[32];
+            tc::tmem_ld32(tl + s0, x);  // all lanes load (the instruction is warp-wide); lanes >= 16 discard
+            if (lane < 16) {
+                const float Gr = Gl[r], br = bet[r];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 a;
+                    a.x = (s0 + i < r) ? br * ex2(Gr - Gl[s0 + i]) * x[i] : 0.f;
+                    a.y = (s0 + i + 1 < r) ? br * ex2(Gr - Gl[s0 + i + 1]) * x[i + 1] : 0.f;
+                    a.z = (s0 + i + 2 < r) ? br * ex2(Gr - Gl[s0 + i + 2]) * x[i + 2] : 0.f;
+                    a.w = (s0 + i + 3 < r) ? br * ex2(Gr - Gl[s0 + i + 3]) * x[i + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(AT + r * AP + s0 + i) = a;
+                }
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        ut::solve64(AT, AT, reinterpret_cast<float *>(smem + pp::XS));
+        // ---- T2 = T diag(beta) as a bf16 operand tile (thread: row tid / 4, columns 16 (tid % 4) ..)
+        {
+            const int r = tid >> 2, s0 = 16 * (tid & 3);
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = AT[r * AP + s0 + i] * bet[s0 + i];
+            st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0, 128, 1024), x);
+            st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0 + 8, 128, 1024), x + 8);
+        }
+        tc::fence_smem_to_async();
+        __syncthreads();
+        if (tid == 0) {
+            int h, cs, L, gc;
+            locate(w, h, cs, L, gc);
+            tc::bulk_store(rec + ((size_t)gc * H + h) * REC_BYTES, sb + pp::REC, REC_BYTES);
+        }
+    }
+    cp_async_wait_all();
+    if (tid == 32 && !ok) {  // a K tile may still be in flight after a timeout
+        drain_bar(&bars[0], 0);
+        drain_bar(&bars[1], 0);
+    }
+    if (tid == 0) tc::bulk_wait_all();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 64);
+}
+
+// ============================================================================ output pass
+namespace ob {
+constexpr uint32_t B_K = 0, B_Q = 16384, B_V = 32768, B_T2 = 49152, B_VEC = 57344;
+constexpr uint32_t BUF = 58368;  // one input buffer (K, Q, V tiles; the record); two of them
+constexpr uint32_t T1 = 2 * BUF;
+constexpr uint32_t P = T1 + 8192;    // two P tiles (rows r, runs along s; sy = 1024)
+constexpr uint32_t W = P + 16384;    // -W tile (rows k, runs along r; sy = 2048)
+constexpr uint32_t S = W + 16384;    // bf16 state (rows v, runs along k; sy = 2048)
+constexpr uint32_t DL = S + 32768;   // Delta^T bf16 (rows v, runs along s; sy = 2048)
+constexpr uint32_t OST = DL + 16384; // output staging: 64 rows o[r][0..127] bf16
+constexpr uint32_t BAR = OST + 16384;
+constexpr uint32_t TOTAL = BAR + 256;
+// TMEM columns
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_X1 = 256, TM_WT = 320, TM_O = 384;
+// mbarriers
+enum {
+    FULL = 0,    // [2] loads of a buffer landed (loader arrive + TMA bytes)
+    EMPTY = 2,   // [2] all MMAs reading a buffer done
+    X1F = 4,     // X1 ready
+    WUF = 5,     // W^T, U^T ready
+    M3 = 6,      // Delta^T ready (state update's first MMA)
+    M4 = 7,      // [2] state update and output done
+    T1R = 9,     // T1 tile written (prep, 128)
+    QR = 10,     // P tile and diag(gamma) Q written (prep, 128)
+    WR = 11,     // -W tile and diag(e) K written (prep, 128)
+    DLR = 12,    // Delta^T tile written (state, 128)
+    SR = 13,     // S tile written, S scaled in TMEM (state, 128)
+    OF = 14,     // [2] O read out of TMEM (output, 128)
+    FIN = 16,    // every MMA of the CTA done (drained before TMEM is freed)
+    NBAR = 17
+};
+}  // namespace ob
+
+__global__ void __launch_bounds__(NT_WS, 1)
+    k_ws_out(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+             const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+             const float *S0, const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o,
+             float *S_T, uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off,
+             const int32_t *__restrict__ chunk_off, int seg_chunks, const uint8_t *__restrict__ rec,
+             const uint8_t *__restrict__ link) {
+    using namespace ob;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;
+    Segment sg;
+    const int h = blockIdx.x;
+    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg)) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sb = tc::smem_u32(smem);
+    if (sb & 1023u) {
+        if (tid == 0) atomicOr(err, ERRBIT_INTERNAL);
+        return;
+    }
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + BAR);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + BAR + 8 * NBAR);
+    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i)
+            tc::mbar_init(&bar[i], (i >= T1R && i < OF + 2) ? 128u : 1u);
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    const int nch = (sg.b - sg.a + C - 1) / C;
+    const size_t sidx = ((size_t)sg.n * H + h) * D * D;
+    const bool last_seg = sg.s == sg.ns - 1;
+    auto buf = [&](int c) { return sb + (uint32_t)(c & 1) * BUF; };
+    auto vecp = [&](int c) { return reinterpret_cast<const float *>(smem + (c & 1) * BUF + B_VEC); };
+
+    if (warp == W_LOAD) {
+        // ---------------------------------------------------------------- loader
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                if (c >= 2 && !wait_bar(&bar[EMPTY + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err)) break;
+                const uint32_t bb = buf(c);
+                const int cs = sg.a + c * C;
+                tc::mbar_arrive_expect_tx(&bar[FULL + b], 3u * 16384u + REC_BYTES);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    tc::tma_load_3d(bb + B_K + hf * 8192, &tm_k, &bar[FULL + b], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_Q + hf * 8192, &tm_q, &bar[FULL + b], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_V + hf * 8192, &tm_v, &bar[FULL + b], 64 * hf, h, cs);
+                }
+                tc::bulk_load(bb + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES, REC_BYTES,
+                              &bar[FULL + b]);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], (uint32_t)((c >> 1) & 1));
+        }
+    } else if (warp == W_MMA) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0 && nch > 0) {
+            const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
+            const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+            const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
+            const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            // X1 = Q K^T (rows 64..127 of the A operand read the next 64 rows of the buffer; never used)
+            auto issue_x1 = [&](int c) {
+                const uint32_t bb = buf(c);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    tc::mma_bf16(tm + TM_X1, tc::make_desc_sw128(bb + B_Q + off, 16, 1024),
+                                 tc::make_desc_sw128(bb + B_K + off, 16, 1024), id_kk64, kk > 0);
+                }
+                tc::mma_commit(&bar[X1F]);
+            };
+            // W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views of the K and V tiles)
+            auto issue_wu = [&](int c) {
+                const uint32_t bb = buf(c);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024),
+                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
+                                 tc::make_desc(bb + B_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                }
+                tc::mma_commit(&bar[WUF]);
+            };
+            bool ok = wait_bar(&bar[FULL], 0, ctl, err);
+            if (ok) {
+                tc::fence_after_sync();
+                issue_x1(0);
+                ok = wait_bar(&bar[T1R], 0, ctl, err);
+            }
+            if (ok) {
+                tc::fence_after_sync();
+                issue_wu(0);
+            }
+            for (int c = 0; ok && c < nch; ++c) {
+                const int b = c & 1;
+                const uint32_t par = (uint32_t)(c & 1), bb = buf(c);
+                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err) &&
+                           wait_bar(&bar[QR], par, ctl, err)))
+                    break;
+                if (c >= 2 && !(ok = wait_bar(&bar[OF + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err))) break;
+                tc::fence_after_sync();
+                // Delta^T = U^T + S (-W)^T, accumulated onto U^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
+                tc::mma_commit(&bar[M3]);
+                // O = S (diag(gamma) Q)^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tm + TM_O + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                                 tc::make_desc_sw128(bb + B_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk64,
+                                 kk > 0);
+                // the next chunk's X1 and W^T, U^T
+                if (c + 1 < nch) {
+                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
+                    tc::fence_after_sync();
+                    issue_x1(c + 1);
+                    if (!(ok = wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err))) break;
+                    tc::fence_after_sync();
+                    issue_wu(c + 1);
+                }
+                if (!(ok = wait_bar(&bar[DLR], par, ctl, err))) break;
+                tc::fence_after_sync();
+                // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K), O += Delta^T P^T
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
+                                 tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16(tm + TM_O + 64 * b, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + P + b * 8192 + kk * 2048, 1024, 128), id_kk64, 1);
+                tc::mma_commit(&bar[M4 + b]);
+                tc::mma_commit(&bar[EMPTY + b]);
+            }
+        }
+    } else if (warp < 4) {
+        // ---------------------------------------------------------------- state (thread = TMEM lane v)
+        const int v = tid;
+        const uint32_t tl = lane_base(tm, warp);
+        bool ok = true;
+        float g0 = 1.f;
+        if (nch > 0) {
+            ok = wait_bar(&bar[FULL], 0, ctl, err);
+            if (ok) g0 = vecp(0)[64 + C - 1];
+        }
+        if (ok) {
+            const uint8_t *lk = nullptr;
+            const float *src = nullptr;
+            if (sg.s > 0)
+                lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
+            else if (S0)
+                src = S0 + sidx + (size_t)v * D;
+            state_init(sb + S, tl + TM_S, v, g0, src, lk, false);
+            if (nch == 0 && last_seg) state_epilogue(sb + S, tl + TM_S, v, 1.f, true, S_T + sidx + (size_t)v * D);
+            handoff(&bar[SR]);
+        }
+        for (int c = 0; ok && c < nch; ++c) {
+            const int b = c & 1;
+            if (!(ok = wait_bar(&bar[M3], (uint32_t)(c & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            tile64_epilogue(sb + DL, tl + TM_U + 64 * b, v);
+            handoff(&bar[DLR]);
+            if (!(ok = wait_bar(&bar[M4 + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            const bool last = c + 1 == nch;
+            float g1 = 1.f;
+            if (!last) {
+                if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
+                g1 = vecp(c + 1)[64 + C - 1];
+            }
+            state_epilogue(sb + S, tl + TM_S, v, g1, last, last && last_seg ? S_T + sidx + (size_t)v * D : nullptr);
+            if (!last) handoff(&bar[SR]);
+        }
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- prep (thread t128 = tid - 128)
+        const int t128 = tid - 128;
+        const uint32_t tl = lane_base(tm, warp);
+        bool ok = true;
+        for (int c = 0; ok && c < nch; ++c) {
+            const int b = c & 1;
+            uint8_t *bp = smem + b * BUF;
+            const float *vec = vecp(c);
+            const float *Gl = vec, *gam = vec + 64, *dte = vec + 128;
+            // T1 = T2 diag(gamma) (WU of the previous chunk has finished reading T1: see WUF below)
+            if (!(ok = wait_bar(&bar[FULL + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            make_t1(smem + T1, bp + B_T2, gam, t128);
+            tc::fence_smem_to_async();
+            tc::mbar_arrive(&bar[T1R]);
+            // P_rs = exp(G_r - G_s) X1_rs for s <= r (rows r = TMEM lanes 0..63: warps 4, 5)
+            if (!(ok = wait_bar(&bar[X1F], (uint32_t)(c & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            if (warp < 6) {
+                const int r = t128;
+                const float Gr = Gl[r];
+                const uint32_t pt = sb + P + b * 8192;
+#pragma unroll
+                for (int s0 = 0; s0 < C; s0 += 32) {
+                    float x[32];
+                    tc::tmem_ld32(tl + TM_X1 + s0, x);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - Gl[s0 + i]) * x[i] : 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) st_run8(pt + tc::tile_off(r, s0 + i, 128, 1024), x + i);
+                }
+            }
+            tc::fence_before_sync();
+            scale_rows_sw128(bp + B_Q, gam, t128);  // X1 has read Q
+            handoff(&bar[QR]);
+            // -W from W^T (thread = TMEM lane k), then K <- diag(e) K (X1 and W^T, U^T have read K)
+            if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            neg_w_epilogue(sb + W, tl + TM_WT, t128);
+            scale_rows_sw128(bp + B_K, dte, t128);
+            handoff(&bar[WR]);
+        }
+    } else {
+        // ---------------------------------------------------------------- output (thread = TMEM lane v)
+        const int v = tid - 256;
+        const uint32_t tl = lane_base(tm, warp);
+        uint8_t *ost = smem + OST;
+        bool ok = true;
+        for (int c = 0; ok && c < nch; ++c) {
+            const int b = c & 1;
+            const int cs = sg.a + c * C, L = min(C, sg.b - cs);
+            if (!(ok = wait_bar(&bar[M4 + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            if (v == 0) tc::bulk_wait_read();  // the previous chunk's store has read the staging rows
+            tc::named_sync(1, 128);
+#pragma unroll
+            for (int c0 = 0; c0 < C; c0 += 32) {
+                float x[32];
+                tc::tmem_ld32(tl + TM_O + 64 * b + c0, x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) *reinterpret_cast<bf16 *>(ost + (c0 + i) * 256 + 2 * v) = __float2bfloat16_rn(x[i]);
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bar[OF + b]);
+            // A whole chunk, or a partial one that ends the tensor (TMA clips the rows past it), goes out
+            // as one bulk tensor store; a partial chunk followed by another sequence's tokens is copied
+            // row by row so that those tokens' outputs are not overwritten.
+            if (L == C || cs + L >= T_tot) {
+                tc::fence_smem_to_async();
+                tc::named_sync(1, 128);
+                if (v == 0) tc::tma_store_3d(&tm_o, sb + OST, 0, h, cs);
+            } else {
+                tc::named_sync(1, 128);
+#pragma unroll
+                for (int it = 0; it < 8; ++it) {
+                    const int idx = it * 128 + v, r = idx >> 4, j = idx & 15;
+                    if (r < L)
+                        *reinterpret_cast<uint4 *>(o + ((size_t)(cs + r) * H + h) * D + 8 * j) =
+                            *reinterpret_cast<const uint4 *>(ost + r * 256 + j * 16);
+                }
+            }
+        }
+        if (v == 0) tc::bulk_wait_all();
+    }
+    if (warp == W_MMA && lane == 0) {
+        tc::mma_commit(&bar[FIN]);
+        drain_bar(&bar[FIN], 0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+// ============================================================================ transition pass + link
+namespace tb {
+constexpr uint32_t B_K = 0, B_V = 16384, B_T2 = 32768, B_VEC = 40960;
+constexpr uint32_t BUF = 41984;
+constexpr uint32_t T1 = 2 * BUF;
+constexpr uint32_t W = T1 + 8192;
+constexpr uint32_t S = W + 16384;
+constexpr uint32_t X = S + 32768;
+constexpr uint32_t DTS = X + 32768;
+constexpr uint32_t DTX = DTS + 16384;
+constexpr uint32_t BAR = DTX + 16384;
+constexpr uint32_t TOTAL = BAR + 256;
+// link phase (after the chunk loop, the buffers are free)
+constexpr uint32_t PHI = 0;      // Phi hi | lo as B operands (rows k, runs along k'; sy = 2048)
+constexpr uint32_t SIN = 65536;  // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
+// TMEM columns
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
+enum {
+    FULL = 0, EMPTY = 2, WUF = 4, M3S = 5, M4S = 6, M3X = 7, M4X = 8,
+    T1R = 9,    // prep (128)
+    WR = 10,    // prep (128)
+    SR = 11,    // state S (128)
+    XR = 12,    // state X (128)
+    DSR = 13,   // state S (128)
+    DXR = 14,   // state X (128)
+    LNK = 15,   // S_in tiles landed
+    LMMA = 16,  // link MMAs done
+    FIN = 17,   // every MMA of the CTA done (drained before TMEM is freed)
+    NBAR = 18
+};
+}  // namespace tb
+
+__global__ void __launch_bounds__(NT_WS, 1)
+    k_ws_trans(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const float *S0,
+               const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
+               const int32_t *__restrict__ seg_off, const int32_t *__restrict__ chunk_off, int seg_chunks,
+               const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags) {
+    using namespace tb;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (*err & ERRBIT_SEQLENS) return;
+    Segment sg;
+    const int h = blockIdx.x;
+    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg)) return;
+    if (sg.s == sg.ns - 1) return;  // the last segment's end state is never needed
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sb = tc::smem_u32(smem);
+    const int gseg = blockIdx.y;
+    uint32_t *my_flag = flags + (size_t)gseg * H + h;
+    if (sb & 1023u) {
+        if (tid == 0) {
+            atomicOr(err, ERRBIT_INTERNAL);
+            tc::st_release_gpu(my_flag, FLAG_FAILED);
+        }
+        return;
+    }
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + BAR);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + BAR + 8 * NBAR);
+    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
+    if (tid == 0) {
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i >= T1R && i <= DXR) ? 128u : 1u);
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    const int nch = (sg.b - sg.a + C - 1) / C;
+    const bool has_x = sg.s > 0;  // the first segment starts from S0 and needs no Phi
+    const size_t sidx = ((size_t)sg.n * H + h) * D * D;
+    auto buf = [&](int c) { return sb + (uint32_t)(c & 1) * BUF; };
+    auto vecp = [&](int c) { return reinterpret_cast<const float *>(smem + (c & 1) * BUF + B_VEC); };
+
+    if (warp == W_LOAD) {
+        if (lane == 0) {
+            int issued = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                if (c >= 2 && !wait_bar(&bar[EMPTY + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err)) break;
+                const uint32_t bb = buf(c);
+                const int cs = sg.a + c * C;
+                tc::mbar_arrive_expect_tx(&bar[FULL + b], 2u * 16384u + REC_BYTES);
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    tc::tma_load_3d(bb + B_K + hf * 8192, &tm_k, &bar[FULL + b], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_V + hf * 8192, &tm_v, &bar[FULL + b], 64 * hf, h, cs);
+                }
+                tc::bulk_load(bb + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES, REC_BYTES,
+                              &bar[FULL + b]);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], (uint32_t)((c >> 1) & 1));
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0 && nch > 0) {
+            const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+            const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
+            const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            auto issue_wu = [&](int c) {
+                const uint32_t bb = buf(c);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024),
+                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
+                                 tc::make_desc(bb + B_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                }
+                tc::mma_commit(&bar[WUF]);
+            };
+            bool ok = wait_bar(&bar[FULL], 0, ctl, err) && wait_bar(&bar[T1R], 0, ctl, err);
+            if (ok) {
+                tc::fence_after_sync();
+                issue_wu(0);
+            }
+            for (int c = 0; ok && c < nch; ++c) {
+                const int b = c & 1;
+                const uint32_t par = (uint32_t)(c & 1), bb = buf(c);
+                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
+                tc::mma_commit(&bar[M3S]);
+                if (has_x) {
+                    if (!(ok = wait_bar(&bar[XR], par, ctl, err))) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        tc::mma_bf16(tm + TM_DX, tc::make_desc(sb + X + kk * 4096, 2048, 128),
+                                     tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
+                    tc::mma_commit(&bar[M3X]);
+                }
+                if (c + 1 < nch) {
+                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err) &&
+                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
+                        break;
+                    tc::fence_after_sync();
+                    issue_wu(c + 1);
+                }
+                if (!(ok = wait_bar(&bar[DSR], par, ctl, err))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DTS + kk * 4096, 2048, 128),
+                                 tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                tc::mma_commit(&bar[M4S]);
+                if (has_x) {
+                    if (!(ok = wait_bar(&bar[DXR], par, ctl, err))) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        tc::mma_bf16(tm + TM_X, tc::make_desc(sb + DTX + kk * 4096, 2048, 128),
+                                     tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                    tc::mma_commit(&bar[M4X]);
+                }
+                tc::mma_commit(&bar[EMPTY + b]);
+            }
+        }
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- S state (warps 0-3), X state (4-7)
+        const bool is_x = warp >= 4;
+        if (!is_x || has_x) {
+            const int v = tid & 127;
+            const uint32_t tl = lane_base(tm, warp);
+            const uint32_t s_tile = sb + (is_x ? X : S), dt_tile = sb + (is_x ? DTX : DTS);
+            const uint32_t tm_state = is_x ? TM_X : TM_S;
+            uint64_t *b_r = &bar[is_x ? XR : SR], *b_d = &bar[is_x ? DXR : DSR];
+            uint64_t *b_m3 = &bar[is_x ? M3X : M3S], *b_m4 = &bar[is_x ? M4X : M4S];
+            bool ok = nch > 0 && wait_bar(&bar[FULL], 0, ctl, err);
+            if (ok) {
+                const float g0 = vecp(0)[64 + C - 1];
+                const float *src = (!is_x && sg.s == 0 && S0) ? S0 + sidx + (size_t)v * D : nullptr;
+                state_init(s_tile, tl + tm_state, v, g0, src, nullptr, is_x);
+                handoff(b_r);
+            }
+            for (int c = 0; ok && c < nch; ++c) {
+                const int b = c & 1;
+                if (!(ok = wait_bar(b_m3, (uint32_t)(c & 1), ctl, err))) break;
+                tc::fence_after_sync();
+                tile64_epilogue(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * b), v);
+                handoff(b_d);
+                if (!(ok = wait_bar(b_m4, (uint32_t)(c & 1), ctl, err))) break;
+                tc::fence_after_sync();
+                const bool last = c + 1 == nch;
+                float g1 = 1.f;
+                if (!last) {
+                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
+                    g1 = vecp(c + 1)[64 + C - 1];
+                }
+                state_epilogue(s_tile, tl + tm_state, v, g1, last, nullptr);
+                if (!last) handoff(b_r);
+            }
+        }
+    } else if (warp < 12) {
+        // ---------------------------------------------------------------- prep
+        const int t128 = tid - 256;
+        const uint32_t tl = lane_base(tm, warp);
+        bool ok = true;
+        for (int c = 0; ok && c < nch; ++c) {
+            const int b = c & 1;
+            uint8_t *bp = smem + b * BUF;
+            const float *vec = vecp(c);
+            if (!(ok = wait_bar(&bar[FULL + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            make_t1(smem + T1, bp + B_T2, vec + 64, t128);
+            tc::fence_smem_to_async();
+            tc::mbar_arrive(&bar[T1R]);
+            if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            neg_w_epilogue(sb + W, tl + TM_WT, t128);
+            scale_rows_sw128(bp + B_K, vec + 128, t128);
+            handoff(&bar[WR]);
+        }
+    }
+    // ---------------------------------------------------------------- link (all threads)
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    bool ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
+    if (ok && has_x) {
+        // Phi = X_end as bf16 hi / lo B-operand tiles (X warps), S_in from the previous segment (loader)
+        if (warp >= 4 && warp < 8) {
+            const int k = tid - 128;
+            const uint32_t tl = lane_base(tm, warp);
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                float x[32], hi[32], lo[32];
+                tc::tmem_ld32(tl + TM_X + c0, x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+                    lo[i] = x[i] - hi[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    st_run8(sb + PHI + tc::tile_off(k, c0 + i, 128, 2048), hi + i);
+                    st_run8(sb + PHI + 32768 + tc::tile_off(k, c0 + i, 128, 2048), lo + i);
+                }
+            }
+            tc::fence_smem_to_async();
+        }
+        if (warp == W_LOAD && lane == 0) {
+            const uint32_t *prev = flags + (size_t)(gseg - 1) * H + h;
+            const uint64_t t0 = tc::globaltimer();
+            uint32_t f = 0;
+            while ((f = tc::ld_acquire_gpu(prev)) == 0) {
+                if (tc::globaltimer() - t0 > kWaitNs) break;
+                __nanosleep(64);
+            }
+            if (f == FLAG_DONE) {
+                tc::fence_proxy_async_global();
+                tc::mbar_arrive_expect_tx(&bar[LNK], LINK_BYTES);
+                tc::bulk_load(sb + SIN, link + ((size_t)(gseg - 1) * H + h) * LINK_BYTES, LINK_BYTES, &bar[LNK]);
+            } else {
+                if (f == 0) atomicOr(err, ERRBIT_TIMEOUT);
+                ctl->abort = 1;
+            }
+        }
+        tc::fence_before_sync();
+        __syncthreads();
+        tc::fence_after_sync();
+        ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort);
+        if (ok && warp == W_MMA && lane == 0) {
+            // S_end = S_loc + S_in Phi = S_loc + S_in_hi Phi_hi + S_in_hi Phi_lo + S_in_lo Phi_hi
+            if (wait_bar(&bar[LNK], 0, ctl, err)) {
+                const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
+                    const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
+                    const uint64_t bh = tc::make_desc(sb + PHI + kk * 256, 128, 2048);
+                    const uint64_t bl = tc::make_desc(sb + PHI + 32768 + kk * 256, 128, 2048);
+                    tc::mma_bf16(tm + TM_S, ah, bh, id_km128, 1);
+                    tc::mma_bf16(tm + TM_S, ah, bl, id_km128, 1);
+                    tc::mma_bf16(tm + TM_S, al, bh, id_km128, 1);
+                }
+                tc::mma_commit(&bar[LMMA]);
+            }
+        }
+        if (ok && warp < 4) ok = wait_bar(&bar[LMMA], 0, ctl, err);
+        if (warp == W_LOAD && lane == 0 && ok) drain_bar(&bar[LNK], 0);
+    }
+    // publish S_end (S warps): bf16 hi / lo tiles in the link slot, then the flag
+    if (ok && warp < 4) {
+        tc::fence_after_sync();
+        const int v = tid;
+        const uint32_t tl = lane_base(tm, warp);
+        uint8_t *dst = link + ((size_t)gseg * H + h) * LINK_BYTES;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+            float x[32];
+            tc::tmem_ld32(tl + TM_S + c0, x);
+#pragma unroll
+            for (int i = 0; i < 32; i += 8) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float h0 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j]));
+                    const float h1 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j + 1]));
+                    hw[j] = tc::pack_bf16x2(h0, h1);
+                    lw[j] = tc::pack_bf16x2(x[i + 2 * j] - h0, x[i + 2 * j + 1] - h1);
+                }
+                const uint32_t off = tc::tile_off(v, c0 + i, 128, 2048);
+                *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                *reinterpret_cast<uint4 *>(dst + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            }
+        }
+        __threadfence();
+    }
+    if (warp == W_MMA && lane == 0) {
+        tc::mma_commit(&bar[FIN]);
+        drain_bar(&bar[FIN], 0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+        const bool good = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
+        tc::st_release_gpu(my_flag, good ? FLAG_DONE : FLAG_FAILED);
+        if (!good) atomicOr(err, ERRBIT_TIMEOUT);
+    }
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+// ============================================================================ plan
+// Validates cu_seqlens (error word), writes seg_off[0..N] (exclusive prefix of
+// max(1, ceil(ceil(L_n / C) / seg_chunks)), or of 1 with seg_chunks = 0),
+// chunk_off[0..N] (exclusive prefix of ceil(L_n / C)) and clears nflags flags.
+__global__ void __launch_bounds__(256) k_ws_plan(const int32_t *__restrict__ cu, int N, int T_tot, int seg_chunks,
+                                                 uint32_t *__restrict__ err, int32_t *__restrict__ seg_off,
+                                                 int32_t *__restrict__ chunk_off, uint32_t *__restrict__ flags,
+                                                 int nflags) {
+    __shared__ int ps[256], pc[256];
+    __shared__ int bad;
+    const int tid = threadIdx.x;
+    if (tid == 0) bad = 0;
+    for (int i = tid; i < nflags; i += 256) flags[i] = 0u;
+    __syncthreads();
+    const int per = (N + 255) / 256;
+    const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
+    auto nchunks = [&](int n) {
+        int L = cu ? cu[n + 1] - cu[n] : T_tot / N;
+        L = max(L, 0);
+        return (L + C - 1) / C;
+    };
+    auto nseg = [&](int n) { return seg_chunks > 0 ? max(1, (nchunks(n) + seg_chunks - 1) / seg_chunks) : 1; };
+    int ssum = 0, csum = 0;
+    bool b = false;
+    for (int n = n0; n < n1; ++n) {
+        if (cu) b |= cu[n + 1] < cu[n];
+        ssum += nseg(n);
+        csum += nchunks(n);
+    }
+    if (tid == 0 && cu) b |= (cu[0] != 0) || (cu[N] != T_tot);
+    if (b) atomicOr(&bad, 1);
+    ps[tid] = ssum;
+    pc[tid] = csum;
+    __syncthreads();
+    if (tid == 0) {
+        int as = 0, ac = 0;
+        for (int i = 0; i < 256; ++i) {
+            const int xs = ps[i], xc = pc[i];
+            ps[i] = as;
+            pc[i] = ac;
+            as += xs;
+            ac += xc;
+        }
+        seg_off[N] = as;
+        chunk_off[N] = bad ? 0 : ac;
+        *err = bad ? ERRBIT_SEQLENS : 0u;
+    }
+    __syncthreads();
+    int as = ps[tid], ac = pc[tid];
+    for (int n = n0; n < n1; ++n) {
+        seg_off[n] = as;
+        chunk_off[n] = ac;
+        as += nseg(n);
+        ac += nchunks(n);
+    }
+}
+
+int num_sms() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    });
+    return n;
+}
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct WsLayout {
+    size_t seg_off, chunk_off, flags, s0copy, rec, link, total;
+    int nslots, nc_bound;
+};
+
+// Workspace regions (byte offsets; the first 256 bytes hold the error word).
+WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
+    WsLayout l;
+    l.nc_bound = (int)(((long)T_tot + (long)(C - 1) * N) / C);
+    l.nslots = seg_chunks > 0 ? (int)(l.nc_bound / seg_chunks + N) : N;
+    l.seg_off = 256;
+    l.chunk_off = l.seg_off + align256((size_t)(N + 1) * 4);
+    l.flags = l.chunk_off + align256((size_t)(N + 1) * 4);
+    l.s0copy = l.flags + align256((size_t)l.nslots * H * 4);
+    l.rec = l.s0copy + (seg_chunks > 0 ? (size_t)N * H * D * D * sizeof(float) : 0);
+    l.link = l.rec + align256((size_t)l.nc_bound * H * REC_BYTES);
+    l.total = l.link + (seg_chunks > 0 ? (size_t)l.nslots * H * LINK_BYTES : 0);
+    return l;
+}
+
+}  // namespace
+
+// Segment length (in chunks) for the pipelined path, 0 = one segment per
+// sequence. Splitting pays when few (sequence, head) pairs leave SMs idle: the
+// segments of a sequence run their chunks concurrently, at the cost of the
+// transition pass and one link per segment boundary on the critical path.
+// Time ~ n/s (t_trans + t_out) + (s - 1) t_link is smallest near s = sqrt(n)
+// (measured per chunk ~ t_link), capped so that all CTAs fit on the GPU at once.
+int chunk_ws_seg_chunks(int N, int T_tot, int H) {
+    const long pairs = (long)N * H;
+    const long nc_avg = ((long)T_tot / N + C - 1) / C;
+    const int sms = num_sms();
+    if (pairs * 2 > sms || nc_avg < 8) return 0;
+    long s = 1;
+    while ((s + 1) * (s + 1) <= nc_avg) ++s;  // floor(sqrt(nc_avg))
+    s = std::min(s, (long)sms / pairs);
+    if (s < 2) return 0;
+    return (int)((nc_avg + s - 1) / s);
+}
+
+size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks) { return ws_layout(N, T_tot, H, seg_chunks).total; }
+
+cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
+                            const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
+                            void *workspace, int seg_chunks, cudaStream_t st, const char **stage) {
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    uint32_t *err = static_cast<uint32_t *>(workspace);
+    const WsLayout l = ws_layout(N, T_tot, H, seg_chunks);
+    int32_t *seg_off = reinterpret_cast<int32_t *>(wsb + l.seg_off);
+    int32_t *chunk_off = reinterpret_cast<int32_t *>(wsb + l.chunk_off);
+    uint32_t *flags = reinterpret_cast<uint32_t *>(wsb + l.flags);
+    uint8_t *rec = wsb + l.rec, *link = wsb + l.link;
+    CUtensorMap tm_q, tm_k, tm_v, tm_o;
+    cudaError_t e;
+    *stage = "TMA descriptor encoding";
+    if ((e = make_row_map(&tm_o, o, H, T_tot, true)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tm_q, q, H, T_tot)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tm_k, k, H, T_tot)) != cudaSuccess) return e;
+    if ((e = make_row_map(&tm_v, v, H, T_tot)) != cudaSuccess) return e;
+    // With segments, the output pass of a sequence's first segment reads S0 while its last
+    // segment writes S_T: if the two overlap, read S0 from a snapshot.
+    if (seg_chunks > 0 && S0) {
+        const size_t bytes = (size_t)N * H * D * D * sizeof(float);
+        const uint8_t *a = reinterpret_cast<const uint8_t *>(S0), *b = reinterpret_cast<const uint8_t *>(S_T);
+        if (a < b + bytes && b < a + bytes) {
+            *stage = "S0 snapshot";
+            if ((e = cudaMemcpyAsync(wsb + l.s0copy, S0, bytes, cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
+            S0 = reinterpret_cast<const float *>(wsb + l.s0copy);
+        }
+    }
+    *stage = "plan";
+    void *pr = prof_start("ws_plan", st);
+    const int nflags = seg_chunks > 0 ? l.nslots * H : 0;
+    k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
+    prof_stop(pr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (T_tot == 0 && seg_chunks == 0) {
+        // nothing to prepare; the output pass still writes S_T = S0
+    } else {
+        *stage = "ws_prep";
+        e = cudaFuncSetAttribute(k_ws_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pp::TOTAL);
+        if (e != cudaSuccess) return e;
+        const long items_bound = (long)l.nc_bound * H;
+        const int grid = (int)std::max(1L, std::min(items_bound, 3L * num_sms()));
+        pr = prof_start("ws_prep", st);
+        k_ws_prep<<<grid, 256, pp::TOTAL, st>>>(tm_k, g, beta, cu, N, T_tot, H, err, chunk_off, rec);
+        prof_stop(pr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (seg_chunks > 0) {
+        *stage = "ws_trans";
+        e = cudaFuncSetAttribute(k_ws_trans, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb::TOTAL);
+        if (e != cudaSuccess) return e;
+        pr = prof_start("ws_trans", st);
+        k_ws_trans<<<dim3(H, l.nslots), NT_WS, tb::TOTAL, st>>>(tm_k, tm_v, S0, cu, N, T_tot, H, err, seg_off,
+                                                                 chunk_off, seg_chunks, rec, link, flags);
+        prof_stop(pr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    *stage = "ws_out";
+    e = cudaFuncSetAttribute(k_ws_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ob::TOTAL);
+    if (e != cudaSuccess) return e;
+    pr = prof_start("ws_out", st);
+    k_ws_out<<<dim3(H, l.nslots), NT_WS, ob::TOTAL, st>>>(tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot, H, o, S_T, err,
+                                                          seg_chunks > 0 ? seg_off : nullptr, chunk_off,
+                                                          seg_chunks > 0 ? seg_chunks : 1, rec, link);
+    prof_stop(pr);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -34,6 +34,17 @@ cudaError_t launch_chunk_tc(const __nv_bfloat16 *q, const __nv_bfloat16 *k, cons
 int chunk_tc_seg_chunks(int N, int T_tot, int H);
 size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks);
 
+// Pipelined tensor-core chunked forward (same contract as launch_chunk_tc):
+// plan, the parallel prep pass (decay scalars and UT solve of every chunk),
+// the transition pass with its links (seg_chunks > 0 only) and the output
+// pass. Needs chunk_ws_workspace(N, T_tot, H, seg_chunks) bytes of workspace.
+cudaError_t launch_chunk_ws(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const float *g,
+                            const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
+                            __nv_bfloat16 *o, float *S_T, void *workspace, int seg_chunks, cudaStream_t st,
+                            const char **stage);
+int chunk_ws_seg_chunks(int N, int T_tot, int H);
+size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks);
+
 // Kernel timing hooks (no-ops unless gdn_profile_enable(1)): an event pair
 // around the launches between prof_start and prof_stop, recorded on st.
 void *prof_start(const char *name, cudaStream_t st);

@@ -64,7 +64,9 @@ __device__ __forceinline__ void warp_store(float *Z, int p, const float (&d)[4],
 
 // Block-wide solve; requires blockDim.x == 256. A, T: [64][AP] fp32 in shared
 // memory (A zero on and above the diagonal). X: scratch of 32 * XP floats.
-// Ends with a __syncthreads.
+// T may be the same buffer as A: every block of A is read (and the reads
+// synchronised) before the block of T at its place is written. Ends with a
+// __syncthreads.
 __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // ---- 1. diagonal blocks (warps 0-3) and the zero upper blocks (warps 4-7)
@@ -79,6 +81,7 @@ __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
                 for (int s = 0; s < i; ++s) acc = fmaf(-A[(o + i) * AP + o + s], x[s], acc);
                 x[i] = acc;
             }
+            __syncwarp(0x0000ffffu);  // every lane has read its block of A before T overwrites it (A may be T)
 #pragma unroll
             for (int i = 0; i < 16; ++i) T[(o + i) * AP + o + j] = x[i];
         }
