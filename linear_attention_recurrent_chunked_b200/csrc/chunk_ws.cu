@@ -10,14 +10,15 @@
 //   T1 = T diag(beta gamma),  T2 = T diag(beta)
 //   W^T = K^T T1^T,  U^T = V^T T2^T
 //   Delta^T = U^T - S W^T
-//   O^T = S (diag(gamma) Q)^T + Delta^T P^T,  P_rs = exp(G_r - G_s)(q_r . k_s), s <= r
+//   O^T = diag-scaled O1 + O2:  O1 = S Q^T (column r times gamma_r),  O2 = Delta^T P^T,
+//         P_rs = exp(G_r - G_s)(q_r . k_s) for s <= r
 //   S  <- gamma_C S + Delta^T (diag(e) K)
 //
 // Work is split three ways:
 //  1. k_ws_prep, over every (chunk, head) in parallel (several CTAs per SM):
 //     the state-independent scalars and the UT solve. One 9 KB record per
 //     (chunk, head): T2 as a ready bf16 operand tile, then G (log2 units),
-//     gamma, e and beta.
+//     gamma, e and beta (T1 = T2 diag(gamma) is rebuilt on chip).
 //  2. k_ws_trans, one CTA per segment except the last of its sequence (only
 //     when a sequence is split into segments that run concurrently): runs the
 //     segment from S = 0 (S_loc) and, on a second state, from X = I with the
@@ -30,17 +31,17 @@
 //     state of the previous segment and writes the outputs (and S_T).
 //
 // In 2 and 3 the warps have fixed roles and pass tiles to each other through
-// mbarriers, so that the next chunk's loads and operand preparation overlap
-// the current chunk's dependent state step:
+// mbarriers, so that the next chunk's loads and operand preparation and the
+// current chunk's outputs overlap the dependent state step:
 //   loader (1 thread)  K, Q, V by TMA (128-byte swizzle), the record by bulk copy
-//   MMA    (1 thread)  every tcgen05.mma, in an order that keeps the chain first
-//   prep   (4 warps)   T1 from T2; P from X1 = Q K^T; Q <- diag(gamma) Q and
-//                      K <- diag(e) K in place; -W from W^T
-//   state  (4 warps)   Delta^T (accumulated on top of U^T in TMEM) -> bf16 tile;
-//                      S -> bf16 tile, and S <- gamma_C' S in TMEM so that the
-//                      next update accumulates onto it
-//   output (4 warps)   O^T -> bf16 rows -> TMA store  (k_ws_out)
-//   X-state (4 warps)  the Phi chain                   (k_ws_trans)
+//   MMA    (1 thread)  every tcgen05.mma; the state step's two MMAs are issued
+//                      as soon as their inputs are ready, the rest fills in after
+//   state  (8 warps)   Delta^T (accumulated onto U^T in TMEM) -> bf16 tile;
+//                      S -> bf16 tile and S <- gamma_C' S in TMEM, so that the
+//                      next update accumulates onto it (two threads per row)
+//   prep   (8 / 4 warps) T1 from T2; -W from W^T; P from X1 = Q K^T; K <- diag(e) K in place
+//   output (4 warps)   gamma_r O1 + O2 -> bf16 rows -> TMA store   (k_ws_out)
+//   X-state (8 warps)  the Phi chain                               (k_ws_trans)
 // Every wait is bounded in time; a timeout sets the error word and makes all
 // roles of the CTA leave their loops.
 #include "chunk_common.cuh"
@@ -66,9 +67,9 @@ constexpr uint32_t REC_BYTES = 9216;
 constexpr uint32_t LINK_BYTES = 65536;
 constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 
-// Warp roles of the pipelined kernels (448 threads).
-constexpr int NT_WS = 448;
-constexpr int W_LOAD = 12, W_MMA = 13;
+// Warp roles of the pipelined kernels (22 warps).
+constexpr int NT_WS = 704;
+constexpr int W_LOAD = 20, W_MMA = 21;
 
 struct Ctl {
     uint32_t tmem;   // TMEM base written by tcgen05.alloc
@@ -102,12 +103,12 @@ __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
 __device__ __forceinline__ uint32_t lane_base(uint32_t tm, int warp) { return tm + ((uint32_t)((warp & 3) * 32) << 16); }
 
 // Scale the 64 rows of a 128-byte-swizzled 64 x 128 bf16 tile (two 8 KB column
-// halves) by f[row], in place. The swizzle only permutes 16-byte chunks within
-// a row, so a chunk's row is its offset within the half / 128. 128 threads.
-__device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, int t128) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int idx = t128 + 128 * i, row = (idx & 511) >> 3;
+// halves) by f[row], in place, with n threads (t = 0..n-1). The swizzle only
+// permutes 16-byte chunks within a row, so a chunk's row is its offset within
+// the half / 128.
+__device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, int t, int n) {
+    for (int idx = t; idx < 1024; idx += n) {
+        const int row = (idx & 511) >> 3;
         uint4 *p = reinterpret_cast<uint4 *>(tile + 16 * idx);
         uint4 x = *p;
         const float s = f[row];
@@ -121,11 +122,10 @@ __device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, 
     }
 }
 
-// T1 = T2 diag(gamma) between two 64 x 64 bf16 tiles (rows r, runs along s; sy = 1024). 128 threads.
-__device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t128) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int idx = t128 + 128 * i, s0 = 8 * (idx >> 6);
+// T1 = T2 diag(gamma) between two 64 x 64 bf16 tiles (rows r, runs along s; sy = 1024), n threads.
+__device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t, int n) {
+    for (int idx = t; idx < 512; idx += n) {
+        const int s0 = 8 * (idx >> 6);
         uint4 x = *reinterpret_cast<const uint4 *>(t2 + 16 * idx);
         uint32_t *w = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
@@ -137,67 +137,59 @@ __device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const fl
     }
 }
 
-// -W tile (rows k, runs along r; sx = 128, sy = 2048) from this thread's TMEM lane k of W^T (64 columns).
-__device__ __forceinline__ void neg_w_epilogue(uint32_t w_tile, uint32_t tl_wt, int k) {
+// bf16 tile (rows = this thread's TMEM lane, 16-byte runs along 32 columns from
+// col0; sx = 128, sy = 2048) from 32 accumulator columns, times `scale`.
+__device__ __forceinline__ void tile32_epilogue(uint32_t tile, uint32_t taddr, int row, int col0, float scale) {
+    float x[32];
+    tc::tmem_ld32(taddr, x);
 #pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 32) {
-        float x[32];
-        tc::tmem_ld32(tl_wt + c0, x);
+    for (int i = 0; i < 32; ++i) x[i] *= scale;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = -x[i];
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) st_run8(w_tile + tc::tile_off(k, c0 + i, 128, 2048), x + i);
-    }
+    for (int i = 0; i < 32; i += 8) st_run8(tile + tc::tile_off(row, col0 + i, 128, 2048), x + i);
 }
 
-// bf16 tile (rows v, runs along the 64 columns; sx = 128, sy = 2048) from this thread's TMEM lane v.
-__device__ __forceinline__ void tile64_epilogue(uint32_t tile, uint32_t tl, int v) {
-#pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 32) {
-        float x[32];
-        tc::tmem_ld32(tl + c0, x);
-#pragma unroll
-        for (int i = 0; i < 32; i += 8) st_run8(tile + tc::tile_off(v, c0 + i, 128, 2048), x + i);
-    }
-}
-
-// The state step after the update MMA: read row v of S (fp32, 128 columns) from
-// TMEM, write its bf16 copy to the S tile and S * g_next back to TMEM (the
-// next update accumulates onto gamma_C S). With last set, nothing is written
-// back and the row goes to dst_row (fp32, global) if given.
-__device__ __forceinline__ void state_epilogue(uint32_t s_tile, uint32_t tl_s, int v, float g_next, bool last,
-                                               float *dst_row) {
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-        float x[32];
-        tc::tmem_ld32(tl_s + c0, x);
+// The state step after the update MMA, for 64 columns [c_begin, c_begin + 64)
+// of row v: read S from TMEM, write its bf16 copy to the S tile and S * g_next
+// back to TMEM (the next update accumulates onto gamma_C S). With last set,
+// nothing is written back and the row goes to dst_row (fp32, global) if given.
+// The second 32-column load is in flight while the first is processed.
+__device__ __forceinline__ void state_epilogue64(uint32_t s_tile, uint32_t tl_s, int v, int c_begin, float g_next,
+                                                 bool last, float *dst_row) {
+    uint32_t a[32], b[32];
+    tc::tmem_ld32_nowait(tl_s + c_begin, a);
+    tc::tmem_wait_ld(a);
+    tc::tmem_ld32_nowait(tl_s + c_begin + 32, b);
+    auto process = [&](uint32_t(&u)[32], int c0) {
+        float *x = reinterpret_cast<float *>(u);
         if (!last) {
 #pragma unroll
             for (int i = 0; i < 32; i += 8) st_run8(s_tile + tc::tile_off(v, c0 + i, 128, 2048), x + i);
 #pragma unroll
             for (int i = 0; i < 32; ++i) x[i] *= g_next;
-            tc::tmem_st16(tl_s + c0, *reinterpret_cast<float(*)[16]>(x));
-            tc::tmem_st16(tl_s + c0 + 16, *reinterpret_cast<float(*)[16]>(x + 16));
+            tc::tmem_st32(tl_s + c0, u);
         } else if (dst_row) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
                 *reinterpret_cast<float4 *>(dst_row + c0 + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
         }
-    }
+    };
+    process(a, c_begin);
+    tc::tmem_wait_ld(b);
+    process(b, c_begin + 32);
     if (!last) tc::tmem_st_wait();
 }
 
-// Initial state row v: fp32 values from src_f32 (row-major, may be null: zeros),
-// or from a published hi/lo tile pair (link, may be null), or the identity row.
-// Written as g0 * S to TMEM and as bf16 to the tile.
-__device__ __forceinline__ void state_init(uint32_t s_tile, uint32_t tl_s, int v, float g0, const float *src_f32,
-                                           const uint8_t *link, bool identity) {
+// Initial state, columns [c_begin, c_begin + 64) of row v: fp32 values from
+// src_row (may be null: zeros), or from a published hi/lo tile pair (link, may
+// be null), or the identity row. Written as g0 * S to TMEM and as bf16 to the tile.
+__device__ __forceinline__ void state_init64(uint32_t s_tile, uint32_t tl_s, int v, int c_begin, float g0,
+                                             const float *src_row, const uint8_t *link, bool identity) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 16) {
-        float x[16];
-        if (link) {
+    for (int c0 = c_begin; c0 < c_begin + 64; c0 += 32) {
+        float x[32];
 #pragma unroll
-            for (int h8 = 0; h8 < 16; h8 += 8) {
+        for (int h8 = 0; h8 < 32; h8 += 8) {
+            if (link) {
                 const uint32_t off = tc::tile_off(v, c0 + h8, 128, 2048);
                 uint4 hi = *reinterpret_cast<const uint4 *>(link + off);
                 uint4 lo = *reinterpret_cast<const uint4 *>(link + 32768 + off);
@@ -205,30 +197,46 @@ __device__ __forceinline__ void state_init(uint32_t s_tile, uint32_t tl_s, int v
                 const uint32_t *wl = reinterpret_cast<const uint32_t *>(&lo);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wh[j]));
-                    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wl[j]));
-                    x[h8 + 2 * j] = a.x + b.x;
-                    x[h8 + 2 * j + 1] = a.y + b.y;
+                    const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wh[j]));
+                    const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wl[j]));
+                    x[h8 + 2 * j] = p.x + q.x;
+                    x[h8 + 2 * j + 1] = p.y + q.y;
                 }
-            }
-        } else {
+            } else {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-                float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (src_f32) a = *reinterpret_cast<const float4 *>(src_f32 + c0 + i);
-                x[i] = a.x; x[i + 1] = a.y; x[i + 2] = a.z; x[i + 3] = a.w;
-            }
-            if (identity)
+                for (int i = 0; i < 8; i += 4) {
+                    float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (src_row) p = *reinterpret_cast<const float4 *>(src_row + c0 + h8 + i);
+                    x[h8 + i] = p.x; x[h8 + i + 1] = p.y; x[h8 + i + 2] = p.z; x[h8 + i + 3] = p.w;
+                }
+                if (identity)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[i] = (c0 + i == v) ? 1.f : 0.f;
+                    for (int i = 0; i < 8; ++i) x[h8 + i] = (c0 + h8 + i == v) ? 1.f : 0.f;
+            }
         }
-        st_run8(s_tile + tc::tile_off(v, c0, 128, 2048), x);
-        st_run8(s_tile + tc::tile_off(v, c0 + 8, 128, 2048), x + 8);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] *= g0;
-        tc::tmem_st16(tl_s + c0, x);
+        for (int i = 0; i < 32; i += 8) st_run8(s_tile + tc::tile_off(v, c0 + i, 128, 2048), x + i);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] *= g0;
+        tc::tmem_st32(tl_s + c0, *reinterpret_cast<uint32_t(*)[32]>(x));
     }
     tc::tmem_st_wait();
+}
+
+// bf16 hi / lo split of 32 values of row `row` into two tiles (sx = 128, sy = 2048)
+// in shared memory (hi at base, lo at base + 32 KB).
+__device__ __forceinline__ void st_split32(uint32_t base, int row, int c0, const float *x) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+        float hi[8], lo[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            hi[j] = __bfloat162float(__float2bfloat16_rn(x[i + j]));
+            lo[j] = x[i + j] - hi[j];
+        }
+        st_run8(base + tc::tile_off(row, c0 + i, 128, 2048), hi);
+        st_run8(base + 32768 + tc::tile_off(row, c0 + i, 128, 2048), lo);
+    }
 }
 
 // Signal an mbarrier after this thread's shared-memory writes (for the tensor
@@ -288,7 +296,7 @@ __global__ void __launch_bounds__(256, 3)
     float *vec = reinterpret_cast<float *>(smem + pp::REC + REC_VEC);
     float *Gl = vec, *gam = vec + 64, *dte = vec + 128, *bet = vec + 192;
 
-    // where item w lives: sequence n, chunk start cs, valid length L
+    // where item w lives: head h, chunk start cs, valid length L, global chunk gc
     auto locate = [&](int w, int &h, int &cs, int &L, int &gc) {
         gc = w / H;
         h = w - gc * H;
@@ -394,7 +402,7 @@ __global__ void __launch_bounds__(256, 3)
         tc::fence_before_sync();
         __syncthreads();
         ut::solve64(AT, AT, reinterpret_cast<float *>(smem + pp::XS));
-        // ---- T2 = T diag(beta) as a bf16 operand tile (thread: row tid / 4, columns 16 (tid % 4) ..)
+        // ---- T2 = T diag(beta) as a bf16 operand tile (thread: row tid / 4, 16 columns)
         {
             const int r = tid >> 2, s0 = 16 * (tid & 3);
             float x[16];
@@ -425,34 +433,37 @@ __global__ void __launch_bounds__(256, 3)
 // ============================================================================ output pass
 namespace ob {
 constexpr uint32_t B_K = 0, B_Q = 16384, B_V = 32768, B_T2 = 49152, B_VEC = 57344;
-constexpr uint32_t BUF = 58368;  // one input buffer (K, Q, V tiles; the record); two of them
-constexpr uint32_t T1 = 2 * BUF;
-constexpr uint32_t P = T1 + 8192;    // two P tiles (rows r, runs along s; sy = 1024)
-constexpr uint32_t W = P + 16384;    // -W tile (rows k, runs along r; sy = 2048)
-constexpr uint32_t S = W + 16384;    // bf16 state (rows v, runs along k; sy = 2048)
-constexpr uint32_t DL = S + 32768;   // Delta^T bf16 (rows v, runs along s; sy = 2048)
-constexpr uint32_t OST = DL + 16384; // output staging: 64 rows o[r][0..127] bf16
+constexpr uint32_t BUF = 58368;       // one input buffer (K, Q, V tiles; the record); two of them
+constexpr uint32_t T1 = 2 * BUF;      // T1 = T2 diag(gamma) (rows r, runs along s; sy = 1024)
+constexpr uint32_t P = T1 + 8192;     // two P tiles (same layout)
+constexpr uint32_t W = P + 16384;     // -W tile (rows k, runs along r; sy = 2048)
+constexpr uint32_t S = W + 16384;     // bf16 state (rows v, runs along k; sy = 2048)
+constexpr uint32_t DL = S + 32768;    // Delta^T bf16 (rows v, runs along s; sy = 2048)
+constexpr uint32_t OST = DL + 16384;  // output staging: 64 rows o[r][0..127] bf16
 constexpr uint32_t BAR = OST + 16384;
 constexpr uint32_t TOTAL = BAR + 256;
-// TMEM columns
-constexpr uint32_t TM_S = 0, TM_U = 128, TM_X1 = 256, TM_WT = 320, TM_O = 384;
-// mbarriers
+// TMEM columns: S, U^T (then Delta^T), X1, W^T, O1 (two buffers), O2
+constexpr uint32_t TM_S = 0, TM_U = 128, TM_X1 = 192, TM_WT = 256, TM_O1 = 320, TM_O2 = 448;
 enum {
-    FULL = 0,    // [2] loads of a buffer landed (loader arrive + TMA bytes)
-    EMPTY = 2,   // [2] all MMAs reading a buffer done
-    X1F = 4,     // X1 ready
-    WUF = 5,     // W^T, U^T ready
-    M3 = 6,      // Delta^T ready (state update's first MMA)
-    M4 = 7,      // [2] state update and output done
-    T1R = 9,     // T1 tile written (prep, 128)
-    QR = 10,     // P tile and diag(gamma) Q written (prep, 128)
-    WR = 11,     // -W tile and diag(e) K written (prep, 128)
-    DLR = 12,    // Delta^T tile written (state, 128)
-    SR = 13,     // S tile written, S scaled in TMEM (state, 128)
-    OF = 14,     // [2] O read out of TMEM (output, 128)
-    FIN = 16,    // every MMA of the CTA done (drained before TMEM is freed)
-    NBAR = 17
+    FULL = 0,   // [2] loads of a buffer landed (loader arrive + bytes)
+    EMPTY = 2,  // [2] a buffer is free again: MMA commit + output warps done reading its gamma
+    WUF = 4,    // W^T, U^T ready
+    X1F = 5,    // X1 ready
+    M3 = 6,     // Delta^T ready
+    M4S = 7,    // state update done
+    M4O = 8,    // O1 and O2 ready
+    T1R = 9,    // T1 tile written (prep, 256)
+    WR = 10,    // -W tile written (prep, 256)
+    PR = 11,    // P tile and diag(e) K written (prep, 256)
+    DLR = 12,   // Delta^T tile written (state, 256)
+    SR = 13,    // S tile written, S scaled in TMEM (state, 256)
+    OF = 14,    // O1, O2 read out of TMEM (output, 128)
+    FIN = 15,   // every MMA of the CTA done (drained before TMEM is freed)
+    NBAR = 16
 };
+__device__ __forceinline__ constexpr uint32_t bar_count(int i) {
+    return i == EMPTY || i == EMPTY + 1 ? 2u : (i >= T1R && i <= SR) ? 256u : i == OF ? 128u : 1u;
+}
 }  // namespace ob
 
 __global__ void __launch_bounds__(NT_WS, 1)
@@ -478,8 +489,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + BAR + 8 * NBAR);
     if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i)
-            tc::mbar_init(&bar[i], (i >= T1R && i < OF + 2) ? 128u : 1u);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -490,8 +500,10 @@ __global__ void __launch_bounds__(NT_WS, 1)
     const int nch = (sg.b - sg.a + C - 1) / C;
     const size_t sidx = ((size_t)sg.n * H + h) * D * D;
     const bool last_seg = sg.s == sg.ns - 1;
+    const int quarter_lane = (warp & 3) * 32 + lane;  // this thread's TMEM lane
     auto buf = [&](int c) { return sb + (uint32_t)(c & 1) * BUF; };
     auto vecp = [&](int c) { return reinterpret_cast<const float *>(smem + (c & 1) * BUF + B_VEC); };
+    auto full_par = [](int c) { return (uint32_t)((c >> 1) & 1); };
 
     if (warp == W_LOAD) {
         // ---------------------------------------------------------------- loader
@@ -499,7 +511,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             int issued = 0;
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1;
-                if (c >= 2 && !wait_bar(&bar[EMPTY + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err)) break;
+                if (c >= 2 && !wait_bar(&bar[EMPTY + b], full_par(c - 2), ctl, err)) break;
                 const uint32_t bb = buf(c);
                 const int cs = sg.a + c * C;
                 tc::mbar_arrive_expect_tx(&bar[FULL + b], 3u * 16384u + REC_BYTES);
@@ -513,7 +525,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                               &bar[FULL + b]);
                 issued = c + 1;
             }
-            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], (uint32_t)((c >> 1) & 1));
+            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], full_par(c));
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------------- MMA issuer
@@ -540,68 +552,64 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 for (int kk = 0; kk < C / 16; ++kk) {
                     tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024),
                                  tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
+                    tc::mma_bf16(tm + TM_U, tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
                                  tc::make_desc(bb + B_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
                 }
                 tc::mma_commit(&bar[WUF]);
             };
-            bool ok = wait_bar(&bar[FULL], 0, ctl, err);
-            if (ok) {
-                tc::fence_after_sync();
-                issue_x1(0);
-                ok = wait_bar(&bar[T1R], 0, ctl, err);
-            }
+            bool ok = wait_bar(&bar[FULL], 0, ctl, err) && wait_bar(&bar[T1R], 0, ctl, err);
             if (ok) {
                 tc::fence_after_sync();
                 issue_wu(0);
+                issue_x1(0);
             }
             for (int c = 0; ok && c < nch; ++c) {
                 const int b = c & 1;
                 const uint32_t par = (uint32_t)(c & 1), bb = buf(c);
-                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err) &&
-                           wait_bar(&bar[QR], par, ctl, err)))
-                    break;
-                if (c >= 2 && !(ok = wait_bar(&bar[OF + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err))) break;
+                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
-                // Delta^T = U^T + S (-W)^T, accumulated onto U^T
+                // Delta^T = U^T + S (-W)^T, accumulated onto U^T; then O1 = S Q^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                    tc::mma_bf16(tm + TM_U, tc::make_desc(sb + S + kk * 4096, 2048, 128),
                                  tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
                 tc::mma_commit(&bar[M3]);
-                // O = S (diag(gamma) Q)^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_O + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                    tc::mma_bf16(tm + TM_O1 + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
                                  tc::make_desc_sw128(bb + B_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk64,
                                  kk > 0);
-                // the next chunk's X1 and W^T, U^T
-                if (c + 1 < nch) {
-                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
-                    tc::fence_after_sync();
-                    issue_x1(c + 1);
-                    if (!(ok = wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err))) break;
-                    tc::fence_after_sync();
-                    issue_wu(c + 1);
-                }
-                if (!(ok = wait_bar(&bar[DLR], par, ctl, err))) break;
+                // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K)
+                if (!(ok = wait_bar(&bar[DLR], par, ctl, err) && wait_bar(&bar[PR], par, ctl, err))) break;
                 tc::fence_after_sync();
-                // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K), O += Delta^T P^T
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
                                  tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                tc::mma_commit(&bar[M4S]);
+                tc::mma_commit(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
+                // the next chunk's W^T, U^T and X1
+                if (c + 1 < nch) {
+                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], full_par(c + 1), ctl, err) &&
+                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
+                        break;
+                    tc::fence_after_sync();
+                    issue_wu(c + 1);
+                    issue_x1(c + 1);
+                }
+                // O2 = Delta^T P^T (after the output warps have read the previous O2)
+                if (c >= 1 && !(ok = wait_bar(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err))) break;
+                tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_O + 64 * b, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + P + b * 8192 + kk * 2048, 1024, 128), id_kk64, 1);
-                tc::mma_commit(&bar[M4 + b]);
-                tc::mma_commit(&bar[EMPTY + b]);
+                    tc::mma_bf16(tm + TM_O2, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + P + b * 8192 + kk * 2048, 1024, 128), id_kk64, kk > 0);
+                tc::mma_commit(&bar[M4O]);
             }
         }
-    } else if (warp < 4) {
-        // ---------------------------------------------------------------- state (thread = TMEM lane v)
-        const int v = tid;
+    } else if (warp < 8) {
+        // ---------------------------------------------------------------- state (row v, columns by half)
+        const int v = quarter_lane, half = warp >> 2;
         const uint32_t tl = lane_base(tm, warp);
         bool ok = true;
         float g0 = 1.f;
@@ -616,100 +624,103 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
             else if (S0)
                 src = S0 + sidx + (size_t)v * D;
-            state_init(sb + S, tl + TM_S, v, g0, src, lk, false);
-            if (nch == 0 && last_seg) state_epilogue(sb + S, tl + TM_S, v, 1.f, true, S_T + sidx + (size_t)v * D);
+            state_init64(sb + S, tl + TM_S, v, 64 * half, g0, src, lk, false);
+            if (nch == 0 && last_seg)
+                state_epilogue64(sb + S, tl + TM_S, v, 64 * half, 1.f, true, S_T + sidx + (size_t)v * D);
             handoff(&bar[SR]);
         }
         for (int c = 0; ok && c < nch; ++c) {
-            const int b = c & 1;
             if (!(ok = wait_bar(&bar[M3], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
-            tile64_epilogue(sb + DL, tl + TM_U + 64 * b, v);
+            tile32_epilogue(sb + DL, tl + TM_U + 32 * half, v, 32 * half, 1.f);
             handoff(&bar[DLR]);
-            if (!(ok = wait_bar(&bar[M4 + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            if (!(ok = wait_bar(&bar[M4S], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
             const bool last = c + 1 == nch;
             float g1 = 1.f;
             if (!last) {
-                if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
+                if (!(ok = wait_bar(&bar[FULL + ((c + 1) & 1)], full_par(c + 1), ctl, err))) break;
                 g1 = vecp(c + 1)[64 + C - 1];
             }
-            state_epilogue(sb + S, tl + TM_S, v, g1, last, last && last_seg ? S_T + sidx + (size_t)v * D : nullptr);
+            state_epilogue64(sb + S, tl + TM_S, v, 64 * half, g1, last,
+                             last && last_seg ? S_T + sidx + (size_t)v * D : nullptr);
             if (!last) handoff(&bar[SR]);
         }
-    } else if (warp < 8) {
-        // ---------------------------------------------------------------- prep (thread t128 = tid - 128)
-        const int t128 = tid - 128;
+    } else if (warp < 16) {
+        // ---------------------------------------------------------------- prep (TMEM lane k, columns by half)
+        const int t256 = tid - 256, k = quarter_lane, half = (warp >> 2) & 1;
         const uint32_t tl = lane_base(tm, warp);
         bool ok = true;
         for (int c = 0; ok && c < nch; ++c) {
             const int b = c & 1;
-            uint8_t *bp = smem + b * BUF;
-            const float *vec = vecp(c);
-            const float *Gl = vec, *gam = vec + 64, *dte = vec + 128;
-            // T1 = T2 diag(gamma) (WU of the previous chunk has finished reading T1: see WUF below)
-            if (!(ok = wait_bar(&bar[FULL + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
-            make_t1(smem + T1, bp + B_T2, gam, t128);
+            // T1 = T2 diag(gamma) (the previous chunk's W^T, U^T have read T1: WUF was waited below)
+            if (!(ok = wait_bar(&bar[FULL + b], full_par(c), ctl, err))) break;
+            make_t1(smem + T1, smem + b * BUF + B_T2, vecp(c) + 64, t256, 256);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
-            // P_rs = exp(G_r - G_s) X1_rs for s <= r (rows r = TMEM lanes 0..63: warps 4, 5)
-            if (!(ok = wait_bar(&bar[X1F], (uint32_t)(c & 1), ctl, err))) break;
-            tc::fence_after_sync();
-            if (warp < 6) {
-                const int r = t128;
-                const float Gr = Gl[r];
-                const uint32_t pt = sb + P + b * 8192;
-#pragma unroll
-                for (int s0 = 0; s0 < C; s0 += 32) {
-                    float x[32];
-                    tc::tmem_ld32(tl + TM_X1 + s0, x);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - Gl[s0 + i]) * x[i] : 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) st_run8(pt + tc::tile_off(r, s0 + i, 128, 1024), x + i);
-                }
-            }
-            tc::fence_before_sync();
-            scale_rows_sw128(bp + B_Q, gam, t128);  // X1 has read Q
-            handoff(&bar[QR]);
-            // -W from W^T (thread = TMEM lane k), then K <- diag(e) K (X1 and W^T, U^T have read K)
+            // -W from W^T (all earlier readers of the W tile are covered by WUF: W^T, U^T come after them)
             if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
-            neg_w_epilogue(sb + W, tl + TM_WT, t128);
-            scale_rows_sw128(bp + B_K, dte, t128);
+            tile32_epilogue(sb + W, tl + TM_WT + 32 * half, k, 32 * half, -1.f);
             handoff(&bar[WR]);
+            // P_rs = exp(G_r - G_s) X1_rs for s <= r (rows r = TMEM lanes 0..63), then K <- diag(e) K
+            if (!(ok = wait_bar(&bar[X1F], (uint32_t)(c & 1), ctl, err))) break;
+            tc::fence_after_sync();
+            const float *vec = vecp(c);
+            if ((warp & 3) < 2) {
+                const int r = k, s0 = 32 * half;
+                const float Gr = vec[r];
+                float x[32];
+                tc::tmem_ld32(tl + TM_X1 + s0, x);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - vec[s0 + i]) * x[i] : 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) st_run8(sb + P + b * 8192 + tc::tile_off(r, s0 + i, 128, 1024), x + i);
+            }
+            tc::fence_before_sync();
+            scale_rows_sw128(smem + b * BUF + B_K, vec + 128, t256, 256);  // X1 and W^T, U^T have read K
+            handoff(&bar[PR]);
         }
     } else {
-        // ---------------------------------------------------------------- output (thread = TMEM lane v)
-        const int v = tid - 256;
+        // ---------------------------------------------------------------- output (TMEM lane v)
+        const int v = quarter_lane;
         const uint32_t tl = lane_base(tm, warp);
         uint8_t *ost = smem + OST;
         bool ok = true;
         for (int c = 0; ok && c < nch; ++c) {
             const int b = c & 1;
             const int cs = sg.a + c * C, L = min(C, sg.b - cs);
-            if (!(ok = wait_bar(&bar[M4 + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
+            // gamma of this chunk into registers (lane l: gamma_l, gamma_{32+l}) so that the buffer
+            // can be refilled as soon as the MMAs are done with it
+            if (!(ok = wait_bar(&bar[FULL + b], full_par(c), ctl, err))) break;
+            const float g_lo = vecp(c)[64 + lane], g_hi = vecp(c)[96 + lane];
+            tc::named_sync(1, 128);
+            if (v == 0) tc::mbar_arrive(&bar[EMPTY + b]);
+            if (!(ok = wait_bar(&bar[M4O], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
             if (v == 0) tc::bulk_wait_read();  // the previous chunk's store has read the staging rows
             tc::named_sync(1, 128);
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < C; c0 += 32) {
-                float x[32];
-                tc::tmem_ld32(tl + TM_O + 64 * b + c0, x);
+                float x[32], y[32];
+                tc::tmem_ld32(tl + TM_O1 + 64 * b + c0, x);
+                tc::tmem_ld32(tl + TM_O2 + c0, y);
+                const float gsrc = c0 ? g_hi : g_lo;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) *reinterpret_cast<bf16 *>(ost + (c0 + i) * 256 + 2 * v) = __float2bfloat16_rn(x[i]);
+                for (int i = 0; i < 32; ++i)
+                    *reinterpret_cast<bf16 *>(ost + (c0 + i) * 256 + 2 * v) =
+                        __float2bfloat16_rn(fmaf(__shfl_sync(0xffffffffu, gsrc, i), x[i], y[i]));
             }
+            tc::fence_smem_to_async();
             tc::fence_before_sync();
-            tc::mbar_arrive(&bar[OF + b]);
+            tc::mbar_arrive(&bar[OF]);
+            tc::named_sync(1, 128);
             // A whole chunk, or a partial one that ends the tensor (TMA clips the rows past it), goes out
             // as one bulk tensor store; a partial chunk followed by another sequence's tokens is copied
             // row by row so that those tokens' outputs are not overwritten.
             if (L == C || cs + L >= T_tot) {
-                tc::fence_smem_to_async();
-                tc::named_sync(1, 128);
                 if (v == 0) tc::tma_store_3d(&tm_o, sb + OST, 0, h, cs);
             } else {
-                tc::named_sync(1, 128);
 #pragma unroll
                 for (int it = 0; it < 8; ++it) {
                     const int idx = it * 128 + v, r = idx >> 4, j = idx & 15;
@@ -732,34 +743,45 @@ __global__ void __launch_bounds__(NT_WS, 1)
 
 // ============================================================================ transition pass + link
 namespace tb {
-constexpr uint32_t B_K = 0, B_V = 16384, B_T2 = 32768, B_VEC = 40960;
-constexpr uint32_t BUF = 41984;
-constexpr uint32_t T1 = 2 * BUF;
-constexpr uint32_t W = T1 + 8192;
+// K ring (three slots: K tile and the chunk's vectors) and V ring (two slots: V tile and T2): K is
+// read until the chunk's last update, V and T2 only by W^T, U^T one chunk earlier, so each load
+// has about two chunks to arrive.
+constexpr uint32_t KS_K = 0, KS_VEC = 16384, KSLOT = 17408;
+constexpr uint32_t VS_V = 0, VS_T2 = 16384, VSLOT = 24576;
+constexpr uint32_t KRING = 0;
+constexpr uint32_t VRING = 3 * KSLOT;
+constexpr uint32_t T1 = VRING + 2 * VSLOT;  // T1 = T2 diag(gamma)
+constexpr uint32_t W = T1 + 8192;            // -W tile
 constexpr uint32_t S = W + 16384;
 constexpr uint32_t X = S + 32768;
 constexpr uint32_t DTS = X + 32768;
 constexpr uint32_t DTX = DTS + 16384;
 constexpr uint32_t BAR = DTX + 16384;
 constexpr uint32_t TOTAL = BAR + 256;
-// link phase (after the chunk loop, the buffers are free)
+// link phase (after the chunk loop, the rings and tiles below S's end are free)
 constexpr uint32_t PHI = 0;      // Phi hi | lo as B operands (rows k, runs along k'; sy = 2048)
 constexpr uint32_t SIN = 65536;  // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
-// TMEM columns
+// TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T
 constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
 enum {
-    FULL = 0, EMPTY = 2, WUF = 4, M3S = 5, M4S = 6, M3X = 7, M4X = 8,
-    T1R = 9,    // prep (128)
-    WR = 10,    // prep (128)
-    SR = 11,    // state S (128)
-    XR = 12,    // state X (128)
-    DSR = 13,   // state S (128)
-    DXR = 14,   // state X (128)
-    LNK = 15,   // S_in tiles landed
-    LMMA = 16,  // link MMAs done
-    FIN = 17,   // every MMA of the CTA done (drained before TMEM is freed)
-    NBAR = 18
+    FULLK = 0, EMPTYK = 3, FULLV = 6, EMPTYV = 8,
+    WUF = 10, M3S = 11, M4S = 12, M3X = 13, M4X = 14,
+    T1R = 15,   // T1 tile written (prep, 128)
+    WR = 16,    // -W tile written (prep, 128)
+    KR = 17,    // [2] diag(e) K written (prep, 128); two phases apart because the next chunk's
+                //     W^T, U^T (which let prep run ahead) are issued before this is waited for
+    SR = 19,    // S state (256)
+    XR = 20,    // X state (256)
+    DSR = 21,   // S state (256)
+    DXR = 22,   // X state (256)
+    LNK = 23,   // S_in tiles landed
+    LMMA = 24,  // link MMAs done
+    FIN = 25,   // every MMA of the CTA done (drained before TMEM is freed)
+    NBAR = 26
 };
+__device__ __forceinline__ constexpr uint32_t bar_count(int i) {
+    return (i >= T1R && i <= KR + 1) ? 128u : (i >= SR && i <= DXR) ? 256u : 1u;
+}
 }  // namespace tb
 
 __global__ void __launch_bounds__(NT_WS, 1)
@@ -789,7 +811,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + BAR + 8 * NBAR);
     if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i >= T1R && i <= DXR) ? 128u : 1u);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -800,55 +822,69 @@ __global__ void __launch_bounds__(NT_WS, 1)
     const int nch = (sg.b - sg.a + C - 1) / C;
     const bool has_x = sg.s > 0;  // the first segment starts from S0 and needs no Phi
     const size_t sidx = ((size_t)sg.n * H + h) * D * D;
-    auto buf = [&](int c) { return sb + (uint32_t)(c & 1) * BUF; };
-    auto vecp = [&](int c) { return reinterpret_cast<const float *>(smem + (c & 1) * BUF + B_VEC); };
+    const int quarter_lane = (warp & 3) * 32 + lane;
+    auto kslot = [&](int c) { return KRING + (uint32_t)(c % 3) * KSLOT; };
+    auto vslot = [&](int c) { return VRING + (uint32_t)(c & 1) * VSLOT; };
+    auto vecp = [&](int c) { return reinterpret_cast<const float *>(smem + kslot(c) + KS_VEC); };
+    auto kpar = [](int c) { return (uint32_t)((c / 3) & 1); };
+    auto vpar = [](int c) { return (uint32_t)((c >> 1) & 1); };
 
     if (warp == W_LOAD) {
         if (lane == 0) {
             int issued = 0;
             for (int c = 0; c < nch; ++c) {
-                const int b = c & 1;
-                if (c >= 2 && !wait_bar(&bar[EMPTY + b], (uint32_t)(((c - 2) >> 1) & 1), ctl, err)) break;
-                const uint32_t bb = buf(c);
                 const int cs = sg.a + c * C;
-                tc::mbar_arrive_expect_tx(&bar[FULL + b], 2u * 16384u + REC_BYTES);
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    tc::tma_load_3d(bb + B_K + hf * 8192, &tm_k, &bar[FULL + b], 64 * hf, h, cs);
-                    tc::tma_load_3d(bb + B_V + hf * 8192, &tm_v, &bar[FULL + b], 64 * hf, h, cs);
+                const uint8_t *rp = rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES;
+                if (c >= 3 && !wait_bar(&bar[EMPTYK + c % 3], kpar(c - 3), ctl, err)) break;
+                uint64_t *fk = &bar[FULLK + c % 3];
+                tc::mbar_arrive_expect_tx(fk, 16384u + 1024u);
+                tc::tma_load_3d(sb + kslot(c) + KS_K, &tm_k, fk, 0, h, cs);
+                tc::tma_load_3d(sb + kslot(c) + KS_K + 8192, &tm_k, fk, 64, h, cs);
+                tc::bulk_load(sb + kslot(c) + KS_VEC, rp + REC_VEC, 1024u, fk);
+                if (c >= 2 && !wait_bar(&bar[EMPTYV + (c & 1)], vpar(c - 2), ctl, err)) {
+                    drain_bar(fk, kpar(c));
+                    break;
                 }
-                tc::bulk_load(bb + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES, REC_BYTES,
-                              &bar[FULL + b]);
+                uint64_t *fv = &bar[FULLV + (c & 1)];
+                tc::mbar_arrive_expect_tx(fv, 16384u + 8192u);
+                tc::tma_load_3d(sb + vslot(c) + VS_V, &tm_v, fv, 0, h, cs);
+                tc::tma_load_3d(sb + vslot(c) + VS_V + 8192, &tm_v, fv, 64, h, cs);
+                tc::bulk_load(sb + vslot(c) + VS_T2, rp + REC_T2, 8192u, fv);
                 issued = c + 1;
             }
-            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], (uint32_t)((c >> 1) & 1));
+            for (int c = max(0, issued - 3); c < issued; ++c) drain_bar(&bar[FULLK + c % 3], kpar(c));
+            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULLV + (c & 1)], vpar(c));
         }
     } else if (warp == W_MMA) {
         if (lane == 0 && nch > 0) {
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            // W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views of the K and V tiles)
             auto issue_wu = [&](int c) {
-                const uint32_t bb = buf(c);
+                const uint32_t kt = sb + kslot(c) + KS_K, vs = sb + vslot(c);
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024),
+                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(kt + kk * 2048, 8192, 1024),
                                  tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
-                                 tc::make_desc(bb + B_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(vs + VS_V + kk * 2048, 8192, 1024),
+                                 tc::make_desc(vs + VS_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
                 }
                 tc::mma_commit(&bar[WUF]);
+                tc::mma_commit(&bar[EMPTYV + (c & 1)]);
             };
-            bool ok = wait_bar(&bar[FULL], 0, ctl, err) && wait_bar(&bar[T1R], 0, ctl, err);
+            bool ok = wait_bar(&bar[FULLK], 0, ctl, err) && wait_bar(&bar[FULLV], 0, ctl, err) &&
+                      wait_bar(&bar[T1R], 0, ctl, err);
             if (ok) {
                 tc::fence_after_sync();
                 issue_wu(0);
             }
             for (int c = 0; ok && c < nch; ++c) {
                 const int b = c & 1;
-                const uint32_t par = (uint32_t)(c & 1), bb = buf(c);
+                const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
                 if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
+                // Delta_S^T = U^T + S (-W)^T, accumulated onto U^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
@@ -863,19 +899,23 @@ __global__ void __launch_bounds__(NT_WS, 1)
                                      tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
                     tc::mma_commit(&bar[M3X]);
                 }
+                // the next chunk's W^T, U^T (the -W tile has been read by both products above)
                 if (c + 1 < nch) {
-                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err) &&
+                    if (!(ok = wait_bar(&bar[FULLK + (c + 1) % 3], kpar(c + 1), ctl, err) &&
+                               wait_bar(&bar[FULLV + ((c + 1) & 1)], vpar(c + 1), ctl, err) &&
                                wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
                         break;
                     tc::fence_after_sync();
                     issue_wu(c + 1);
                 }
-                if (!(ok = wait_bar(&bar[DSR], par, ctl, err))) break;
+                // S <- gamma_C S + Delta_S^T (diag(e) K), X <- gamma_C X + X (-W)^T diag(e) K
+                if (!(ok = wait_bar(&bar[DSR], par, ctl, err) && wait_bar(&bar[KR + b], (uint32_t)((c >> 1) & 1), ctl, err)))
+                    break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DTS + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
                 tc::mma_commit(&bar[M4S]);
                 if (has_x) {
                     if (!(ok = wait_bar(&bar[DXR], par, ctl, err))) break;
@@ -883,65 +923,68 @@ __global__ void __launch_bounds__(NT_WS, 1)
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
                         tc::mma_bf16(tm + TM_X, tc::make_desc(sb + DTX + kk * 4096, 2048, 128),
-                                     tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                                     tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
                     tc::mma_commit(&bar[M4X]);
                 }
-                tc::mma_commit(&bar[EMPTY + b]);
+                tc::mma_commit(&bar[EMPTYK + c % 3]);
             }
         }
-    } else if (warp < 8) {
-        // ---------------------------------------------------------------- S state (warps 0-3), X state (4-7)
-        const bool is_x = warp >= 4;
+    } else if (warp < 16) {
+        // ---------------------------------------------------------------- S state (warps 0-7), X state (8-15)
+        const bool is_x = warp >= 8;
         if (!is_x || has_x) {
-            const int v = tid & 127;
+            const int v = quarter_lane, half = (warp >> 2) & 1;
             const uint32_t tl = lane_base(tm, warp);
             const uint32_t s_tile = sb + (is_x ? X : S), dt_tile = sb + (is_x ? DTX : DTS);
             const uint32_t tm_state = is_x ? TM_X : TM_S;
             uint64_t *b_r = &bar[is_x ? XR : SR], *b_d = &bar[is_x ? DXR : DSR];
             uint64_t *b_m3 = &bar[is_x ? M3X : M3S], *b_m4 = &bar[is_x ? M4X : M4S];
-            bool ok = nch > 0 && wait_bar(&bar[FULL], 0, ctl, err);
+            bool ok = nch > 0 && wait_bar(&bar[FULLK], 0, ctl, err);
             if (ok) {
                 const float g0 = vecp(0)[64 + C - 1];
                 const float *src = (!is_x && sg.s == 0 && S0) ? S0 + sidx + (size_t)v * D : nullptr;
-                state_init(s_tile, tl + tm_state, v, g0, src, nullptr, is_x);
+                state_init64(s_tile, tl + tm_state, v, 64 * half, g0, src, nullptr, is_x);
                 handoff(b_r);
             }
             for (int c = 0; ok && c < nch; ++c) {
-                const int b = c & 1;
                 if (!(ok = wait_bar(b_m3, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
-                tile64_epilogue(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * b), v);
+                tile32_epilogue(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * (c & 1)) + 32 * half, v, 32 * half, 1.f);
                 handoff(b_d);
                 if (!(ok = wait_bar(b_m4, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
                 const bool last = c + 1 == nch;
                 float g1 = 1.f;
                 if (!last) {
-                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], (uint32_t)(((c + 1) >> 1) & 1), ctl, err))) break;
+                    if (!(ok = wait_bar(&bar[FULLK + (c + 1) % 3], kpar(c + 1), ctl, err))) break;
                     g1 = vecp(c + 1)[64 + C - 1];
                 }
-                state_epilogue(s_tile, tl + tm_state, v, g1, last, nullptr);
+                state_epilogue64(s_tile, tl + tm_state, v, 64 * half, g1, last, nullptr);
                 if (!last) handoff(b_r);
             }
         }
-    } else if (warp < 12) {
-        // ---------------------------------------------------------------- prep
-        const int t128 = tid - 256;
+    } else if (warp < 20) {
+        // ---------------------------------------------------------------- prep (TMEM lane k, all 64 columns)
+        const int t128 = tid - 512, k = quarter_lane;
         const uint32_t tl = lane_base(tm, warp);
         bool ok = true;
         for (int c = 0; ok && c < nch; ++c) {
-            const int b = c & 1;
-            uint8_t *bp = smem + b * BUF;
-            const float *vec = vecp(c);
-            if (!(ok = wait_bar(&bar[FULL + b], (uint32_t)((c >> 1) & 1), ctl, err))) break;
-            make_t1(smem + T1, bp + B_T2, vec + 64, t128);
+            // T1 = T2 diag(gamma) (the previous chunk's W^T, U^T have read T1: WUF was waited below)
+            if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
+                       wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err)))
+                break;
+            make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
+            // -W from W^T (the products that read the previous -W were issued before this W^T)
             if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
-            neg_w_epilogue(sb + W, tl + TM_WT, t128);
-            scale_rows_sw128(bp + B_K, vec + 128, t128);
+            tile32_epilogue(sb + W, tl + TM_WT, k, 0, -1.f);
+            tile32_epilogue(sb + W, tl + TM_WT + 32, k, 32, -1.f);
             handoff(&bar[WR]);
+            scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 128, t128, 128);  // W^T has read K
+            tc::fence_smem_to_async();
+            tc::mbar_arrive(&bar[KR + (c & 1)]);
         }
     }
     // ---------------------------------------------------------------- link (all threads)
@@ -951,23 +994,14 @@ __global__ void __launch_bounds__(NT_WS, 1)
     bool ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
     if (ok && has_x) {
         // Phi = X_end as bf16 hi / lo B-operand tiles (X warps), S_in from the previous segment (loader)
-        if (warp >= 4 && warp < 8) {
-            const int k = tid - 128;
+        if (warp >= 8 && warp < 16) {
+            const int k = quarter_lane, half = (warp >> 2) & 1;
             const uint32_t tl = lane_base(tm, warp);
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                float x[32], hi[32], lo[32];
+            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                float x[32];
                 tc::tmem_ld32(tl + TM_X + c0, x);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
-                    lo[i] = x[i] - hi[i];
-                }
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    st_run8(sb + PHI + tc::tile_off(k, c0 + i, 128, 2048), hi + i);
-                    st_run8(sb + PHI + 32768 + tc::tile_off(k, c0 + i, 128, 2048), lo + i);
-                }
+                st_split32(sb + PHI, k, c0, x);
             }
             tc::fence_smem_to_async();
         }
@@ -1009,17 +1043,17 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 tc::mma_commit(&bar[LMMA]);
             }
         }
-        if (ok && warp < 4) ok = wait_bar(&bar[LMMA], 0, ctl, err);
+        if (ok && warp < 8) ok = wait_bar(&bar[LMMA], 0, ctl, err);
         if (warp == W_LOAD && lane == 0 && ok) drain_bar(&bar[LNK], 0);
     }
     // publish S_end (S warps): bf16 hi / lo tiles in the link slot, then the flag
-    if (ok && warp < 4) {
+    if (ok && warp < 8) {
         tc::fence_after_sync();
-        const int v = tid;
+        const int v = quarter_lane, half = (warp >> 2) & 1;
         const uint32_t tl = lane_base(tm, warp);
         uint8_t *dst = link + ((size_t)gseg * H + h) * LINK_BYTES;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
             float x[32];
             tc::tmem_ld32(tl + TM_S + c0, x);
 #pragma unroll
