@@ -67,9 +67,10 @@ constexpr uint32_t REC_BYTES = 9216;
 constexpr uint32_t LINK_BYTES = 65536;
 constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 
-// Warp roles of the pipelined kernels (22 warps).
-constexpr int NT_WS = 704;
-constexpr int W_LOAD = 20, W_MMA = 21;
+// Warp roles of the pipelined kernels: 22 warps in the output pass, 23 in the
+// transition pass (a second MMA issuer for the X chain and the next chunk's W^T, U^T).
+constexpr int NT_WS = 704, NT_TRANS = 736;
+constexpr int W_LOAD = 20, W_MMA = 21, W_XMMA = 22;
 
 struct Ctl {
     uint32_t tmem;   // TMEM base written by tcgen05.alloc
@@ -763,28 +764,32 @@ constexpr uint32_t PHI = 0;      // Phi hi | lo as B operands (rows k, runs alon
 constexpr uint32_t SIN = 65536;  // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
 // TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T
 constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
+// Two MMA issuers: the S issuer (S chain) and the X issuer (X chain and the next chunk's W^T, U^T).
+// A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
+// kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
 enum {
-    FULLK = 0, EMPTYK = 3, FULLV = 6, EMPTYV = 8,
+    FULLK = 0, EMPTYK = 3,  // [3] K ring; EMPTYK takes one commit from each issuer
+    FULLV = 6, EMPTYV = 8,  // [2] V ring
     WUF = 10, M3S = 11, M4S = 12, M3X = 13, M4X = 14,
     T1R = 15,   // T1 tile written (prep, 128)
     WR = 16,    // -W tile written (prep, 128)
-    KR = 17,    // [2] diag(e) K written (prep, 128); two phases apart because the next chunk's
-                //     W^T, U^T (which let prep run ahead) are issued before this is waited for
-    SR = 19,    // S state (256)
-    XR = 20,    // X state (256)
-    DSR = 21,   // S state (256)
-    DXR = 22,   // X state (256)
-    LNK = 23,   // S_in tiles landed
-    LMMA = 24,  // link MMAs done
-    FIN = 25,   // every MMA of the CTA done (drained before TMEM is freed)
-    NBAR = 26
+    KR = 17,    // [4] diag(e) K written (prep, 128)
+    SR = 21,    // S state (256)
+    XR = 22,    // X state (256)
+    DSR = 23,   // [2] Delta_S^T tile written (S state, 256)
+    DXR = 25,   // X state (256)
+    LNK = 26,   // S_in tiles landed
+    LMMA = 27,  // link MMAs done
+    FIN = 28,   // every MMA of the S issuer done (drained before TMEM is freed)
+    FINX = 29,  // the same for the X issuer
+    NBAR = 30
 };
 __device__ __forceinline__ constexpr uint32_t bar_count(int i) {
-    return (i >= T1R && i <= KR + 1) ? 128u : (i >= SR && i <= DXR) ? 256u : 1u;
+    return (i >= EMPTYK && i < EMPTYK + 3) ? 2u : (i >= T1R && i < KR + 4) ? 128u : (i >= SR && i <= DXR) ? 256u : 1u;
 }
 }  // namespace tb
 
-__global__ void __launch_bounds__(NT_WS, 1)
+__global__ void __launch_bounds__(NT_TRANS, 1)
     k_ws_trans(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const float *S0,
                const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
                const int32_t *__restrict__ seg_off, const int32_t *__restrict__ chunk_off, int seg_chunks,
@@ -856,6 +861,37 @@ __global__ void __launch_bounds__(NT_WS, 1)
             for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULLV + (c & 1)], vpar(c));
         }
     } else if (warp == W_MMA) {
+        // ---------------------------------------------------------------- S issuer
+        if (lane == 0 && nch > 0) {
+            const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
+            const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            bool ok = true;
+            for (int c = 0; ok && c < nch; ++c) {
+                const int b = c & 1;
+                const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
+                // Delta_S^T = U^T + S (-W)^T, accumulated onto U^T (W^T, U^T are complete: prep saw WUF before WR)
+                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
+                tc::mma_commit(&bar[M3S]);
+                // S <- gamma_C S + Delta_S^T (diag(e) K)
+                if (!(ok = wait_bar(&bar[DSR + b], (uint32_t)((c >> 1) & 1), ctl, err) &&
+                           wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                    break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DTS + kk * 4096, 2048, 128),
+                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
+                tc::mma_commit(&bar[M4S]);
+                tc::mma_commit(&bar[EMPTYK + c % 3]);
+            }
+        }
+    } else if (warp == W_XMMA) {
+        // ---------------------------------------------------------------- X issuer (and W^T, U^T)
         if (lane == 0 && nch > 0) {
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
@@ -880,16 +916,9 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 issue_wu(0);
             }
             for (int c = 0; ok && c < nch; ++c) {
-                const int b = c & 1;
                 const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
-                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
-                tc::fence_after_sync();
-                // Delta_S^T = U^T + S (-W)^T, accumulated onto U^T
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
-                tc::mma_commit(&bar[M3S]);
+                // prep has read W^T(c) (WR); with the X chain, X (-W)^T
+                if (!(ok = wait_bar(&bar[WR], par, ctl, err))) break;
                 if (has_x) {
                     if (!(ok = wait_bar(&bar[XR], par, ctl, err))) break;
                     tc::fence_after_sync();
@@ -899,26 +928,21 @@ __global__ void __launch_bounds__(NT_WS, 1)
                                      tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
                     tc::mma_commit(&bar[M3X]);
                 }
-                // the next chunk's W^T, U^T (the -W tile has been read by both products above)
+                // the next chunk's W^T, U^T (into the U^T buffer whose Delta_S^T of chunk c - 1 has been read)
                 if (c + 1 < nch) {
                     if (!(ok = wait_bar(&bar[FULLK + (c + 1) % 3], kpar(c + 1), ctl, err) &&
                                wait_bar(&bar[FULLV + ((c + 1) & 1)], vpar(c + 1), ctl, err) &&
-                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
+                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err) &&
+                               (c == 0 || wait_bar(&bar[DSR + ((c - 1) & 1)], (uint32_t)(((c - 1) >> 1) & 1), ctl, err))))
                         break;
                     tc::fence_after_sync();
                     issue_wu(c + 1);
                 }
-                // S <- gamma_C S + Delta_S^T (diag(e) K), X <- gamma_C X + X (-W)^T diag(e) K
-                if (!(ok = wait_bar(&bar[DSR], par, ctl, err) && wait_bar(&bar[KR + b], (uint32_t)((c >> 1) & 1), ctl, err)))
-                    break;
-                tc::fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DTS + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
-                tc::mma_commit(&bar[M4S]);
+                // X <- gamma_C X + X (-W)^T diag(e) K
                 if (has_x) {
-                    if (!(ok = wait_bar(&bar[DXR], par, ctl, err))) break;
+                    if (!(ok = wait_bar(&bar[DXR], par, ctl, err) &&
+                               wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                        break;
                     tc::fence_after_sync();
 #pragma unroll
                     for (int kk = 0; kk < C / 16; ++kk)
@@ -937,7 +961,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const uint32_t tl = lane_base(tm, warp);
             const uint32_t s_tile = sb + (is_x ? X : S), dt_tile = sb + (is_x ? DTX : DTS);
             const uint32_t tm_state = is_x ? TM_X : TM_S;
-            uint64_t *b_r = &bar[is_x ? XR : SR], *b_d = &bar[is_x ? DXR : DSR];
+            uint64_t *b_r = &bar[is_x ? XR : SR];
             uint64_t *b_m3 = &bar[is_x ? M3X : M3S], *b_m4 = &bar[is_x ? M4X : M4S];
             bool ok = nch > 0 && wait_bar(&bar[FULLK], 0, ctl, err);
             if (ok) {
@@ -950,7 +974,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 if (!(ok = wait_bar(b_m3, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
                 tile32_epilogue(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * (c & 1)) + 32 * half, v, 32 * half, 1.f);
-                handoff(b_d);
+                handoff(&bar[is_x ? DXR : DSR + (c & 1)]);
                 if (!(ok = wait_bar(b_m4, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
                 const bool last = c + 1 == nch;
@@ -976,15 +1000,18 @@ __global__ void __launch_bounds__(NT_WS, 1)
             make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
-            // -W from W^T (the products that read the previous -W were issued before this W^T)
-            if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err))) break;
+            // -W from W^T: the X product that read the previous -W was issued before this W^T; the S
+            // product is waited for explicitly (it comes from the other issuer)
+            if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err) &&
+                       (c == 0 || wait_bar(&bar[M3S], (uint32_t)((c - 1) & 1), ctl, err))))
+                break;
             tc::fence_after_sync();
             tile32_epilogue(sb + W, tl + TM_WT, k, 0, -1.f);
             tile32_epilogue(sb + W, tl + TM_WT + 32, k, 32, -1.f);
             handoff(&bar[WR]);
             scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 128, t128, 128);  // W^T has read K
             tc::fence_smem_to_async();
-            tc::mbar_arrive(&bar[KR + (c & 1)]);
+            tc::mbar_arrive(&bar[KR + (c & 3)]);
         }
     }
     // ---------------------------------------------------------------- link (all threads)
@@ -1077,6 +1104,10 @@ __global__ void __launch_bounds__(NT_WS, 1)
         tc::mma_commit(&bar[FIN]);
         drain_bar(&bar[FIN], 0);
     }
+    if (warp == W_XMMA && lane == 0) {
+        tc::mma_commit(&bar[FINX]);
+        drain_bar(&bar[FINX], 0);
+    }
     tc::fence_before_sync();
     __syncthreads();
     if (tid == 0) {
@@ -1095,12 +1126,13 @@ __global__ void __launch_bounds__(256) k_ws_plan(const int32_t *__restrict__ cu,
                                                  uint32_t *__restrict__ err, int32_t *__restrict__ seg_off,
                                                  int32_t *__restrict__ chunk_off, uint32_t *__restrict__ flags,
                                                  int nflags) {
-    __shared__ int ps[256], pc[256];
+    __shared__ int wsum[2][8];
     __shared__ int bad;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) bad = 0;
     for (int i = tid; i < nflags; i += 256) flags[i] = 0u;
     __syncthreads();
+    // thread tid owns sequences [n0, n1)
     const int per = (N + 255) / 256;
     const int n0 = min(N, tid * per), n1 = min(N, n0 + per);
     auto nchunks = [&](int n) {
@@ -1118,29 +1150,42 @@ __global__ void __launch_bounds__(256) k_ws_plan(const int32_t *__restrict__ cu,
     }
     if (tid == 0 && cu) b |= (cu[0] != 0) || (cu[N] != T_tot);
     if (b) atomicOr(&bad, 1);
-    ps[tid] = ssum;
-    pc[tid] = csum;
-    __syncthreads();
-    if (tid == 0) {
-        int as = 0, ac = 0;
-        for (int i = 0; i < 256; ++i) {
-            const int xs = ps[i], xc = pc[i];
-            ps[i] = as;
-            pc[i] = ac;
-            as += xs;
-            ac += xc;
+    // exclusive block-wide prefix of (ssum, csum): warp shuffles, then the 8 warp totals
+    int si = ssum, ci = csum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int ys = __shfl_up_sync(0xffffffffu, si, off), yc = __shfl_up_sync(0xffffffffu, ci, off);
+        if (lane >= off) {
+            si += ys;
+            ci += yc;
         }
-        seg_off[N] = as;
-        chunk_off[N] = bad ? 0 : ac;
-        *err = bad ? ERRBIT_SEQLENS : 0u;
+    }
+    if (lane == 31) {
+        wsum[0][warp] = si;
+        wsum[1][warp] = ci;
     }
     __syncthreads();
-    int as = ps[tid], ac = pc[tid];
+    int ws_ = 0, wc_ = 0, ts = 0, tcn = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+        if (w < warp) {
+            ws_ += wsum[0][w];
+            wc_ += wsum[1][w];
+        }
+        ts += wsum[0][w];
+        tcn += wsum[1][w];
+    }
+    int as = ws_ + si - ssum, ac = wc_ + ci - csum;
     for (int n = n0; n < n1; ++n) {
         seg_off[n] = as;
         chunk_off[n] = ac;
         as += nseg(n);
         ac += nchunks(n);
+    }
+    if (tid == 0) {
+        seg_off[N] = ts;
+        chunk_off[N] = bad ? 0 : tcn;
+        *err = bad ? ERRBIT_SEQLENS : 0u;
     }
 }
 
@@ -1185,14 +1230,15 @@ WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
 // segments of a sequence run their chunks concurrently, at the cost of the
 // transition pass and one link per segment boundary on the critical path.
 // Time ~ n/s (t_trans + t_out) + (s - 1) t_link is smallest near s = sqrt(n)
-// (measured per chunk ~ t_link), capped so that all CTAs fit on the GPU at once.
+// (a link costs about as much as a chunk); a sweep on B200 put the best count
+// at about 1.2 sqrt(n), capped so that all CTAs fit on the GPU at once.
 int chunk_ws_seg_chunks(int N, int T_tot, int H) {
     const long pairs = (long)N * H;
     const long nc_avg = ((long)T_tot / N + C - 1) / C;
     const int sms = num_sms();
     if (pairs * 2 > sms || nc_avg < 8) return 0;
     long s = 1;
-    while ((s + 1) * (s + 1) <= nc_avg) ++s;  // floor(sqrt(nc_avg))
+    while (100 * s * s < 144 * nc_avg) ++s;  // ceil(1.2 sqrt(nc_avg))
     s = std::min(s, (long)sms / pairs);
     if (s < 2) return 0;
     return (int)((nc_avg + s - 1) / s);
@@ -1252,7 +1298,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         e = cudaFuncSetAttribute(k_ws_trans, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb::TOTAL);
         if (e != cudaSuccess) return e;
         pr = prof_start("ws_trans", st);
-        k_ws_trans<<<dim3(H, l.nslots), NT_WS, tb::TOTAL, st>>>(tm_k, tm_v, S0, cu, N, T_tot, H, err, seg_off,
+        k_ws_trans<<<dim3(H, l.nslots), NT_TRANS, tb::TOTAL, st>>>(tm_k, tm_v, S0, cu, N, T_tot, H, err, seg_off,
                                                                  chunk_off, seg_chunks, rec, link, flags);
         prof_stop(pr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

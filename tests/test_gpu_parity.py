@@ -156,6 +156,17 @@ def test_chunk_in_place_state():
     check(o, S, o_ref, S_ref, "bf16", "in place")
 
 
+def test_chunk_in_place_state_segmented():
+    """S0 may alias S_T also when the sequence is split into segments: the first segment reads
+    S0 while the last one writes S_T."""
+    w = make_prefill("prefill_2k", seqlens=[2000], H=2, s0=True, stress=True, seed=9)
+    dw = to_dev(w)
+    S = dw["S0"].clone()
+    o, S_T = gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], S, None, S_T=S, check=True)
+    o_ref, S_ref = run_oracle(w)
+    check(o, S, o_ref, S_ref, "bf16", "in place, segmented")
+
+
 def test_chunk_equals_decode_steps():
     """Prefill over T tokens equals T decode steps (one sequence)."""
     w = make_prefill("prefill_2k", seqlens=[70], H=2, s0=True, seed=8)
@@ -262,6 +273,18 @@ def test_segmented_slow_decay_stress():
     o, S_T = chunk(to_dev(w))
     o_ref, S_ref = run_oracle(w)
     check(o, S_T, o_ref, S_ref, "bf16", "segmented stress")
+
+
+def test_medium_workspace_falls_back_correctly():
+    """Workspaces between the error word and the preferred size select a plan that fits."""
+    w = make_prefill("prefill_2k", seqlens=[1500], H=2, s0=True, stress=True, seed=24)
+    dw = to_dev(w)
+    need = gdn.chunk_fwd_workspace_size(1, 1500, 2, 128, 128, torch.bfloat16)
+    o_ref, S_ref = run_oracle(w)
+    for frac in (0.8, 0.5, 0.25):
+        ws = torch.empty(int(need * frac) // 256 * 256, dtype=torch.uint8, device="cuda")
+        o, S_T = chunk(dw, workspace=ws)
+        check(o, S_T, o_ref, S_ref, "bf16", "workspace %.2f of preferred" % frac)
 
 
 def test_small_workspace_selects_coarser_plan():
