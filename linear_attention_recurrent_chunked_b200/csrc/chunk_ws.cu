@@ -67,10 +67,11 @@ constexpr uint32_t REC_BYTES = 9216;
 constexpr uint32_t LINK_BYTES = 65536;
 constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 
-// Warp roles of the pipelined kernels: 22 warps in the output pass, 23 in the
-// transition pass (a second MMA issuer for the X chain and the next chunk's W^T, U^T).
-constexpr int NT_WS = 704, NT_TRANS = 736;
-constexpr int W_LOAD = 20, W_MMA = 21, W_XMMA = 22;
+// Warp roles of the pipelined kernels: 22 warps in the output pass, 24 in the
+// transition pass (MMA issuers for the S chain, the X chain and the next chunk's W^T, U^T:
+// one tcgen05.mma costs its issuing thread ~50 cycles, so the chains get their own issuers).
+constexpr int NT_WS = 704, NT_TRANS = 768;
+constexpr int W_LOAD = 20, W_MMA = 21, W_XMMA = 22, W_WMMA = 23;
 
 struct Ctl {
     uint32_t tmem;   // TMEM base written by tcgen05.alloc
@@ -764,11 +765,11 @@ constexpr uint32_t PHI = 0;      // Phi hi | lo as B operands (rows k, runs alon
 constexpr uint32_t SIN = 65536;  // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
 // TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T
 constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
-// Two MMA issuers: the S issuer (S chain) and the X issuer (X chain and the next chunk's W^T, U^T).
+// Three MMA issuers: S chain, X chain, and the W issuer (the next chunk's W^T, U^T).
 // A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
 // kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
 enum {
-    FULLK = 0, EMPTYK = 3,  // [3] K ring; EMPTYK takes one commit from each issuer
+    FULLK = 0, EMPTYK = 3,  // [3] K ring
     FULLV = 6, EMPTYV = 8,  // [2] V ring
     WUF = 10, M3S = 11, M4S = 12, M3X = 13, M4X = 14,
     T1R = 15,   // T1 tile written (prep, 128)
@@ -782,10 +783,15 @@ enum {
     LMMA = 27,  // link MMAs done
     FIN = 28,   // every MMA of the S issuer done (drained before TMEM is freed)
     FINX = 29,  // the same for the X issuer
-    NBAR = 30
+    FINW = 30,  // the same for the W issuer
+    NBAR = 31
 };
-__device__ __forceinline__ constexpr uint32_t bar_count(int i) {
-    return (i >= EMPTYK && i < EMPTYK + 3) ? 2u : (i >= T1R && i < KR + 4) ? 128u : (i >= SR && i <= DXR) ? 256u : 1u;
+// (EMPTYK takes a commit from each issuer: count 2 with an X chain, 1 without.)
+__device__ __forceinline__ constexpr uint32_t bar_count(int i, bool has_x) {
+    return (i >= EMPTYK && i < EMPTYK + 3) ? (has_x ? 2u : 1u)
+           : (i >= T1R && i < KR + 4)     ? 128u
+           : (i >= SR && i <= DXR)        ? 256u
+                                          : 1u;
 }
 }  // namespace tb
 
@@ -814,9 +820,10 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     }
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + BAR);
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + BAR + 8 * NBAR);
+    const bool has_x = sg.s > 0;  // the first segment starts from S0 and needs no Phi
     if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
     if (tid == 0) {
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i, has_x));
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -825,7 +832,6 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     tc::fence_after_sync();
     const uint32_t tm = ctl->tmem;
     const int nch = (sg.b - sg.a + C - 1) / C;
-    const bool has_x = sg.s > 0;  // the first segment starts from S0 and needs no Phi
     const size_t sidx = ((size_t)sg.n * H + h) * D * D;
     const int quarter_lane = (warp & 3) * 32 + lane;
     auto kslot = [&](int c) { return KRING + (uint32_t)(c % 3) * KSLOT; };
@@ -860,6 +866,33 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             for (int c = max(0, issued - 3); c < issued; ++c) drain_bar(&bar[FULLK + c % 3], kpar(c));
             for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULLV + (c & 1)], vpar(c));
         }
+    } else if (warp == W_WMMA) {
+        // ---------------------------------------------------------------- W issuer: W^T = K^T T1^T, U^T = V^T T2^T
+        if (lane == 0 && nch > 0) {
+            const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+            bool ok = true;
+            for (int c = 0; ok && c < nch; ++c) {
+                // W^T(c - 1) read by prep (WR), the U^T buffer's Delta_S^T of chunk c - 2 read (DSR),
+                // this chunk's K, V, T2 and T1 in place
+                if (c >= 1 && !(ok = wait_bar(&bar[WR], (uint32_t)((c - 1) & 1), ctl, err))) break;
+                if (c >= 2 && !(ok = wait_bar(&bar[DSR + (c & 1)], (uint32_t)(((c - 2) >> 1) & 1), ctl, err))) break;
+                if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
+                           wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err) &&
+                           wait_bar(&bar[T1R], (uint32_t)(c & 1), ctl, err)))
+                    break;
+                tc::fence_after_sync();
+                const uint32_t kt = sb + kslot(c) + KS_K, vs = sb + vslot(c);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk) {
+                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(kt + kk * 2048, 8192, 1024),
+                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(vs + VS_V + kk * 2048, 8192, 1024),
+                                 tc::make_desc(vs + VS_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                }
+                tc::mma_commit(&bar[WUF]);
+                tc::mma_commit(&bar[EMPTYV + (c & 1)]);
+            }
+        }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------------- S issuer
         if (lane == 0 && nch > 0) {
@@ -891,65 +924,31 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             }
         }
     } else if (warp == W_XMMA) {
-        // ---------------------------------------------------------------- X issuer (and W^T, U^T)
-        if (lane == 0 && nch > 0) {
-            const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+        // ---------------------------------------------------------------- X issuer (segments with a Phi chain)
+        if (lane == 0 && nch > 0 && has_x) {
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
-            // W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views of the K and V tiles)
-            auto issue_wu = [&](int c) {
-                const uint32_t kt = sb + kslot(c) + KS_K, vs = sb + vslot(c);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(kt + kk * 2048, 8192, 1024),
-                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(vs + VS_V + kk * 2048, 8192, 1024),
-                                 tc::make_desc(vs + VS_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                }
-                tc::mma_commit(&bar[WUF]);
-                tc::mma_commit(&bar[EMPTYV + (c & 1)]);
-            };
-            bool ok = wait_bar(&bar[FULLK], 0, ctl, err) && wait_bar(&bar[FULLV], 0, ctl, err) &&
-                      wait_bar(&bar[T1R], 0, ctl, err);
-            if (ok) {
-                tc::fence_after_sync();
-                issue_wu(0);
-            }
+            bool ok = true;
             for (int c = 0; ok && c < nch; ++c) {
                 const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
-                // prep has read W^T(c) (WR); with the X chain, X (-W)^T
-                if (!(ok = wait_bar(&bar[WR], par, ctl, err))) break;
-                if (has_x) {
-                    if (!(ok = wait_bar(&bar[XR], par, ctl, err))) break;
-                    tc::fence_after_sync();
+                // X (-W)^T
+                if (!(ok = wait_bar(&bar[XR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                tc::fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        tc::mma_bf16(tm + TM_DX, tc::make_desc(sb + X + kk * 4096, 2048, 128),
-                                     tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
-                    tc::mma_commit(&bar[M3X]);
-                }
-                // the next chunk's W^T, U^T (into the U^T buffer whose Delta_S^T of chunk c - 1 has been read)
-                if (c + 1 < nch) {
-                    if (!(ok = wait_bar(&bar[FULLK + (c + 1) % 3], kpar(c + 1), ctl, err) &&
-                               wait_bar(&bar[FULLV + ((c + 1) & 1)], vpar(c + 1), ctl, err) &&
-                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err) &&
-                               (c == 0 || wait_bar(&bar[DSR + ((c - 1) & 1)], (uint32_t)(((c - 1) >> 1) & 1), ctl, err))))
-                        break;
-                    tc::fence_after_sync();
-                    issue_wu(c + 1);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    tc::mma_bf16(tm + TM_DX, tc::make_desc(sb + X + kk * 4096, 2048, 128),
+                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
+                tc::mma_commit(&bar[M3X]);
                 // X <- gamma_C X + X (-W)^T diag(e) K
-                if (has_x) {
-                    if (!(ok = wait_bar(&bar[DXR], par, ctl, err) &&
-                               wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
-                        break;
-                    tc::fence_after_sync();
+                if (!(ok = wait_bar(&bar[DXR], par, ctl, err) &&
+                           wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                    break;
+                tc::fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < C / 16; ++kk)
-                        tc::mma_bf16(tm + TM_X, tc::make_desc(sb + DTX + kk * 4096, 2048, 128),
-                                     tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
-                    tc::mma_commit(&bar[M4X]);
-                }
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16(tm + TM_X, tc::make_desc(sb + DTX + kk * 4096, 2048, 128),
+                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
+                tc::mma_commit(&bar[M4X]);
                 tc::mma_commit(&bar[EMPTYK + c % 3]);
             }
         }
@@ -1000,10 +999,10 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
-            // -W from W^T: the X product that read the previous -W was issued before this W^T; the S
-            // product is waited for explicitly (it comes from the other issuer)
+            // -W from W^T, once both chains' products have read the previous -W (other issuers)
             if (!(ok = wait_bar(&bar[WUF], (uint32_t)(c & 1), ctl, err) &&
-                       (c == 0 || wait_bar(&bar[M3S], (uint32_t)((c - 1) & 1), ctl, err))))
+                       (c == 0 || wait_bar(&bar[M3S], (uint32_t)((c - 1) & 1), ctl, err)) &&
+                       (c == 0 || !has_x || wait_bar(&bar[M3X], (uint32_t)((c - 1) & 1), ctl, err))))
                 break;
             tc::fence_after_sync();
             tile32_epilogue(sb + W, tl + TM_WT, k, 0, -1.f);
@@ -1107,6 +1106,10 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     if (warp == W_XMMA && lane == 0) {
         tc::mma_commit(&bar[FINX]);
         drain_bar(&bar[FINX], 0);
+    }
+    if (warp == W_WMMA && lane == 0) {
+        tc::mma_commit(&bar[FINW]);
+        drain_bar(&bar[FINW], 0);
     }
     tc::fence_before_sync();
     __syncthreads();
