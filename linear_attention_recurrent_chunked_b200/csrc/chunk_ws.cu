@@ -73,6 +73,13 @@ constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 constexpr int NT_WS = 704, NT_TRANS = 768;
 constexpr int W_LOAD = 20, W_MMA = 21, W_XMMA = 22, W_WMMA = 23;
 
+// Programmatic dependent launch: the kernels after the plan are launched early
+// (overlapping their predecessor's tail); each waits here for its predecessor
+// grid to complete before touching anything the predecessor writes, and lets
+// its own dependent launch as soon as all of its CTAs are running.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 struct Ctl {
     uint32_t tmem;   // TMEM base written by tcgen05.alloc
     uint32_t abort;  // set by the first role that gives up
@@ -274,6 +281,8 @@ __global__ void __launch_bounds__(256, 3)
               const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
               const int32_t *__restrict__ chunk_off, uint8_t *__restrict__ rec) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    griddep_wait();
+    griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     const int items = chunk_off[N] * H;
     if ((int)blockIdx.x >= items) return;
@@ -477,6 +486,8 @@ __global__ void __launch_bounds__(NT_WS, 1)
              const uint8_t *__restrict__ link) {
     using namespace ob;
     extern __shared__ __align__(1024) uint8_t smem[];
+    griddep_wait();
+    griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
     const int h = blockIdx.x;
@@ -802,6 +813,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags) {
     using namespace tb;
     extern __shared__ __align__(1024) uint8_t smem[];
+    griddep_wait();
+    griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
     const int h = blockIdx.x;
@@ -1132,6 +1145,7 @@ __global__ void __launch_bounds__(256) k_ws_plan(const int32_t *__restrict__ cu,
     __shared__ int wsum[2][8];
     __shared__ int bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_launch();  // the prep kernel may launch now; it waits for this grid to complete
     if (tid == 0) bad = 0;
     for (int i = tid; i < nflags; i += 256) flags[i] = 0u;
     __syncthreads();
@@ -1205,6 +1219,23 @@ int num_sms() {
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Launch with programmatic stream serialization (see griddep_wait).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Params>(args)...);
+}
 
 struct WsLayout {
     size_t seg_off, chunk_off, flags, s0copy, rec, link, total;
@@ -1292,28 +1323,31 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         const long items_bound = (long)l.nc_bound * H;
         const int grid = (int)std::max(1L, std::min(items_bound, 3L * num_sms()));
         pr = prof_start("ws_prep", st);
-        k_ws_prep<<<grid, 256, pp::TOTAL, st>>>(tm_k, g, beta, cu, N, T_tot, H, err, chunk_off, rec);
+        e = launch_pdl(k_ws_prep, dim3(grid), dim3(256), pp::TOTAL, st, tm_k, g, beta, cu, N, T_tot, H, err,
+                       (const int32_t *)chunk_off, rec);
         prof_stop(pr);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     if (seg_chunks > 0) {
         *stage = "ws_trans";
         e = cudaFuncSetAttribute(k_ws_trans, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tb::TOTAL);
         if (e != cudaSuccess) return e;
         pr = prof_start("ws_trans", st);
-        k_ws_trans<<<dim3(H, l.nslots), NT_TRANS, tb::TOTAL, st>>>(tm_k, tm_v, S0, cu, N, T_tot, H, err, seg_off,
-                                                                 chunk_off, seg_chunks, rec, link, flags);
+        e = launch_pdl(k_ws_trans, dim3(H, l.nslots), dim3(NT_TRANS), tb::TOTAL, st, tm_k, tm_v, S0, cu, N, T_tot, H,
+                       err, (const int32_t *)seg_off, (const int32_t *)chunk_off, seg_chunks, (const uint8_t *)rec, link,
+                       flags);
         prof_stop(pr);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
     }
     *stage = "ws_out";
     e = cudaFuncSetAttribute(k_ws_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ob::TOTAL);
     if (e != cudaSuccess) return e;
     pr = prof_start("ws_out", st);
-    k_ws_out<<<dim3(H, l.nslots), NT_WS, ob::TOTAL, st>>>(tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot, H, o, S_T, err,
-                                                          seg_chunks > 0 ? seg_off : nullptr, chunk_off,
-                                                          seg_chunks > 0 ? seg_chunks : 1, rec, link);
+    e = launch_pdl(k_ws_out, dim3(H, l.nslots), dim3(NT_WS), ob::TOTAL, st, tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot,
+                   H, o, S_T, err, seg_chunks > 0 ? (const int32_t *)seg_off : nullptr, (const int32_t *)chunk_off,
+                   seg_chunks > 0 ? seg_chunks : 1, (const uint8_t *)rec, (const uint8_t *)link);
     prof_stop(pr);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
