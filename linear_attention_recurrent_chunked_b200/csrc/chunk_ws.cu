@@ -23,10 +23,11 @@
 //     when a sequence is split into segments that run concurrently): runs the
 //     segment from S = 0 (S_loc) and, on a second state, from X = I with the
 //     V-term dropped (Phi = X_end), since over a segment the state map is
-//     affine, S_end = S_in Phi + S_loc. It then waits for the previous
-//     segment's published end state S_in, forms S_end on the tensor cores
-//     (bf16 hi/lo split operands, fp32 accumulation) and publishes it. The
-//     first segment starts from S0 and needs no Phi.
+//     affine, S_end = S_in Phi + S_loc. It publishes its part (Phi, S_loc),
+//     then folds the parts of the sequence's earlier segments onto the first
+//     segment's end state, S_end(j) = S_loc(j) + S_end(j - 1) Phi(j), on the
+//     tensor cores (bf16 hi/lo split operands, fp32 accumulation), and
+//     publishes its own S_end. The first segment starts from S0 and needs no Phi.
 //  3. k_ws_out, one CTA per segment: starts from S0 or the published end
 //     state of the previous segment and writes the outputs (and S_T).
 //
@@ -65,6 +66,11 @@ constexpr uint32_t REC_VEC = 8192;  // G (log2 units), gamma, e, beta: 4 x 64 fp
 constexpr uint32_t REC_BYTES = 9216;
 // ---- published segment end state: bf16 hi and lo tiles, rows v, runs along k (sx = 128, sy = 2048)
 constexpr uint32_t LINK_BYTES = 65536;
+// ---- published part of a segment after the first (S_end = S_in Phi + S_loc): Phi as bf16 hi and lo
+// tiles in the B-operand layout of the link step (rows k, runs along k'; sx = 128, sy = 2048), then
+// S_loc in fp32 as [k / 4][v][4] (one 16-byte group per TMEM lane and column quad, so that a warp's
+// 32 lanes touch 512 contiguous bytes)
+constexpr uint32_t PART_PHI = 0, PART_S = 65536, PART_BYTES = 131072;
 constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 
 // Warp roles of the pipelined kernels: 22 warps in the output pass, 24 in the
@@ -107,6 +113,24 @@ __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = tc::globaltimer();
     while (!tc::mbar_try_wait(bar, parity))
         if (tc::globaltimer() - t0 > kWaitNs) return;
+}
+
+// Bounded wait for a flag that another CTA publishes with a release store: true once it reads
+// FLAG_DONE. A failed flag, another role's abort or the time bound end it with false (and abort
+// this CTA; the time bound also records the timeout).
+__device__ __noinline__ bool wait_flag(const uint32_t *p, Ctl *ctl, uint32_t *err) {
+    const uint64_t t0 = tc::globaltimer();
+    uint32_t f;
+    while ((f = tc::ld_acquire_gpu(p)) == 0u) {
+        if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
+        if (tc::globaltimer() - t0 > kWaitNs) {
+            atomicOr(err, ERRBIT_TIMEOUT);
+            break;
+        }
+        __nanosleep(32);
+    }
+    if (f != FLAG_DONE) *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+    return f == FLAG_DONE;
 }
 
 __device__ __forceinline__ uint32_t lane_base(uint32_t tm, int warp) { return tm + ((uint32_t)((warp & 3) * 32) << 16); }
@@ -245,6 +269,25 @@ __device__ __forceinline__ void st_split32(uint32_t base, int row, int c0, const
         }
         st_run8(base + tc::tile_off(row, c0 + i, 128, 2048), hi);
         st_run8(base + 32768 + tc::tile_off(row, c0 + i, 128, 2048), lo);
+    }
+}
+
+// The same split into global memory (hi at base, lo at base + 32 KB; same byte layout, so that a
+// bulk copy reproduces the shared-memory tiles).
+__device__ __forceinline__ void st_split32_global(uint8_t *base, int row, int c0, const float *x) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float h0 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j]));
+            const float h1 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j + 1]));
+            hw[j] = tc::pack_bf16x2(h0, h1);
+            lw[j] = tc::pack_bf16x2(x[i + 2 * j] - h0, x[i + 2 * j + 1] - h1);
+        }
+        const uint32_t off = tc::tile_off(row, c0 + i, 128, 2048);
+        *reinterpret_cast<uint4 *>(base + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4 *>(base + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
 }
 
@@ -770,12 +813,13 @@ constexpr uint32_t X = S + 32768;
 constexpr uint32_t DTS = X + 32768;
 constexpr uint32_t DTX = DTS + 16384;
 constexpr uint32_t BAR = DTX + 16384;
-constexpr uint32_t TOTAL = BAR + 256;
-// link phase (after the chunk loop, the rings and tiles below S's end are free)
-constexpr uint32_t PHI = 0;      // Phi hi | lo as B operands (rows k, runs along k'; sy = 2048)
-constexpr uint32_t SIN = 65536;  // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
-// TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
+constexpr uint32_t TOTAL = BAR + 320;
+// link phase (after the chunk loop every tile is free)
+constexpr uint32_t SIN = 0;      // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
+constexpr uint32_t PHI = 65536;  // two buffers: Phi_j hi | lo as B operands (rows k, runs along k'; sy = 2048)
+// TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T;
+// in the link phase two fold accumulators take the columns from TM_F on
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_F = 256;
 // Three MMA issuers: S chain, X chain, and the W issuer (the next chunk's W^T, U^T).
 // A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
 // kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
@@ -790,27 +834,35 @@ enum {
     XR = 22,    // X state (256)
     DSR = 23,   // [2] Delta_S^T tile written (S state, 256)
     DXR = 25,   // X state (256)
-    LNK = 26,   // S_in tiles landed
-    LMMA = 27,  // link MMAs done
-    FIN = 28,   // every MMA of the S issuer done (drained before TMEM is freed)
-    FINX = 29,  // the same for the X issuer
-    FINW = 30,  // the same for the W issuer
-    NBAR = 31
+    FIN = 26,   // every MMA of the S issuer done (drained before TMEM is freed)
+    FINX = 27,  // the same for the X issuer
+    FINW = 28,  // the same for the W issuer
+    // link phase, fold step j (buffer j & 1 where there are two)
+    LNK = 29,     // the first segment's end state landed in SIN
+    AREADY = 30,  // [2] SIN holds split(S_end(j)) and fold accumulator j & 1 is read (S warps, 256)
+    PFULL = 32,   // [2] Phi_j landed
+    MDONE = 34,   // [2] the step's MMAs are done
+    DINIT = 36,   // [2] fold accumulator j & 1 holds S_loc(j) (X warps, 256)
+    NBAR = 38
 };
 // (EMPTYK takes a commit from each issuer: count 2 with an X chain, 1 without.)
 __device__ __forceinline__ constexpr uint32_t bar_count(int i, bool has_x) {
-    return (i >= EMPTYK && i < EMPTYK + 3) ? (has_x ? 2u : 1u)
-           : (i >= T1R && i < KR + 4)     ? 128u
-           : (i >= SR && i <= DXR)        ? 256u
-                                          : 1u;
+    return (i >= EMPTYK && i < EMPTYK + 3)                                  ? (has_x ? 2u : 1u)
+           : (i >= T1R && i < KR + 4)                                       ? 128u
+           : (i >= SR && i <= DXR)                                          ? 256u
+           : ((i >= AREADY && i < AREADY + 2) || (i >= DINIT && i < DINIT + 2)) ? 256u
+                                                                            : 1u;
 }
+static_assert(BAR + 8 * NBAR + 8 <= TOTAL, "barrier area");
+static_assert(PHI + 2 * 65536 <= BAR, "link-phase tiles");
 }  // namespace tb
 
 __global__ void __launch_bounds__(NT_TRANS, 1)
     k_ws_trans(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, const float *S0,
                const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
                const int32_t *__restrict__ seg_off, const int32_t *__restrict__ chunk_off, int seg_chunks,
-               const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags) {
+               const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags,
+               uint8_t *__restrict__ part, uint32_t *__restrict__ pflags) {
     using namespace tb;
     extern __shared__ __align__(1024) uint8_t smem[];
     griddep_wait();
@@ -827,6 +879,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     if (sb & 1023u) {
         if (tid == 0) {
             atomicOr(err, ERRBIT_INTERNAL);
+            tc::st_release_gpu(pflags + (size_t)gseg * H + h, FLAG_FAILED);
             tc::st_release_gpu(my_flag, FLAG_FAILED);
         }
         return;
@@ -1027,63 +1080,136 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         }
     }
     // ---------------------------------------------------------------- link (all threads)
+    // S_end(j) = S_loc(j) + S_end(j - 1) Phi(j) along the sequence's segments. Every segment after
+    // the first publishes its part (Phi, S_loc) as soon as its chunk loop ends; segment s then folds
+    // the parts of segments 1 .. s itself, starting from the first segment's published end state,
+    // instead of waiting for its predecessor's end state (a chain of s cross-CTA hand-offs). Each
+    // fold step is the arithmetic of the chained form: bf16 hi/lo split operands (hi hi + hi lo +
+    // lo hi) accumulated in fp32 onto S_loc(j), so both give the same bits.
+    //   X warps   publish the part, then load S_loc(j) into fold accumulator j & 1 (TMEM)
+    //   loader    the first segment's end state (SIN), Phi_j into buffer j & 1
+    //   S issuer  the step's 24 MMAs; the last step accumulates onto this segment's own S_loc
+    //   S warps   split the step's result into SIN for the next step; publish S_end(s)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     bool ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
-    if (ok && has_x) {
-        // Phi = X_end as bf16 hi / lo B-operand tiles (X warps), S_in from the previous segment (loader)
+    const int nfold = sg.s;                              // fold steps; the last is this segment's own
+    const size_t slot0 = (size_t)(gseg - sg.s) * H + h;  // the sequence's first segment
+    auto part_of = [&](int j) { return part + (slot0 + (size_t)j * H) * PART_BYTES; };
+    if (has_x) {
         if (warp >= 8 && warp < 16) {
-            const int k = quarter_lane, half = (warp >> 2) & 1;
+            const int r = quarter_lane, half = (warp >> 2) & 1;
             const uint32_t tl = lane_base(tm, warp);
+            if (ok) {
+                uint8_t *pt = part_of(nfold);
+                float4 *ps = reinterpret_cast<float4 *>(pt + PART_S);
 #pragma unroll 1
-            for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                float x[32];
-                tc::tmem_ld32(tl + TM_X + c0, x);
-                st_split32(sb + PHI, k, c0, x);
-            }
-            tc::fence_smem_to_async();
-        }
-        if (warp == W_LOAD && lane == 0) {
-            const uint32_t *prev = flags + (size_t)(gseg - 1) * H + h;
-            const uint64_t t0 = tc::globaltimer();
-            uint32_t f = 0;
-            while ((f = tc::ld_acquire_gpu(prev)) == 0) {
-                if (tc::globaltimer() - t0 > kWaitNs) break;
-                __nanosleep(64);
-            }
-            if (f == FLAG_DONE) {
-                tc::fence_proxy_async_global();
-                tc::mbar_arrive_expect_tx(&bar[LNK], LINK_BYTES);
-                tc::bulk_load(sb + SIN, link + ((size_t)(gseg - 1) * H + h) * LINK_BYTES, LINK_BYTES, &bar[LNK]);
-            } else {
-                if (f == 0) atomicOr(err, ERRBIT_TIMEOUT);
-                ctl->abort = 1;
-            }
-        }
-        tc::fence_before_sync();
-        __syncthreads();
-        tc::fence_after_sync();
-        ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort);
-        if (ok && warp == W_MMA && lane == 0) {
-            // S_end = S_loc + S_in Phi = S_loc + S_in_hi Phi_hi + S_in_hi Phi_lo + S_in_lo Phi_hi
-            if (wait_bar(&bar[LNK], 0, ctl, err)) {
-                const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                    float x[32];
+                    tc::tmem_ld32(tl + TM_X + c0, x);
+                    st_split32_global(pt + PART_PHI, r, c0, x);
+                    tc::tmem_ld32(tl + TM_S + c0, x);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
-                    const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
-                    const uint64_t bh = tc::make_desc(sb + PHI + kk * 256, 128, 2048);
-                    const uint64_t bl = tc::make_desc(sb + PHI + 32768 + kk * 256, 128, 2048);
-                    tc::mma_bf16(tm + TM_S, ah, bh, id_km128, 1);
-                    tc::mma_bf16(tm + TM_S, ah, bl, id_km128, 1);
-                    tc::mma_bf16(tm + TM_S, al, bh, id_km128, 1);
+                    for (int i = 0; i < 32; i += 4)
+                        ps[((c0 + i) >> 2) * D + r] = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                 }
-                tc::mma_commit(&bar[LMMA]);
+                __threadfence();
+            }
+            tc::fence_before_sync();  // the reads of S_loc precede the own fold step, which accumulates onto it
+            tc::named_sync(1, 256);
+            if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
+            for (int j = 1; ok && j < nfold; ++j) {
+                const int b = j & 1;
+                // accumulator b was last read by the split of step j - 2
+                if (j >= 3 && !(ok = wait_bar(&bar[AREADY + b], (uint32_t)(((j - 3) >> 1) & 1), ctl, err))) break;
+                if (!(ok = __all_sync(0xffffffffu, wait_flag(pflags + slot0 + (size_t)j * H, ctl, err)))) break;
+                tc::fence_after_sync();
+                const float4 *src = reinterpret_cast<const float4 *>(part_of(j) + PART_S);
+#pragma unroll 1
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                    float x[32];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 p4 = __ldcg(src + ((c0 + i) >> 2) * D + r);
+                        x[i] = p4.x;
+                        x[i + 1] = p4.y;
+                        x[i + 2] = p4.z;
+                        x[i + 3] = p4.w;
+                    }
+                    tc::tmem_st32(tl + TM_F + 128 * b + c0, *reinterpret_cast<uint32_t(*)[32]>(x));
+                }
+                tc::tmem_st_wait();
+                handoff(&bar[DINIT + b]);
+            }
+        } else if (warp == W_LOAD) {
+            if (lane == 0 && ok) {
+                int last[2] = {0, 0};
+                bool lnk = false, good = wait_flag(flags + slot0, ctl, err);
+                if (good) {
+                    tc::fence_proxy_async_global();
+                    tc::mbar_arrive_expect_tx(&bar[LNK], LINK_BYTES);
+                    tc::bulk_load(sb + SIN, link + slot0 * LINK_BYTES, LINK_BYTES, &bar[LNK]);
+                    lnk = true;
+                }
+                for (int j = 1; good && j <= nfold; ++j) {
+                    const int b = j & 1;
+                    // buffer b was last read by step j - 2
+                    if (j >= 3 && !(good = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 3) >> 1) & 1), ctl, err)))
+                        break;
+                    if (!(good = wait_flag(pflags + slot0 + (size_t)j * H, ctl, err))) break;
+                    tc::fence_proxy_async_global();
+                    tc::mbar_arrive_expect_tx(&bar[PFULL + b], 65536u);
+                    tc::bulk_load(sb + PHI + 65536u * b, part_of(j) + PART_PHI, 65536u, &bar[PFULL + b]);
+                    last[b] = j;
+                }
+                if (lnk) drain_bar(&bar[LNK], 0);
+                for (int b = 0; b < 2; ++b)
+                    if (last[b]) drain_bar(&bar[PFULL + b], (uint32_t)(((last[b] - 1) >> 1) & 1));
+            }
+        } else if (warp == W_MMA) {
+            if (lane == 0 && ok) {
+                const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+                for (int j = 1; j <= nfold; ++j) {
+                    const int b = j & 1;
+                    const bool own = j == nfold;
+                    if (!(j == 1 ? wait_bar(&bar[LNK], 0, ctl, err)
+                                 : wait_bar(&bar[AREADY + ((j - 1) & 1)], (uint32_t)(((j - 2) >> 1) & 1), ctl, err)))
+                        break;
+                    if (!wait_bar(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
+                    if (!own && !wait_bar(&bar[DINIT + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
+                    tc::fence_after_sync();
+                    const uint32_t d = tm + (own ? TM_S : TM_F + 128u * b), phi = sb + PHI + 65536u * b;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
+                        const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
+                        const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
+                        const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
+                        tc::mma_bf16(d, ah, bh, id_km128, 1);
+                        tc::mma_bf16(d, ah, bl, id_km128, 1);
+                        tc::mma_bf16(d, al, bh, id_km128, 1);
+                    }
+                    tc::mma_commit(&bar[MDONE + b]);
+                }
+            }
+        } else if (warp < 8 && ok) {
+            const int v = quarter_lane, half = (warp >> 2) & 1;
+            const uint32_t tl = lane_base(tm, warp);
+            for (int j = 1; j <= nfold; ++j) {
+                const int b = j & 1;
+                if (!(ok = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err))) break;
+                if (j == nfold) break;
+                tc::fence_after_sync();
+#pragma unroll 1
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                    float x[32];
+                    tc::tmem_ld32(tl + TM_F + 128 * b + c0, x);
+                    st_split32(sb + SIN, v, c0, x);
+                }
+                handoff(&bar[AREADY + b]);
             }
         }
-        if (ok && warp < 8) ok = wait_bar(&bar[LMMA], 0, ctl, err);
-        if (warp == W_LOAD && lane == 0 && ok) drain_bar(&bar[LNK], 0);
     }
     // publish S_end (S warps): bf16 hi / lo tiles in the link slot, then the flag
     if (ok && warp < 8) {
@@ -1095,20 +1221,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
             float x[32];
             tc::tmem_ld32(tl + TM_S + c0, x);
-#pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                uint32_t hw[4], lw[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float h0 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j]));
-                    const float h1 = __bfloat162float(__float2bfloat16_rn(x[i + 2 * j + 1]));
-                    hw[j] = tc::pack_bf16x2(h0, h1);
-                    lw[j] = tc::pack_bf16x2(x[i + 2 * j] - h0, x[i + 2 * j + 1] - h1);
-                }
-                const uint32_t off = tc::tile_off(v, c0 + i, 128, 2048);
-                *reinterpret_cast<uint4 *>(dst + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-                *reinterpret_cast<uint4 *>(dst + 32768 + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-            }
+            st_split32_global(dst, v, c0, x);
         }
         __threadfence();
     }
@@ -1238,7 +1351,7 @@ cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t 
 }
 
 struct WsLayout {
-    size_t seg_off, chunk_off, flags, s0copy, rec, link, total;
+    size_t seg_off, chunk_off, flags, s0copy, rec, link, part, total;
     int nslots, nc_bound;
 };
 
@@ -1250,10 +1363,11 @@ WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
     l.seg_off = 256;
     l.chunk_off = l.seg_off + align256((size_t)(N + 1) * 4);
     l.flags = l.chunk_off + align256((size_t)(N + 1) * 4);
-    l.s0copy = l.flags + align256((size_t)l.nslots * H * 4);
+    l.s0copy = l.flags + align256((size_t)2 * l.nslots * H * 4);  // end-state flags, then part flags
     l.rec = l.s0copy + (seg_chunks > 0 ? (size_t)N * H * D * D * sizeof(float) : 0);
     l.link = l.rec + align256((size_t)l.nc_bound * H * REC_BYTES);
-    l.total = l.link + (seg_chunks > 0 ? (size_t)l.nslots * H * LINK_BYTES : 0);
+    l.part = l.link + (seg_chunks > 0 ? (size_t)l.nslots * H * LINK_BYTES : 0);
+    l.total = l.part + (seg_chunks > 0 ? (size_t)l.nslots * H * PART_BYTES : 0);
     return l;
 }
 
@@ -1289,7 +1403,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     int32_t *seg_off = reinterpret_cast<int32_t *>(wsb + l.seg_off);
     int32_t *chunk_off = reinterpret_cast<int32_t *>(wsb + l.chunk_off);
     uint32_t *flags = reinterpret_cast<uint32_t *>(wsb + l.flags);
-    uint8_t *rec = wsb + l.rec, *link = wsb + l.link;
+    uint8_t *rec = wsb + l.rec, *link = wsb + l.link, *part = wsb + l.part;
     CUtensorMap tm_q, tm_k, tm_v, tm_o;
     cudaError_t e;
     *stage = "TMA descriptor encoding";
@@ -1310,7 +1424,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     }
     *stage = "plan";
     void *pr = prof_start("ws_plan", st);
-    const int nflags = seg_chunks > 0 ? l.nslots * H : 0;
+    const int nflags = seg_chunks > 0 ? 2 * l.nslots * H : 0;
     k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
     prof_stop(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1335,7 +1449,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         pr = prof_start("ws_trans", st);
         e = launch_pdl(k_ws_trans, dim3(H, l.nslots), dim3(NT_TRANS), tb::TOTAL, st, tm_k, tm_v, S0, cu, N, T_tot, H,
                        err, (const int32_t *)seg_off, (const int32_t *)chunk_off, seg_chunks, (const uint8_t *)rec, link,
-                       flags);
+                       flags, part, flags + (size_t)l.nslots * H);
         prof_stop(pr);
         if (e != cudaSuccess) return e;
     }
