@@ -818,8 +818,10 @@ constexpr uint32_t TOTAL = BAR + 320;
 constexpr uint32_t SIN = 0;      // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
 constexpr uint32_t PHI = 65536;  // two buffers: Phi_j hi | lo as B operands (rows k, runs along k'; sy = 2048)
 // TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T;
-// in the link phase two fold accumulators take the columns from TM_F on
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_F = 256;
+// in the link phase two fold accumulators take the columns from TM_F on, and once Phi has been
+// read out of X, the fold's A operand split(S_end(j)) takes X's columns: for K step kk (16 values
+// of k), 8 columns of bf16 pairs hi then 8 of lo, at TM_A + 16 kk
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_F = 256, TM_A = 128;
 // Three MMA issuers: S chain, X chain, and the W issuer (the next chunk's W^T, U^T).
 // A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
 // kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
@@ -839,7 +841,7 @@ enum {
     FINW = 28,  // the same for the W issuer
     // link phase, fold step j (buffer j & 1 where there are two)
     LNK = 29,     // the first segment's end state landed in SIN
-    AREADY = 30,  // [2] SIN holds split(S_end(j)) and fold accumulator j & 1 is read (S warps, 256)
+    AREADY = 30,  // [2] split(S_end(j)) is in TM_A and fold accumulator j & 1 is read (S warps, 256)
     PFULL = 32,   // [2] Phi_j landed
     MDONE = 34,   // [2] the step's MMAs are done
     DINIT = 36,   // [2] fold accumulator j & 1 holds S_loc(j) (X warps, 256)
@@ -1087,9 +1089,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     // fold step is the arithmetic of the chained form: bf16 hi/lo split operands (hi hi + hi lo +
     // lo hi) accumulated in fp32 onto S_loc(j), so both give the same bits.
     //   X warps   publish the part, then load S_loc(j) into fold accumulator j & 1 (TMEM)
-    //   loader    the first segment's end state (SIN), Phi_j into buffer j & 1
+    //   loader    the first segment's end state (SIN, the first step's A), Phi_j into buffer j & 1
     //   S issuer  the step's 24 MMAs; the last step accumulates onto this segment's own S_loc
-    //   S warps   split the step's result into SIN for the next step; publish S_end(s)
+    //   S warps   split the step's result into TM_A, the next step's A; publish S_end(s)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -1180,15 +1182,27 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                     if (!own && !wait_bar(&bar[DINIT + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
                     tc::fence_after_sync();
                     const uint32_t d = tm + (own ? TM_S : TM_F + 128u * b), phi = sb + PHI + 65536u * b;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
-                        const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
-                        const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
-                        const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
-                        tc::mma_bf16(d, ah, bh, id_km128, 1);
-                        tc::mma_bf16(d, ah, bl, id_km128, 1);
-                        tc::mma_bf16(d, al, bh, id_km128, 1);
+                    if (j == 1) {
+#pragma unroll 1
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
+                            const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
+                            const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
+                            const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
+                            tc::mma_bf16(d, ah, bh, id_km128, 1);
+                            tc::mma_bf16(d, ah, bl, id_km128, 1);
+                            tc::mma_bf16(d, al, bh, id_km128, 1);
+                        }
+                    } else {
+#pragma unroll 1
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ah = tm + TM_A + 16 * kk, al = ah + 8;
+                            const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
+                            const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
+                            tc::mma_bf16_ts(d, ah, bh, id_km128, 1);
+                            tc::mma_bf16_ts(d, ah, bl, id_km128, 1);
+                            tc::mma_bf16_ts(d, al, bh, id_km128, 1);
+                        }
                     }
                     tc::mma_commit(&bar[MDONE + b]);
                 }
@@ -1202,12 +1216,23 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 if (j == nfold) break;
                 tc::fence_after_sync();
 #pragma unroll 1
-                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                    float x[32];
-                    tc::tmem_ld32(tl + TM_F + 128 * b + c0, x);
-                    st_split32(sb + SIN, v, c0, x);
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+                    // columns c0 .. c0 + 15 are K step c0 / 16: 8 columns of hi pairs, then 8 of lo
+                    float x[16];
+                    tc::tmem_ld16(tl + TM_F + 128 * b + c0, x);
+                    float u[16];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * i]));
+                        const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * i + 1]));
+                        u[i] = __uint_as_float(tc::pack_bf16x2(h0, h1));
+                        u[8 + i] = __uint_as_float(tc::pack_bf16x2(x[2 * i] - h0, x[2 * i + 1] - h1));
+                    }
+                    tc::tmem_st16(tl + TM_A + c0, u);
                 }
-                handoff(&bar[AREADY + b]);
+                tc::tmem_st_wait();
+                tc::fence_before_sync();
+                tc::mbar_arrive(&bar[AREADY + b]);
             }
         }
     }
