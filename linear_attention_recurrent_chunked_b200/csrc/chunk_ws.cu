@@ -307,19 +307,23 @@ __device__ __forceinline__ size_t rec_index(const int32_t *chunk_off, const Segm
 
 // ============================================================================ prep
 namespace pp {
-constexpr uint32_t K0 = 0;                          // two K tiles (128-byte swizzle), 16 KB each
-constexpr uint32_t AT = 32768;                      // A, then T in place: fp32 [64][AP]
+constexpr uint32_t K0 = 0;                          // K tile (128-byte swizzle), 16 KB
+constexpr uint32_t AT = 16384;                      // A, then T in place: fp32 [64][AP]
 constexpr uint32_t XS = AT + 64 * AP * 4;           // solve scratch, 32 x XP fp32
 constexpr uint32_t REC = XS + 32 * ut::XP * 4;      // record staging (bulk-stored)
 constexpr uint32_t RAW = REC + REC_BYTES;           // raw g, beta of two items: 2 x 512 B
-constexpr uint32_t BAR = RAW + 1024;                // full[2], mma, TMEM slot
+constexpr uint32_t VS = RAW + 1024;                 // G, gamma, e, beta of the current item (4 x 64 fp32)
+constexpr uint32_t BAR = VS + 1024;                 // K full, mma, TMEM slot
 constexpr uint32_t TOTAL = BAR + 64;
+constexpr int CTAS_PER_SM = 4;
 }  // namespace pp
 
 // Persistent: CTA b handles items b, b + gridDim.x, ... where item = gc * H + h
 // (gc = global chunk index, prefix chunk_off over sequences). The next item's
-// K tile (TMA) and g, beta (cp.async) are fetched while the current one runs.
-__global__ void __launch_bounds__(256, 3)
+// g, beta (cp.async) are fetched while the current one runs, and its K tile
+// (TMA) as soon as the current K K^T product has read the single K buffer.
+// Four CTAs share an SM, so that one's solve overlaps another's loads.
+__global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
     k_ws_prep(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ g, const float *__restrict__ beta,
               const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
               const int32_t *__restrict__ chunk_off, uint8_t *__restrict__ rec) {
@@ -335,7 +339,7 @@ __global__ void __launch_bounds__(256, 3)
         if (tid == 0) atomicOr(err, ERRBIT_INTERNAL);
         return;
     }
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + pp::BAR);  // [0,1] full, [2] mma
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + pp::BAR);  // [0] K full, [2] mma
     uint32_t *tslot = reinterpret_cast<uint32_t *>(smem + pp::BAR + 32);
     if (warp == 0) tc::tmem_alloc(tslot, 64);
     if (tid == 0) {
@@ -347,7 +351,7 @@ __global__ void __launch_bounds__(256, 3)
     tc::fence_after_sync();
     const uint32_t tm = *tslot;
     float *AT = reinterpret_cast<float *>(smem + pp::AT);
-    float *vec = reinterpret_cast<float *>(smem + pp::REC + REC_VEC);
+    float *vec = reinterpret_cast<float *>(smem + pp::VS);
     float *Gl = vec, *gam = vec + 64, *dte = vec + 128, *bet = vec + 192;
 
     // where item w lives: head h, chunk start cs, valid length L, global chunk gc
@@ -364,14 +368,16 @@ __global__ void __launch_bounds__(256, 3)
         cs = t0 + (gc - chunk_off[lo]) * C;
         L = min(C, t1 - cs);
     };
-    auto issue = [&](int w, int b) {
+    auto issue_k = [&](int w) {  // one thread
         int h, cs, L, gc;
         locate(w, h, cs, L, gc);
-        if (tid == 32) {
-            tc::mbar_arrive_expect_tx(&bars[b], 16384u);
-            tc::tma_load_3d(sb + pp::K0 + b * 16384u, &tm_k, &bars[b], 0, h, cs);
-            tc::tma_load_3d(sb + pp::K0 + b * 16384u + 8192u, &tm_k, &bars[b], 64, h, cs);
-        }
+        tc::mbar_arrive_expect_tx(&bars[0], 16384u);
+        tc::tma_load_3d(sb + pp::K0, &tm_k, &bars[0], 0, h, cs);
+        tc::tma_load_3d(sb + pp::K0 + 8192u, &tm_k, &bars[0], 64, h, cs);
+    };
+    auto issue = [&](int w, int b) {  // g, beta
+        int h, cs, L, gc;
+        locate(w, h, cs, L, gc);
         if (tid < 2 * C) {
             const int r = tid & 63;
             const bool ok = r < L;
@@ -385,18 +391,32 @@ __global__ void __launch_bounds__(256, 3)
     const uint32_t id_m64 = tc::make_idesc_bf16(64, 64, 0, 0);
     const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
     bool ok = true;
+    if (tid == 32) issue_k(blockIdx.x);
     issue(blockIdx.x, 0);
     int it = 0;
     for (int w = blockIdx.x; w < items; w += gridDim.x, ++it) {
         const int b = it & 1;
         const int wn = w + gridDim.x;
+        // ---- X1 = K K^T (M = 64: accumulator row i in TMEM lane (i % 16) + 32 (i / 16)), issued first so that it
+        // runs during the scalars (the previous item's reads of X1 are behind the last __syncthreads)
+        if (tid == 64) {
+            tc::fence_after_sync();
+            if (!tc::mbar_wait(&bars[0], (uint32_t)(it & 1))) atomicOr(err, ERRBIT_TIMEOUT);
+            tc::fence_after_sync();
+            const uint32_t kt = sb + pp::K0;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint64_t a = tc::make_desc_sw128(kt + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
+                tc::mma_bf16(tm, a, a, id_m64, kk > 0);
+            }
+            tc::mma_commit(&bars[2]);
+        }
         if (wn < items) {
             issue(wn, b ^ 1);
             cp_async_wait_1();
         } else {
             cp_async_wait_all();
         }
-        if (tid == 0) tc::bulk_wait_read();  // the previous record has left the staging area
         __syncthreads();
         // ---- scalars: G = cumsum(g) (log2 units), gamma, e, beta
         const float *graw = reinterpret_cast<const float *>(smem + pp::RAW + b * 512u);
@@ -417,24 +437,13 @@ __global__ void __launch_bounds__(256, 3)
             dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
             bet[tid] = graw[64 + tid];
         }
-        // ---- X1 = K K^T (M = 64: accumulator row i in TMEM lane (i % 16) + 32 (i / 16))
-        if (tid == 0) {
-            if (!tc::mbar_wait(&bars[b], (uint32_t)((it >> 1) & 1))) atomicOr(err, ERRBIT_TIMEOUT);
-            tc::fence_after_sync();
-            const uint32_t kt = sb + pp::K0 + b * 16384u;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint64_t a = tc::make_desc_sw128(kt + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024);
-                tc::mma_bf16(tm, a, a, id_m64, kk > 0);
-            }
-            tc::mma_commit(&bars[2]);
-        }
         ok = tc::mbar_wait(&bars[2], (uint32_t)(it & 1));
         tc::fence_after_sync();
         if (!__syncthreads_and(ok)) {
             if (tid == 0) atomicOr(err, ERRBIT_TIMEOUT);
             break;
         }
+        if (tid == 32 && wn < items) issue_k(wn);  // the product has read the K buffer
         // ---- A_rs = beta_r exp(G_r - G_s) X1_rs for s < r (warp w: rows 16 (w%4) + lane, columns 32 (w/4) ..)
         {
             const int lane = tid & 31, r = 16 * (warp & 3) + (lane & 15), s0 = 32 * (warp >> 2);
@@ -453,6 +462,7 @@ __global__ void __launch_bounds__(256, 3)
                 }
             }
         }
+        if (tid == 0) tc::bulk_wait_read();  // the previous record has left the staging area (written after the solve)
         tc::fence_before_sync();
         __syncthreads();
         ut::solve64(AT, AT, reinterpret_cast<float *>(smem + pp::XS));
@@ -464,6 +474,7 @@ __global__ void __launch_bounds__(256, 3)
             for (int i = 0; i < 16; ++i) x[i] = AT[r * AP + s0 + i] * bet[s0 + i];
             st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0, 128, 1024), x);
             st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0 + 8, 128, 1024), x + 8);
+            reinterpret_cast<float *>(smem + pp::REC + REC_VEC)[tid] = vec[tid];
         }
         tc::fence_smem_to_async();
         __syncthreads();
@@ -474,10 +485,7 @@ __global__ void __launch_bounds__(256, 3)
         }
     }
     cp_async_wait_all();
-    if (tid == 32 && !ok) {  // a K tile may still be in flight after a timeout
-        drain_bar(&bars[0], 0);
-        drain_bar(&bars[1], 0);
-    }
+    if (tid == 32 && !ok) drain_bar(&bars[0], (uint32_t)(it & 1));  // this item's K tile may still be in flight
     if (tid == 0) tc::bulk_wait_all();
     tc::fence_before_sync();
     __syncthreads();
@@ -1460,7 +1468,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         e = cudaFuncSetAttribute(k_ws_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pp::TOTAL);
         if (e != cudaSuccess) return e;
         const long items_bound = (long)l.nc_bound * H;
-        const int grid = (int)std::max(1L, std::min(items_bound, 3L * num_sms()));
+        const int grid = (int)std::max(1L, std::min(items_bound, (long)pp::CTAS_PER_SM * num_sms()));
         pr = prof_start("ws_prep", st);
         e = launch_pdl(k_ws_prep, dim3(grid), dim3(256), pp::TOTAL, st, tm_k, g, beta, cu, N, T_tot, H, err,
                        (const int32_t *)chunk_off, rec);
