@@ -537,7 +537,10 @@ __global__ void __launch_bounds__(NT_WS, 1)
              const uint8_t *__restrict__ link) {
     using namespace ob;
     extern __shared__ __align__(1024) uint8_t smem[];
-    griddep_wait();
+    // The loader waits for the predecessor grid only after it has started the first chunks' Q, K, V
+    // loads (inputs, which no kernel of the call writes); the plan (error word, offsets) is complete
+    // before the predecessor can launch this grid.
+    if ((threadIdx.x >> 5) != W_LOAD) griddep_wait();
     griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
@@ -572,21 +575,30 @@ __global__ void __launch_bounds__(NT_WS, 1)
     if (warp == W_LOAD) {
         // ---------------------------------------------------------------- loader
         if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nch; ++c) {
-                const int b = c & 1;
-                if (c >= 2 && !wait_bar(&bar[EMPTY + b], full_par(c - 2), ctl, err)) break;
+            auto load_inputs = [&](int c) {
                 const uint32_t bb = buf(c);
                 const int cs = sg.a + c * C;
-                tc::mbar_arrive_expect_tx(&bar[FULL + b], 3u * 16384u + REC_BYTES);
+                tc::mbar_arrive_expect_tx(&bar[FULL + (c & 1)], 3u * 16384u + REC_BYTES);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    tc::tma_load_3d(bb + B_K + hf * 8192, &tm_k, &bar[FULL + b], 64 * hf, h, cs);
-                    tc::tma_load_3d(bb + B_Q + hf * 8192, &tm_q, &bar[FULL + b], 64 * hf, h, cs);
-                    tc::tma_load_3d(bb + B_V + hf * 8192, &tm_v, &bar[FULL + b], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_K + hf * 8192, &tm_k, &bar[FULL + (c & 1)], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_Q + hf * 8192, &tm_q, &bar[FULL + (c & 1)], 64 * hf, h, cs);
+                    tc::tma_load_3d(bb + B_V + hf * 8192, &tm_v, &bar[FULL + (c & 1)], 64 * hf, h, cs);
                 }
-                tc::bulk_load(bb + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES, REC_BYTES,
-                              &bar[FULL + b]);
+            };
+            auto load_record = [&](int c) {
+                tc::bulk_load(buf(c) + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES,
+                              REC_BYTES, &bar[FULL + (c & 1)]);
+            };
+            const int pre = min(nch, 2);
+            for (int c = 0; c < pre; ++c) load_inputs(c);
+            griddep_wait();
+            for (int c = 0; c < pre; ++c) load_record(c);
+            int issued = pre;
+            for (int c = pre; c < nch; ++c) {
+                if (!wait_bar(&bar[EMPTY + (c & 1)], full_par(c - 2), ctl, err)) break;
+                load_inputs(c);
+                load_record(c);
                 issued = c + 1;
             }
             for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], full_par(c));
@@ -875,7 +887,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                uint8_t *__restrict__ part, uint32_t *__restrict__ pflags) {
     using namespace tb;
     extern __shared__ __align__(1024) uint8_t smem[];
-    griddep_wait();
+    // Only the loader reads what the prep pass writes (the records); it waits for that grid after
+    // starting the first chunks' K, V loads, and the other roles start at once (S0, the identity).
+    // The plan (error word, offsets, cleared flags) is complete before prep can launch this grid.
     griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
@@ -918,29 +932,46 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
 
     if (warp == W_LOAD) {
         if (lane == 0) {
-            int issued = 0;
-            for (int c = 0; c < nch; ++c) {
-                const int cs = sg.a + c * C;
-                const uint8_t *rp = rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES;
-                if (c >= 3 && !wait_bar(&bar[EMPTYK + c % 3], kpar(c - 3), ctl, err)) break;
+            auto rp = [&](int c) { return rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES; };
+            auto load_k = [&](int c) {
                 uint64_t *fk = &bar[FULLK + c % 3];
                 tc::mbar_arrive_expect_tx(fk, 16384u + 1024u);
-                tc::tma_load_3d(sb + kslot(c) + KS_K, &tm_k, fk, 0, h, cs);
-                tc::tma_load_3d(sb + kslot(c) + KS_K + 8192, &tm_k, fk, 64, h, cs);
-                tc::bulk_load(sb + kslot(c) + KS_VEC, rp + REC_VEC, 1024u, fk);
-                if (c >= 2 && !wait_bar(&bar[EMPTYV + (c & 1)], vpar(c - 2), ctl, err)) {
-                    drain_bar(fk, kpar(c));
-                    break;
-                }
+                tc::tma_load_3d(sb + kslot(c) + KS_K, &tm_k, fk, 0, h, sg.a + c * C);
+                tc::tma_load_3d(sb + kslot(c) + KS_K + 8192, &tm_k, fk, 64, h, sg.a + c * C);
+            };
+            auto load_v = [&](int c) {
                 uint64_t *fv = &bar[FULLV + (c & 1)];
                 tc::mbar_arrive_expect_tx(fv, 16384u + 8192u);
-                tc::tma_load_3d(sb + vslot(c) + VS_V, &tm_v, fv, 0, h, cs);
-                tc::tma_load_3d(sb + vslot(c) + VS_V + 8192, &tm_v, fv, 64, h, cs);
-                tc::bulk_load(sb + vslot(c) + VS_T2, rp + REC_T2, 8192u, fv);
-                issued = c + 1;
+                tc::tma_load_3d(sb + vslot(c) + VS_V, &tm_v, fv, 0, h, sg.a + c * C);
+                tc::tma_load_3d(sb + vslot(c) + VS_V + 8192, &tm_v, fv, 64, h, sg.a + c * C);
+            };
+            auto load_kvec = [&](int c) { tc::bulk_load(sb + kslot(c) + KS_VEC, rp(c) + REC_VEC, 1024u, &bar[FULLK + c % 3]); };
+            auto load_t2 = [&](int c) { tc::bulk_load(sb + vslot(c) + VS_T2, rp(c) + REC_T2, 8192u, &bar[FULLV + (c & 1)]); };
+            // the first chunks' K (three slots) and V (two) before the records exist
+            const int pk = min(nch, 3), pv = min(nch, 2);
+            for (int c = 0; c < pk; ++c) load_k(c);
+            for (int c = 0; c < pv; ++c) load_v(c);
+            griddep_wait();
+            for (int c = 0; c < pk; ++c) {
+                load_kvec(c);
+                if (c < pv) load_t2(c);
             }
-            for (int c = max(0, issued - 3); c < issued; ++c) drain_bar(&bar[FULLK + c % 3], kpar(c));
-            for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULLV + (c & 1)], vpar(c));
+            int k_issued = pk, v_issued = pv;  // chunks whose K (V) part is in flight or landed
+            for (int c = pv; c < nch; ++c) {
+                if (c >= k_issued) {
+                    if (!wait_bar(&bar[EMPTYK + c % 3], kpar(c - 3), ctl, err)) break;
+                    load_k(c);
+                    load_kvec(c);
+                    k_issued = c + 1;
+                }
+                if (!wait_bar(&bar[EMPTYV + (c & 1)], vpar(c - 2), ctl, err)) break;
+                load_v(c);
+                load_t2(c);
+                v_issued = c + 1;
+            }
+            // at most three K and two V loads can be outstanding (one per ring slot)
+            for (int c = max(0, k_issued - 3); c < k_issued; ++c) drain_bar(&bar[FULLK + c % 3], kpar(c));
+            for (int c = max(0, v_issued - 2); c < v_issued; ++c) drain_bar(&bar[FULLV + (c & 1)], vpar(c));
         }
     } else if (warp == W_WMMA) {
         // ---------------------------------------------------------------- W issuer: W^T = K^T T1^T, U^T = V^T T2^T
