@@ -859,13 +859,11 @@ constexpr uint32_t DTX = DTS + 16384;
 constexpr uint32_t BAR = DTX + 16384;
 constexpr uint32_t TOTAL = BAR + 320;
 // link phase (after the chunk loop every tile is free)
-constexpr uint32_t SIN = 0;      // S_in hi | lo as A operands (rows v, runs along k; sy = 2048)
-constexpr uint32_t PHI = 65536;  // two buffers: Phi_j hi | lo as B operands (rows k, runs along k'; sy = 2048)
+constexpr uint32_t PHI = 0;  // two buffers: Phi_j hi | lo as B operands (rows k, runs along k'; sy = 2048)
 // TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T;
-// in the link phase two fold accumulators take the columns from TM_F on, and once Phi has been
-// read out of X, the fold's A operand split(S_end(j)) takes X's columns: for K step kk (16 values
-// of k), 8 columns of bf16 pairs hi then 8 of lo, at TM_A + 16 kk
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_F = 256, TM_A = 128;
+// in the link phase the fold's product P takes TM_D and its A operand split(S_end(j)) TM_A: for K
+// step kk (16 values of k), 8 columns of bf16 pairs hi then 8 of lo, at TM_A + 16 kk
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_D = 256, TM_A = 384;
 // Three MMA issuers: S chain, X chain, and the W issuer (the next chunk's W^T, U^T).
 // A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
 // kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
@@ -884,19 +882,19 @@ enum {
     FINX = 27,  // the same for the X issuer
     FINW = 28,  // the same for the W issuer
     // link phase, fold step j (buffer j & 1 where there are two)
-    LNK = 29,     // the first segment's end state landed in SIN
-    AREADY = 30,  // [2] split(S_end(j)) is in TM_A and fold accumulator j & 1 is read (S warps, 256)
-    PFULL = 32,   // [2] Phi_j landed
-    MDONE = 34,   // [2] the step's MMAs are done
-    DINIT = 36,   // [2] fold accumulator j & 1 holds S_loc(j) (X warps, 256)
-    NBAR = 38
+    A1R = 29,     // the first step's A is in TM_A (S warps, 256)
+    AREADY = 30,  // split(S_end(j)) is in TM_A and P has been read (S and X warps, 512)
+    PFULL = 31,   // [2] Phi_j landed
+    MDONE = 33,   // [2] the step's MMAs are done
+    NBAR = 35
 };
 // (EMPTYK takes a commit from each issuer: count 2 with an X chain, 1 without.)
 __device__ __forceinline__ constexpr uint32_t bar_count(int i, bool has_x) {
     return (i >= EMPTYK && i < EMPTYK + 3)                                  ? (has_x ? 2u : 1u)
            : (i >= T1R && i < KR + 4)                                       ? 128u
            : (i >= SR && i <= DXR)                                          ? 256u
-           : ((i >= AREADY && i < AREADY + 2) || (i >= DINIT && i < DINIT + 2)) ? 256u
+           : (i == A1R)                                                     ? 256u
+           : (i == AREADY)                                                  ? 512u
                                                                             : 1u;
 }
 static_assert(BAR + 8 * NBAR + 8 <= TOTAL, "barrier area");
@@ -1148,13 +1146,15 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     // S_end(j) = S_loc(j) + S_end(j - 1) Phi(j) along the sequence's segments. Every segment after
     // the first publishes its part (Phi, S_loc) as soon as its chunk loop ends; segment s then folds
     // the parts of segments 1 .. s itself, starting from the first segment's published end state,
-    // instead of waiting for its predecessor's end state (a chain of s cross-CTA hand-offs). Each
-    // fold step is the arithmetic of the chained form: bf16 hi/lo split operands (hi hi + hi lo +
-    // lo hi) accumulated in fp32 onto S_loc(j), so both give the same bits.
-    //   X warps   publish the part, then load S_loc(j) into fold accumulator j & 1 (TMEM)
-    //   loader    the first segment's end state (SIN, the first step's A), Phi_j into buffer j & 1
-    //   S issuer  the step's 24 MMAs; the last step accumulates onto this segment's own S_loc
-    //   S warps   split the step's result into TM_A, the next step's A; publish S_end(s)
+    // instead of waiting for its predecessor's end state (a chain of s cross-CTA hand-offs). A step
+    // is P = split(S_end(j - 1)) Phi(j) on the tensor cores (bf16 hi/lo operands: hi hi + hi lo +
+    // lo hi, fp32 accumulation; A in TMEM), then S_end(j) = P + S_loc(j) in fp32 and its split for
+    // the next step; the last step accumulates onto this segment's own S_loc in TMEM.
+    //   X warps   publish the part (Phi from X, S_loc from S)
+    //   S warps   the first step's A = the first segment's published end state (already split)
+    //   loader    Phi_j into buffer j & 1
+    //   S issuer  the step's 24 MMAs
+    //   S, X warps  (16, 32 columns each) add S_loc(j) and split into TM_A; S warps publish S_end(s)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -1163,60 +1163,91 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     const size_t slot0 = (size_t)(gseg - sg.s) * H + h;  // the sequence's first segment
     auto part_of = [&](int j) { return part + (slot0 + (size_t)j * H) * PART_BYTES; };
     if (has_x) {
-        if (warp >= 8 && warp < 16) {
-            const int r = quarter_lane, half = (warp >> 2) & 1;
+        if (warp < 16) {
+            const int r = quarter_lane;
             const uint32_t tl = lane_base(tm, warp);
-            if (ok) {
-                uint8_t *pt = part_of(nfold);
-                float4 *ps = reinterpret_cast<float4 *>(pt + PART_S);
+            if (warp >= 8) {
+                const int half = (warp >> 2) & 1;
+                if (ok) {
+                    uint8_t *pt = part_of(nfold);
+                    float4 *ps = reinterpret_cast<float4 *>(pt + PART_S);
 #pragma unroll 1
-                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                    float x[32];
-                    tc::tmem_ld32(tl + TM_X + c0, x);
-                    st_split32_global(pt + PART_PHI, r, c0, x);
-                    tc::tmem_ld32(tl + TM_S + c0, x);
+                    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                        float x[32];
+                        tc::tmem_ld32(tl + TM_X + c0, x);
+                        st_split32_global(pt + PART_PHI, r, c0, x);
+                        tc::tmem_ld32(tl + TM_S + c0, x);
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        ps[((c0 + i) >> 2) * D + r] = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                        for (int i = 0; i < 32; i += 4)
+                            ps[((c0 + i) >> 2) * D + r] = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+                    }
+                    __threadfence();
                 }
-                __threadfence();
+                tc::fence_before_sync();  // the reads of S_loc precede the own fold step, which accumulates onto it
+                tc::named_sync(1, 256);
+                if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
+            } else if (ok) {
+                const int half = (warp >> 2) & 1;
+                if ((ok = __all_sync(0xffffffffu, wait_flag(flags + slot0, ctl, err)))) {
+                    const uint8_t *src = link + slot0 * LINK_BYTES;
+#pragma unroll 1
+                    for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
+                        // K step c0 / 16: the hi runs of columns c0 .., c0 + 8 .., then the lo runs
+                        const uint4 h0 = __ldcg(reinterpret_cast<const uint4 *>(src + tc::tile_off(r, c0, 128, 2048)));
+                        const uint4 h1 = __ldcg(reinterpret_cast<const uint4 *>(src + tc::tile_off(r, c0 + 8, 128, 2048)));
+                        const uint4 l0 = __ldcg(reinterpret_cast<const uint4 *>(src + 32768 + tc::tile_off(r, c0, 128, 2048)));
+                        const uint4 l1 =
+                            __ldcg(reinterpret_cast<const uint4 *>(src + 32768 + tc::tile_off(r, c0 + 8, 128, 2048)));
+                        const float u[16] = {__uint_as_float(h0.x), __uint_as_float(h0.y), __uint_as_float(h0.z),
+                                             __uint_as_float(h0.w), __uint_as_float(h1.x), __uint_as_float(h1.y),
+                                             __uint_as_float(h1.z), __uint_as_float(h1.w), __uint_as_float(l0.x),
+                                             __uint_as_float(l0.y), __uint_as_float(l0.z), __uint_as_float(l0.w),
+                                             __uint_as_float(l1.x), __uint_as_float(l1.y), __uint_as_float(l1.z),
+                                             __uint_as_float(l1.w)};
+                        tc::tmem_st16(tl + TM_A + c0, u);
+                    }
+                    tc::tmem_st_wait();
+                }
+                tc::fence_before_sync();
+                tc::mbar_arrive(&bar[A1R]);
             }
-            tc::fence_before_sync();  // the reads of S_loc precede the own fold step, which accumulates onto it
-            tc::named_sync(1, 256);
-            if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
+            // S_end(j) = P + S_loc(j) and its split, steps 1 .. nfold - 1 (columns c0 .. c0 + 31)
+            const int c0 = 32 * (warp >> 2);
             for (int j = 1; ok && j < nfold; ++j) {
                 const int b = j & 1;
-                // accumulator b was last read by the split of step j - 2
-                if (j >= 3 && !(ok = wait_bar(&bar[AREADY + b], (uint32_t)(((j - 3) >> 1) & 1), ctl, err))) break;
                 if (!(ok = __all_sync(0xffffffffu, wait_flag(pflags + slot0 + (size_t)j * H, ctl, err)))) break;
-                tc::fence_after_sync();
-                const float4 *src = reinterpret_cast<const float4 *>(part_of(j) + PART_S);
-#pragma unroll 1
-                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-                    float x[32];
+                const float4 *src = reinterpret_cast<const float4 *>(part_of(j) + PART_S) + (c0 >> 2) * D + r;
+                float4 sl[8];  // in flight during the step's MMAs
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 p4 = __ldcg(src + ((c0 + i) >> 2) * D + r);
-                        x[i] = p4.x;
-                        x[i + 1] = p4.y;
-                        x[i + 2] = p4.z;
-                        x[i + 3] = p4.w;
+                for (int i = 0; i < 8; ++i) sl[i] = __ldcg(src + i * D);
+                if (!(ok = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err))) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    float x[16], u[16];
+                    tc::tmem_ld16(tl + TM_D + c0 + 16 * t, x);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 s4 = sl[4 * t + (i >> 1)];
+                        const float a0 = x[2 * i] + ((i & 1) ? s4.z : s4.x);
+                        const float a1 = x[2 * i + 1] + ((i & 1) ? s4.w : s4.y);
+                        const float h0 = __bfloat162float(__float2bfloat16_rn(a0));
+                        const float h1 = __bfloat162float(__float2bfloat16_rn(a1));
+                        u[i] = __uint_as_float(tc::pack_bf16x2(h0, h1));
+                        u[8 + i] = __uint_as_float(tc::pack_bf16x2(a0 - h0, a1 - h1));
                     }
-                    tc::tmem_st32(tl + TM_F + 128 * b + c0, *reinterpret_cast<uint32_t(*)[32]>(x));
+                    tc::tmem_st16(tl + TM_A + c0 + 16 * t, u);
                 }
                 tc::tmem_st_wait();
-                handoff(&bar[DINIT + b]);
+                tc::fence_before_sync();
+                tc::mbar_arrive(&bar[AREADY]);
             }
+            if (warp < 8 && ok)
+                ok = wait_bar(&bar[MDONE + (nfold & 1)], (uint32_t)(((nfold - 1) >> 1) & 1), ctl, err);
         } else if (warp == W_LOAD) {
             if (lane == 0 && ok) {
                 int last[2] = {0, 0};
-                bool lnk = false, good = wait_flag(flags + slot0, ctl, err);
-                if (good) {
-                    tc::fence_proxy_async_global();
-                    tc::mbar_arrive_expect_tx(&bar[LNK], LINK_BYTES);
-                    tc::bulk_load(sb + SIN, link + slot0 * LINK_BYTES, LINK_BYTES, &bar[LNK]);
-                    lnk = true;
-                }
+                bool good = true;
                 for (int j = 1; good && j <= nfold; ++j) {
                     const int b = j & 1;
                     // buffer b was last read by step j - 2
@@ -1228,7 +1259,6 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                     tc::bulk_load(sb + PHI + 65536u * b, part_of(j) + PART_PHI, 65536u, &bar[PFULL + b]);
                     last[b] = j;
                 }
-                if (lnk) drain_bar(&bar[LNK], 0);
                 for (int b = 0; b < 2; ++b)
                     if (last[b]) drain_bar(&bar[PFULL + b], (uint32_t)(((last[b] - 1) >> 1) & 1));
             }
@@ -1238,64 +1268,23 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 for (int j = 1; j <= nfold; ++j) {
                     const int b = j & 1;
                     const bool own = j == nfold;
-                    if (!(j == 1 ? wait_bar(&bar[LNK], 0, ctl, err)
-                                 : wait_bar(&bar[AREADY + ((j - 1) & 1)], (uint32_t)(((j - 2) >> 1) & 1), ctl, err)))
+                    if (!(j == 1 ? wait_bar(&bar[A1R], 0, ctl, err)
+                                 : wait_bar(&bar[AREADY], (uint32_t)((j - 2) & 1), ctl, err)))
                         break;
                     if (!wait_bar(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
-                    if (!own && !wait_bar(&bar[DINIT + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
                     tc::fence_after_sync();
-                    const uint32_t d = tm + (own ? TM_S : TM_F + 128u * b), phi = sb + PHI + 65536u * b;
-                    if (j == 1) {
+                    const uint32_t d = tm + (own ? TM_S : TM_D), phi = sb + PHI + 65536u * b;
 #pragma unroll 1
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t ah = tc::make_desc(sb + SIN + kk * 4096, 2048, 128);
-                            const uint64_t al = tc::make_desc(sb + SIN + 32768 + kk * 4096, 2048, 128);
-                            const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
-                            const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
-                            tc::mma_bf16(d, ah, bh, id_km128, 1);
-                            tc::mma_bf16(d, ah, bl, id_km128, 1);
-                            tc::mma_bf16(d, al, bh, id_km128, 1);
-                        }
-                    } else {
-#pragma unroll 1
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t ah = tm + TM_A + 16 * kk, al = ah + 8;
-                            const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
-                            const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
-                            tc::mma_bf16_ts(d, ah, bh, id_km128, 1);
-                            tc::mma_bf16_ts(d, ah, bl, id_km128, 1);
-                            tc::mma_bf16_ts(d, al, bh, id_km128, 1);
-                        }
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ah = tm + TM_A + 16 * kk, al = ah + 8;
+                        const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
+                        const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
+                        tc::mma_bf16_ts(d, ah, bh, id_km128, (own || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16_ts(d, ah, bl, id_km128, 1);
+                        tc::mma_bf16_ts(d, al, bh, id_km128, 1);
                     }
                     tc::mma_commit(&bar[MDONE + b]);
                 }
-            }
-        } else if (warp < 8 && ok) {
-            const int v = quarter_lane, half = (warp >> 2) & 1;
-            const uint32_t tl = lane_base(tm, warp);
-            for (int j = 1; j <= nfold; ++j) {
-                const int b = j & 1;
-                if (!(ok = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err))) break;
-                if (j == nfold) break;
-                tc::fence_after_sync();
-#pragma unroll 1
-                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
-                    // columns c0 .. c0 + 15 are K step c0 / 16: 8 columns of hi pairs, then 8 of lo
-                    float x[16];
-                    tc::tmem_ld16(tl + TM_F + 128 * b + c0, x);
-                    float u[16];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float h0 = __bfloat162float(__float2bfloat16_rn(x[2 * i]));
-                        const float h1 = __bfloat162float(__float2bfloat16_rn(x[2 * i + 1]));
-                        u[i] = __uint_as_float(tc::pack_bf16x2(h0, h1));
-                        u[8 + i] = __uint_as_float(tc::pack_bf16x2(x[2 * i] - h0, x[2 * i + 1] - h1));
-                    }
-                    tc::tmem_st16(tl + TM_A + c0, u);
-                }
-                tc::tmem_st_wait();
-                tc::fence_before_sync();
-                tc::mbar_arrive(&bar[AREADY + b]);
             }
         }
     }
