@@ -872,7 +872,7 @@ __global__ void __launch_bounds__(256) k_plan(const int32_t *__restrict__ cu, in
 
 // Diagnostic wrapper of the solve: one 64 x 64 strictly lower fp32 matrix.
 __global__ void __launch_bounds__(NT) k_diag_ut_solve(const float *__restrict__ Ag, float *__restrict__ Tg) {
-    __shared__ float A[64 * AP], T[64 * AP], X[32 * ut::XP];
+    __shared__ __align__(16) float A[64 * AP], T[64 * AP], X[32 * ut::XP];
     for (int e = threadIdx.x; e < 64 * 64; e += NT) A[(e >> 6) * AP + (e & 63)] = Ag[e];
     __syncthreads();
     ut::solve64(A, T, X);

@@ -468,38 +468,49 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
             break;
         }
         if (tid == 32 && wn < items) issue_k(wn);  // the product has read the K buffer
-        // ---- A_rs = beta_r exp(G_r - G_s) X1_rs for s < r (warp w: rows 16 (w%4) + lane, columns 32 (w/4) ..)
+        // ---- A_rs = beta_r exp(G_r - G_s) X1_rs for s < r (warp w: rows 16 (w%4) + lane % 16, columns
+        // 32 (w/4) + 16 (lane / 16) ..: the accumulator rows sit in lanes 0-15, whose upper 16 columns
+        // lanes 16-31 take over by shuffle)
         {
-            const int lane = tid & 31, r = 16 * (warp & 3) + (lane & 15), s0 = 32 * (warp >> 2);
+            const int lane = tid & 31, l16 = lane & 15, hf = lane >> 4;
+            const int r = 16 * (warp & 3) + l16, c0 = 32 * (warp >> 2) + 16 * hf;
             float x[32];
-            tc::tmem_ld32(tl + s0, x);  // all lanes load (the instruction is warp-wide); lanes >= 16 discard
-            if (lane < 16) {
-                const float Gr = Gl[r], br = bet[r];
+            tc::tmem_ld32(tl + 32 * (warp >> 2), x);  // warp-wide; lanes >= 16 receive nothing of use
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    float4 a;
-                    a.x = (s0 + i < r) ? br * ex2(Gr - Gl[s0 + i]) * x[i] : 0.f;
-                    a.y = (s0 + i + 1 < r) ? br * ex2(Gr - Gl[s0 + i + 1]) * x[i + 1] : 0.f;
-                    a.z = (s0 + i + 2 < r) ? br * ex2(Gr - Gl[s0 + i + 2]) * x[i + 2] : 0.f;
-                    a.w = (s0 + i + 3 < r) ? br * ex2(Gr - Gl[s0 + i + 3]) * x[i + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(AT + r * AP + s0 + i) = a;
-                }
+            for (int i = 0; i < 16; ++i) {
+                const float y = __shfl_sync(0xffffffffu, x[16 + i], l16);
+                x[i] = hf ? y : x[i];
+            }
+            const float Gr = Gl[r], br = bet[r];
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+                const float4 g4 = *reinterpret_cast<const float4 *>(Gl + c0 + i);
+                float4 a;
+                a.x = (c0 + i < r) ? br * ex2(Gr - g4.x) * x[i] : 0.f;
+                a.y = (c0 + i + 1 < r) ? br * ex2(Gr - g4.y) * x[i + 1] : 0.f;
+                a.z = (c0 + i + 2 < r) ? br * ex2(Gr - g4.z) * x[i + 2] : 0.f;
+                a.w = (c0 + i + 3 < r) ? br * ex2(Gr - g4.w) * x[i + 3] : 0.f;
+                *reinterpret_cast<float4 *>(AT + r * AP + c0 + i) = a;
             }
         }
         if (tid == 0) tc::bulk_wait_read();  // the previous record has left the staging area (written after the solve)
         tc::fence_before_sync();
         __syncthreads();
         ut::solve64(AT, AT, reinterpret_cast<float *>(smem + pp::XS));
-        // ---- T2 = T diag(beta) as a bf16 operand tile (thread: row tid / 4, 16 columns)
-        {
-            const int r = tid >> 2, s0 = 16 * (tid & 3);
-            float x[16];
+        // ---- T2 = T diag(beta) as a bf16 operand tile: 16-byte runs (row r, columns 8 j ..), eight
+        // consecutive rows per eight lanes (conflict-free rows of T, contiguous runs of the tile)
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = AT[r * AP + s0 + i] * bet[s0 + i];
-            st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0, 128, 1024), x);
-            st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, s0 + 8, 128, 1024), x + 8);
-            reinterpret_cast<float *>(smem + pp::REC + REC_VEC)[tid] = vec[tid];
+        for (int k = 0; k < 2; ++k) {
+            const int idx = tid + 256 * k, r = (idx & 7) + 8 * ((idx >> 3) & 7), j = idx >> 6;
+            const float4 t0 = *reinterpret_cast<const float4 *>(AT + r * AP + 8 * j);
+            const float4 t1 = *reinterpret_cast<const float4 *>(AT + r * AP + 8 * j + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(bet + 8 * j);
+            const float4 b1 = *reinterpret_cast<const float4 *>(bet + 8 * j + 4);
+            const float x[8] = {t0.x * b0.x, t0.y * b0.y, t0.z * b0.z, t0.w * b0.w,
+                                t1.x * b1.x, t1.y * b1.y, t1.z * b1.z, t1.w * b1.w};
+            st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, 8 * j, 128, 1024), x);
         }
+        reinterpret_cast<float *>(smem + pp::REC + REC_VEC)[tid] = vec[tid];
         tc::fence_smem_to_async();
         __syncthreads();
         if (tid == 0) {

@@ -63,7 +63,7 @@ __device__ __forceinline__ void warp_store(float *Z, int p, const float (&d)[4],
 }
 
 // Block-wide solve; requires blockDim.x == 256. A, T: [64][AP] fp32 in shared
-// memory (A zero on and above the diagonal). X: scratch of 32 * XP floats.
+// memory, 16-byte aligned (A zero on and above the diagonal). X: scratch of 32 * XP floats.
 // T may be the same buffer as A: every block of A is read (and the reads
 // synchronised) before the block of T at its place is written. Ends with a
 // __syncthreads.
@@ -76,9 +76,17 @@ __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
+                // row i of the block in 16-byte broadcast loads (rows are 16-byte aligned: AP % 4 == 0)
+                const float *arow = A + (o + i) * AP + o;
                 float acc = (i == j) ? 1.f : 0.f;
 #pragma unroll
-                for (int s = 0; s < i; ++s) acc = fmaf(-A[(o + i) * AP + o + s], x[s], acc);
+                for (int s4 = 0; s4 < i; s4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + s4);
+                    acc = fmaf(-a4.x, x[s4], acc);
+                    if (s4 + 1 < i) acc = fmaf(-a4.y, x[s4 + 1], acc);
+                    if (s4 + 2 < i) acc = fmaf(-a4.z, x[s4 + 2], acc);
+                    if (s4 + 3 < i) acc = fmaf(-a4.w, x[s4 + 3], acc);
+                }
                 x[i] = acc;
             }
             __syncwarp(0x0000ffffu);  // every lane has read its block of A before T overwrites it (A may be T)
