@@ -71,10 +71,13 @@ const char *gdn_last_error(void);
 /*
  * Workspace bytes with which gdn_chunk_fwd runs its fastest plan for these
  * sizes (always >= 256). Any workspace of at least 256 bytes (the device
- * error word) is accepted: when there are few (sequence, head) pairs the
- * bf16 path splits each sequence into segments that run in parallel and
- * keeps two fp32 d x d matrices per (segment, head) in the workspace; a
- * smaller workspace selects fewer segments, down to none. The workspace is
+ * error word) is accepted. The bf16 path keeps a 9 KB record per (chunk,
+ * head) (the chunk's solved triangular factor and decay vectors); when there
+ * are few (sequence, head) pairs it also splits each sequence into segments
+ * that run in parallel and keeps, per (segment, head), the segment's end
+ * state and its affine map (together 192 KB, three d x d fp32 matrices' worth);
+ * a smaller workspace selects fewer segments, down to none, then a path
+ * without records. The workspace is
  * scratch owned by the caller: its contents on entry are ignored and on exit
  * are meaningless except for the error word read by gdn_chunk_fwd_check.
  * Two calls that overlap on the GPU must not share a workspace.
