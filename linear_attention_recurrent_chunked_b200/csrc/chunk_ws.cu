@@ -224,8 +224,8 @@ __device__ __forceinline__ void state_init64(uint32_t s_tile, uint32_t tl_s, int
         for (int h8 = 0; h8 < 32; h8 += 8) {
             if (link) {
                 const uint32_t off = tc::tile_off(v, c0 + h8, 128, 2048);
-                uint4 hi = *reinterpret_cast<const uint4 *>(link + off);
-                uint4 lo = *reinterpret_cast<const uint4 *>(link + 32768 + off);
+                const uint4 hi = __ldcg(reinterpret_cast<const uint4 *>(link + off));
+                const uint4 lo = __ldcg(reinterpret_cast<const uint4 *>(link + 32768 + off));
                 const uint32_t *wh = reinterpret_cast<const uint32_t *>(&hi);
                 const uint32_t *wl = reinterpret_cast<const uint32_t *>(&lo);
 #pragma unroll
@@ -569,18 +569,24 @@ __global__ void __launch_bounds__(NT_WS, 1)
              const float *S0, const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o,
              float *S_T, uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off,
              const int32_t *__restrict__ chunk_off, int seg_chunks, const uint8_t *__restrict__ rec,
-             const uint8_t *__restrict__ link) {
+             const uint8_t *__restrict__ link, const uint32_t *__restrict__ flags) {
     using namespace ob;
     extern __shared__ __align__(1024) uint8_t smem[];
-    // The loader waits for the predecessor grid only after it has started the first chunks' Q, K, V
-    // loads (inputs, which no kernel of the call writes); the plan (error word, offsets) is complete
-    // before the predecessor can launch this grid.
-    if ((threadIdx.x >> 5) != W_LOAD) griddep_wait();
+    // What this CTA waits for before reading what earlier passes wrote (the plan's error word and
+    // offsets are complete before the preceding grid can launch this one):
+    //  * a segment of a split sequence: the end-state flag it starts from, published by the
+    //    transition pass (the previous segment's; for the first segment its own, published after
+    //    that transition CTA had waited for the records) - not the whole transition grid, so the
+    //    CTA can start while later transition CTAs still fold;
+    //  * otherwise the preceding grid (the loader, after starting the first chunks' Q, K, V loads).
     griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
     const int h = blockIdx.x;
     if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg)) return;
+    const bool split = flags != nullptr && sg.ns > 1;
+    const uint32_t *start_flag = split ? flags + ((size_t)blockIdx.y - (sg.s > 0 ? 1 : 0)) * H + h : nullptr;
+    if (!split && (threadIdx.x >> 5) != W_LOAD) griddep_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = tc::smem_u32(smem);
     if (sb & 1023u) {
@@ -627,7 +633,9 @@ __global__ void __launch_bounds__(NT_WS, 1)
             };
             const int pre = min(nch, 2);
             for (int c = 0; c < pre; ++c) load_inputs(c);
-            griddep_wait();
+            // (a failed or timed-out flag aborts the CTA; the record loads still complete the barriers)
+            if (split) wait_flag(start_flag, ctl, err);
+            else griddep_wait();
             for (int c = 0; c < pre; ++c) load_record(c);
             int issued = pre;
             for (int c = pre; c < nch; ++c) {
@@ -728,6 +736,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             ok = wait_bar(&bar[FULL], 0, ctl, err);
             if (ok) g0 = vecp(0)[64 + C - 1];
         }
+        if (ok && split && sg.s > 0) ok = __all_sync(0xffffffffu, wait_flag(start_flag, ctl, err));
         if (ok) {
             const uint8_t *lk = nullptr;
             const float *src = nullptr;
@@ -847,6 +856,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
         tc::mma_commit(&bar[FIN]);
         drain_bar(&bar[FIN], 0);
     }
+    if (split && tid == 0) griddep_wait();  // complete only after the transition grid (the stream's next work reuses the workspace)
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 0) tc::tmem_dealloc(tm, 512);
@@ -1547,7 +1557,8 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     pr = prof_start("ws_out", st);
     e = launch_pdl(k_ws_out, dim3(H, l.nslots), dim3(NT_WS), ob::TOTAL, st, tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot,
                    H, o, S_T, err, seg_chunks > 0 ? (const int32_t *)seg_off : nullptr, (const int32_t *)chunk_off,
-                   seg_chunks > 0 ? seg_chunks : 1, (const uint8_t *)rec, (const uint8_t *)link);
+                   seg_chunks > 0 ? seg_chunks : 1, (const uint8_t *)rec, (const uint8_t *)link,
+                   seg_chunks > 0 ? (const uint32_t *)flags : nullptr);
     prof_stop(pr);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
