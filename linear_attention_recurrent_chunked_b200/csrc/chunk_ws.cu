@@ -574,18 +574,24 @@ __global__ void __launch_bounds__(NT_WS, 1)
     extern __shared__ __align__(1024) uint8_t smem[];
     // What this CTA waits for before reading what earlier passes wrote (the plan's error word and
     // offsets are complete before the preceding grid can launch this one):
-    //  * a segment of a split sequence: the end-state flag it starts from, published by the
-    //    transition pass (the previous segment's; for the first segment its own, published after
-    //    that transition CTA had waited for the records) - not the whole transition grid, so the
-    //    CTA can start while later transition CTAs still fold;
+    //  * with a transition pass before this one (flags given): a later segment of a split
+    //    sequence, the end-state flag of the segment before it (which also orders it after the
+    //    records); an unsplit sequence, or the first of two segments, the records flag the
+    //    transition CTAs set once the prep grid is complete; the first of three or more segments,
+    //    its own end-state flag (a short segment whose output is off the critical path: started
+    //    early it would only compete with the transition CTAs that are on it). Not the whole
+    //    transition grid, so output CTAs run beside transition CTAs that still run or fold;
     //  * otherwise the preceding grid (the loader, after starting the first chunks' Q, K, V loads).
     griddep_launch();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
     const int h = blockIdx.x;
     if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg)) return;
-    const bool split = flags != nullptr && sg.ns > 1;
-    const uint32_t *start_flag = split ? flags + ((size_t)blockIdx.y - (sg.s > 0 ? 1 : 0)) * H + h : nullptr;
+    const bool split = flags != nullptr;
+    const uint32_t *start_flag = !split             ? nullptr
+                                 : sg.s > 0         ? flags + ((size_t)blockIdx.y - 1) * H + h
+                                 : sg.ns >= 3       ? flags + (size_t)blockIdx.y * H + h
+                                                    : flags + (size_t)2 * gridDim.y * H;
     if (!split && (threadIdx.x >> 5) != W_LOAD) griddep_wait();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = tc::smem_u32(smem);
@@ -937,8 +943,19 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
     const int h = blockIdx.x;
-    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg)) return;
-    if (sg.s == sg.ns - 1) return;  // the last segment's end state is never needed
+    // Records flag (after all end-state and part flags): set once the prep grid is complete, so
+    // that output CTAs that need only the records start without waiting for this grid.
+    uint32_t *rec_flag = pflags + (size_t)gridDim.y * H;
+    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg) || sg.s == sg.ns - 1) {
+        // (the last segment's end state is never needed.) CTA (0, 0), which sets the records flag
+        // from its loader when it has work, sets it here when it has none (no sequence is split);
+        // the others leave at once.
+        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) {
+            griddep_wait();
+            tc::st_release_gpu(rec_flag, FLAG_DONE);
+        }
+        return;
+    }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = tc::smem_u32(smem);
     const int gseg = blockIdx.y;
@@ -999,6 +1016,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 load_kvec(c);
                 if (c < pv) load_t2(c);
             }
+            // CTA (0, 0) (the first segment of the first sequence: no Phi chain, no fold) sets the
+            // records flag, after its first record loads so that the store's fence is not on their path
+            if (blockIdx.x == 0 && blockIdx.y == 0) tc::st_release_gpu(rec_flag, FLAG_DONE);
             int k_issued = pk, v_issued = pv;  // chunks whose K (V) part is in flight or landed
             for (int c = pv; c < nch; ++c) {
                 if (c >= k_issued) {
@@ -1461,7 +1481,7 @@ WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
     l.seg_off = 256;
     l.chunk_off = l.seg_off + align256((size_t)(N + 1) * 4);
     l.flags = l.chunk_off + align256((size_t)(N + 1) * 4);
-    l.s0copy = l.flags + align256((size_t)2 * l.nslots * H * 4);  // end-state flags, then part flags
+    l.s0copy = l.flags + align256(((size_t)2 * l.nslots * H + 1) * 4);  // end-state flags, part flags, records flag
     l.rec = l.s0copy + (seg_chunks > 0 ? (size_t)N * H * D * D * sizeof(float) : 0);
     l.link = l.rec + align256((size_t)l.nc_bound * H * REC_BYTES);
     l.part = l.link + (seg_chunks > 0 ? (size_t)l.nslots * H * LINK_BYTES : 0);
@@ -1478,11 +1498,17 @@ WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
 // Time ~ n/s (t_trans + t_out) + (s - 1) t_link is smallest near s = sqrt(n)
 // (a link costs about as much as a chunk); a sweep on B200 put the best count
 // at about 1.2 sqrt(n), capped so that all CTAs fit on the GPU at once.
-int chunk_ws_seg_chunks(int N, int T_tot, int H) {
+//
+// Many pairs of sequences of different lengths (varlen): one CTA per (sequence, head) already
+// fills the GPU, but the longest sequences set the time. When the pairs fit in one wave, a segment
+// length of 1.25 x the average splits only the sequences longer than that; their first segment's
+// transition CTA runs beside the other sequences' output CTAs.
+int chunk_ws_seg_chunks(int N, int T_tot, int H, bool varlen) {
     const long pairs = (long)N * H;
     const long nc_avg = ((long)T_tot / N + C - 1) / C;
     const int sms = num_sms();
-    if (pairs * 2 > sms || nc_avg < 8) return 0;
+    if (pairs * 2 > sms) return (varlen && N > 1 && pairs <= sms && nc_avg >= 8) ? (int)((5 * nc_avg + 3) / 4) : 0;
+    if (nc_avg < 8) return 0;
     long s = 1;
     while (100 * s * s < 144 * nc_avg) ++s;  // ceil(1.2 sqrt(nc_avg))
     s = std::min(s, (long)sms / pairs);
@@ -1522,7 +1548,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     }
     *stage = "plan";
     void *pr = prof_start("ws_plan", st);
-    const int nflags = seg_chunks > 0 ? 2 * l.nslots * H : 0;
+    const int nflags = seg_chunks > 0 ? 2 * l.nslots * H + 1 : 0;
     k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
     prof_stop(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

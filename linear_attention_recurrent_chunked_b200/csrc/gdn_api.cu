@@ -156,7 +156,9 @@ const char *gdn_last_error(void) { return g_msg; }
 
 size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype) {
     if (dtype == GDN_BF16 && dk == 128 && dv == 128 && N >= 1 && H >= 1 && T_tot >= 0)
-        return std::max(kErrWordBytes, gdn::chunk_ws_workspace(N, T_tot, H, gdn::chunk_ws_seg_chunks(N, T_tot, H)));
+        // (the plan differs with and without cu_seqlens; the larger workspace covers both)
+        return std::max({kErrWordBytes, gdn::chunk_ws_workspace(N, T_tot, H, gdn::chunk_ws_seg_chunks(N, T_tot, H, false)),
+                         gdn::chunk_ws_workspace(N, T_tot, H, gdn::chunk_ws_seg_chunks(N, T_tot, H, true))});
     return kErrWordBytes;
 }
 
@@ -184,7 +186,7 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
         const char *stage = "";
         // The pipelined path needs room for one prep record per (chunk, head) (and, split into
         // segments, the published segment states); with less workspace the single-kernel path runs.
-        const int seg = gdn::chunk_ws_seg_chunks(N, T_tot, H);
+        const int seg = gdn::chunk_ws_seg_chunks(N, T_tot, H, cu_seqlens != nullptr);
         const int use_seg = ws_bytes >= gdn::chunk_ws_workspace(N, T_tot, H, seg) ? seg : 0;
         if (ws_bytes >= gdn::chunk_ws_workspace(N, T_tot, H, use_seg)) {
             e = gdn::launch_chunk_ws(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),

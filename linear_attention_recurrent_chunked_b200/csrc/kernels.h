@@ -42,7 +42,7 @@ cudaError_t launch_chunk_ws(const __nv_bfloat16 *q, const __nv_bfloat16 *k, cons
                             const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
                             __nv_bfloat16 *o, float *S_T, void *workspace, int seg_chunks, cudaStream_t st,
                             const char **stage);
-int chunk_ws_seg_chunks(int N, int T_tot, int H);
+int chunk_ws_seg_chunks(int N, int T_tot, int H, bool varlen);  // varlen: cu_seqlens given
 size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks);
 
 // Kernel timing hooks (no-ops unless gdn_profile_enable(1)): an event pair
