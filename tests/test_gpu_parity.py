@@ -267,6 +267,26 @@ def test_segmented_varlen_mixed_segment_counts():
     assert torch.equal(S_T[3].cpu(), w["S0"][3])
 
 
+def test_many_pairs_varlen_nothing_split():
+    """Many (sequence, head) pairs, no sequence longer than 1.25x the average: the transition
+    pass has no work (only its records flag is set) and every output CTA starts from it."""
+    w = make_prefill("varlen", seqlens=[1000, 1010, 990, 1005, 995, 1000, 1002, 998], H=16, d=128, s0=True,
+                     seed=25)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "many pairs, nothing split")
+
+
+def test_many_pairs_varlen_one_long_sequence_split():
+    """Many pairs, one sequence 8x longer than the rest: only it is split (into four segments,
+    so its first segment waits for its own end state) while the unsplit sequences' output CTAs
+    start from the records flag."""
+    w = make_prefill("varlen", seqlens=[512] * 7 + [4096], H=16, d=128, s0=True, stress=True, seed=26)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "many pairs, one sequence split")
+
+
 def test_segmented_slow_decay_stress():
     """Segment transitions matter when the state is remembered across segments."""
     w = make_prefill("prefill_2k", seqlens=[3000], H=1, s0=True, stress=True, seed=22)
