@@ -29,13 +29,19 @@
 //     tensor cores (bf16 hi/lo split operands, fp32 accumulation), and
 //     publishes its own S_end. The first segment starts from S0 and needs no Phi.
 //  3. k_ws_out, one CTA per segment: starts from S0 or the published end
-//     state of the previous segment and writes the outputs (and S_T).
+//     state of the previous segment and writes the outputs (and S_T). After a
+//     transition pass its CTAs start from flags (the end state they need, or
+//     the records being complete), so they run beside transition CTAs that
+//     are still working.
+// Sequences are split when few (sequence, head) pairs would leave SMs idle,
+// and, with packed sequences of different lengths, when one is much longer
+// than the average (chunk_ws_seg_chunks).
 //
 // In 2 and 3 the warps have fixed roles and pass tiles to each other through
 // mbarriers, so that the next chunk's loads and operand preparation and the
 // current chunk's outputs overlap the dependent state step:
 //   loader (1 thread)  K, Q, V by TMA (128-byte swizzle), the record by bulk copy
-//   MMA    (1 thread)  every tcgen05.mma; the state step's two MMAs are issued
+//   MMA    (1 or 3 threads) every tcgen05.mma; the state step's MMAs are issued
 //                      as soon as their inputs are ready, the rest fills in after
 //   state  (8 warps)   Delta^T (accumulated onto U^T in TMEM) -> bf16 tile;
 //                      S -> bf16 tile and S <- gamma_C' S in TMEM, so that the
