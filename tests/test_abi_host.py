@@ -103,6 +103,17 @@ def test_workspace_size_is_positive(lib):
         assert lib.gdn_chunk_fwd_workspace_size(N, T, 16, 128, 128, 1) >= 256
 
 
+def test_workspace_size_covers_segment_states(lib):
+    """Beyond the 9 KB per (chunk, head) records, a plan that splits sequences keeps 192 KB of
+    segment states per (segment slot, head): the reported size must include them, both for few
+    (sequence, head) pairs (every sequence split) and for many pairs of packed sequences, where
+    only the longer ones are split."""
+    rec = lambda N, T, H: ((T + 63 * N) // 64) * H * 9216
+    for N, T, H in ((1, 2048, 16), (1, 10240, 16), (8, 19679, 16)):
+        size = lib.gdn_chunk_fwd_workspace_size(N, T, H, 128, 128, 1)
+        assert size >= rec(N, T, H) + 2 * H * 192 * 1024, (N, T, H, size)
+
+
 def test_binding_refuses_cpu_tensors(lib):
     import torch
     from linear_attention_recurrent_chunked_b200 import gdn
