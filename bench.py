@@ -83,6 +83,20 @@ def measured_traffic(kernel: str, workload: str):
     return float(v) if v is not None else None
 
 
+def kernel_shares(w) -> dict:
+    """Algorithmic bytes each launch of a bf16 prefill call must move itself (the method's
+    inputs and outputs it touches; workspace records excluded): prep reads k, g, beta; the
+    transition pass reads k and v (and S0); the output pass reads q, k, v (and S0) and writes o
+    and S_T. The shares add up to more than the call's bytes, since k is read by all three."""
+    e = 2 if w["dtype"] == "bf16" else 4
+    T, H, d, N = w["T_tot"], w["H"], w["d"], w["N"]
+    tok = T * H * d * e
+    state = N * H * d * d * 4
+    s0 = state if w["S0"] is not None else 0
+    return {"ws_plan": 4 * (N + 1), "ws_prep": tok + 8 * T * H, "ws_trans": 2 * tok + s0,
+            "ws_out": 4 * tok + s0 + state}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -252,29 +266,49 @@ def gpu_arm(args):
         S_T = torch.empty((w["N"], w["H"], w["d"], w["d"]), dtype=torch.float32, device=dev)
         fn = prefill_call(t, o, S_T)
         times = time_steps(fn, steps, warmup)
+        # the device error word of the last call (malformed cu_seqlens, a bounded wait that gave up):
+        # raises unless it reads GDN_OK
+        gdn.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], t["cu_seqlens"], o=o, S_T=S_T,
+                      check=True)
         ms = statistics.mean(times)
         ms_max = max_over_ranks(dist, ms, dev)
         tokens = w["T_tot"]
-        kt = kernel_times(fn, max(3, min(steps, 10)))
-        top = max(kt.items(), key=lambda kv: kv[1][0])
-        top_ms = top[1][0] / top[1][1]
+        reps = max(3, min(steps, 10))
+        kt = kernel_times(fn, reps)
         nbytes, nflops = prefill_bytes(w), prefill_flops(w)
-        gbs = nbytes / (top_ms * 1e-3) / 1e9
+        # The whole call (plan, prep, transition and output launches) is the unit: its
+        # algorithmic bytes over its device time. Per launch, each kernel's own share.
+        gbs = nbytes / (ms_max * 1e-3) / 1e9
+        shares = kernel_shares(w)
+        per_kernel = {}
+        for k, (tot, cnt) in kt.items():
+            k_ms = tot / cnt
+            own = shares.get(k)
+            per_kernel[k] = {"ms_per_launch": k_ms, "launches_per_step": cnt // reps,
+                             "own_bytes": own, "traffic": measured_traffic(k, name)}
+            if own is not None:
+                per_kernel[k]["achieved_GBs"] = own / (k_ms * 1e-3) / 1e9
+                per_kernel[k]["frac"] = per_kernel[k]["achieved_GBs"] / pk["hbm"]
+        traffic = [v["traffic"] for v in per_kernel.values()]
+        traffic = sum(traffic) if traffic and all(x is not None for x in traffic) else None
+        roofline_ms = max(nbytes / (pk["hbm"] * 1e9), nflops / (pk["bf16"] * 1e12)) * 1e3
+        top = max(kt.items(), key=lambda kv: kv[1][0])
         entry = {
             "workload": name, "tokens": tokens, "seqs": w["N"], "H": w["H"], "d": w["d"], "dtype": w["dtype"],
             "ms_per_step": ms_max, "tokens_per_s": ws * tokens / (ms_max * 1e-3),
-            "algorithmic_bytes": nbytes, "algorithmic_flops": nflops,
-            "roofline_ms": max(nbytes / (pk["hbm"] * 1e9), nflops / (pk["bf16"] * 1e12)) * 1e3,
-            "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches_per_step": v[1] // max(3, min(steps, 10))}
-                        for k, v in kt.items()},
-            "top_kernel": top[0],
+            "algorithmic_bytes": nbytes, "algorithmic_flops": nflops, "roofline_ms": roofline_ms,
+            "kernels": per_kernel, "top_kernel": top[0],
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                         "frac": gbs / pk["hbm"], "traffic": measured_traffic(top[0], name),
-                         "peak_source": pk["src"], "kernel": top[0],
-                         "tensor_tflops": nflops / (top_ms * 1e-3) / 1e12},
-            "launches_per_step": sum(v[1] for v in kt.values()) // max(3, min(steps, 10)),
+                         "frac": gbs / pk["hbm"], "traffic": traffic,
+                         "traffic_over_algorithmic": traffic / nbytes if traffic is not None else None,
+                         "peak_source": pk["src"], "kernel": "chunk_fwd call (%s)" % ", ".join(kt),
+                         "scope": "algorithmic bytes of one call over the call's device time (CUDA events); "
+                                  "traffic = DRAM bytes summed over the call's launches",
+                         "tensor_tflops": nflops / (ms_max * 1e-3) / 1e12},
+            "launches_per_step": sum(v[1] for v in kt.values()) // reps,
+            "device_status": "GDN_OK",
         }
-        entry["roofline_frac_step"] = entry["roofline_ms"] / ms_max
+        entry["roofline_frac_step"] = roofline_ms / ms_max
         return w, t, fn, entry
 
     result = {}
@@ -350,6 +384,7 @@ def gpu_arm(args):
                    "state": "fp32", "S0": None, "parallelism": "replicas" if ws > 1 else "single",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "roofline": main["roofline"],
+        "roofline_prefill_10k": (result["prefill_10k"]["roofline"] if "prefill_10k" in result else None),
         "e2e": {"value": ws * tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": main["launches_per_step"] * args.steps,
@@ -360,7 +395,8 @@ def gpu_arm(args):
                    "whole-model prefill 408 tok/s at 2k, 361 tok/s at 10k",
     }
     if rank == 0:
-        line["cpu_baseline"] = cpu_baseline(args)
+        if ws == 1:
+            line["cpu_baseline"] = cpu_baseline(args)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier(device_ids=[dev.index])
@@ -427,23 +463,85 @@ def decode_entry(args, torch, gdn, dev, dist, pk, make_decode):
 
 # ----------------------------------------------------------------------------- CPU oracle arms
 
-def cpu_baseline(args, budget_s: float = 12.0):
-    """The oracle (fp64 scan, C + OpenMP) on the host cores, on a bounded sample of the
-    prefill_2k workload: whole 2k-token passes over all 16 heads, repeated until
-    ~budget_s of CPU time is spent (at least one)."""
-    import oracle
-    from linear_attention_recurrent_chunked_b200.workloads import make_prefill
-    w = make_prefill("prefill_2k", seed=0)
-    args_o = [oracle.as_f64(w[x]) for x in ("q", "k", "v", "g", "beta")]
+def _oracle_rate(run, units: float, budget_s: float) -> tuple:
+    """Repeat run() until budget_s of wall time has passed (at least once); units per second."""
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle.scan(*args_o, S0=None, cu_seqlens=w["cu_seqlens"])
+        run()
         reps += 1
-        if time.perf_counter() - t0 > budget_s or reps >= 50:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": reps * w["T_tot"] / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "%d full prefill_2k passes (2048 tokens x 16 heads, d=128) in %.1f s" % (reps, dt)}
+        dt = time.perf_counter() - t0
+        if dt > budget_s:
+            return reps * units / dt, reps, dt
+
+
+def cpu_baseline(args, budget_s: float = 2.0):
+    """The oracle (fp64 scan, C + OpenMP) timed on the host cores, on all of them and on one,
+    for three workloads, each on a bounded sample (about budget_s of repeats per figure):
+
+    * prefill_2k: all cores, whole 2048-token passes over the 16 heads; one core, 2 of the heads;
+    * prefill_10k: all cores, whole 10240-token passes; one core, 1 head;
+    * decode (256 chained steps, B=64, H=16): all cores, 8 of the 64 sequences; one core, 1.
+      A chain of single-token steps is the scan over that sequence (the oracle's decode step is
+      the scan over length-one sequences), so each sequence runs as a 256-token scan from S.
+
+    Prefill figures are tokens/s of the whole workload (token-heads/s / 16); decode figures are
+    state GB/s (the decode step's algorithmic bytes per (sequence, head) and step)."""
+    import oracle
+    from linear_attention_recurrent_chunked_b200.workloads import make_decode, make_prefill
+    cores = oracle.num_threads()
+    figs = {}
+
+    def prefill_fig(name, heads_1core):
+        w = make_prefill(name, seed=0)
+        H = w["H"]
+        full = [oracle.as_f64(w[x]) for x in ("q", "k", "v", "g", "beta")]
+        S0 = oracle.as_f64(w["S0"])
+        cu = w["cu_seqlens"]
+        rate, reps, dt = _oracle_rate(lambda: oracle.scan(*full, S0=S0, cu_seqlens=cu), w["T_tot"] * H, budget_s)
+        figs["%s_all_cores" % name] = {"value": rate / H, "unit": "tokens/s", "cores": cores,
+                                       "sample": "%d whole passes (%d tokens x %d heads) in %.1f s"
+                                                 % (reps, w["T_tot"], H, dt)}
+        part = [x[:, :heads_1core].copy() for x in full]
+        S0p = S0[:, :heads_1core].copy() if S0 is not None else None
+        oracle.set_num_threads(1)
+        try:
+            rate, reps, dt = _oracle_rate(lambda: oracle.scan(*part, S0=S0p, cu_seqlens=cu),
+                                          w["T_tot"] * heads_1core, budget_s)
+        finally:
+            oracle.set_num_threads(cores)
+        figs["%s_1_core" % name] = {"value": rate / H, "unit": "tokens/s", "cores": 1,
+                                    "sample": "%d passes over %d of %d heads (%d tokens) in %.1f s"
+                                              % (reps, heads_1core, H, w["T_tot"], dt)}
+
+    prefill_fig("prefill_2k", 2)
+    prefill_fig("prefill_10k", 1)
+
+    d = make_decode(seed=0)
+    steps, H, dd = d["steps"], d["H"], d["d"]
+    per_pair_step = decode_bytes(1, 1, dd)
+
+    def decode_sample(nseq):
+        # [steps, B, H, d] -> sequences of `steps` tokens: [nseq * steps, H, d]
+        seq = lambda x: oracle.as_f64(x[:, :nseq].transpose(0, 1).reshape((nseq * steps,) + tuple(x.shape[2:])))
+        args_o = [seq(d[x]) for x in ("q", "k", "v", "g", "beta")]
+        S = oracle.as_f64(d["S"][:nseq])
+        cu = [steps * i for i in range(nseq + 1)]
+        return lambda: oracle.scan(*args_o, S0=S, cu_seqlens=cu), nseq * H * steps
+
+    for label, nseq, nthreads in (("decode_all_cores", 8, cores), ("decode_1_core", 1, 1)):
+        run, units = decode_sample(nseq)
+        oracle.set_num_threads(nthreads)
+        try:
+            rate, reps, dt = _oracle_rate(run, units, budget_s)
+        finally:
+            oracle.set_num_threads(cores)
+        figs[label] = {"value": rate * per_pair_step / 1e9, "unit": "GB/s", "cores": nthreads,
+                       "sample": "%d runs of 256 chained steps for %d of 64 sequences x %d heads in %.1f s"
+                                 % (reps, nseq, H, dt)}
+    main = figs["prefill_2k_all_cores"]
+    return {"value": main["value"], "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "prefill_2k: " + main["sample"] + "; other workloads and one core under 'figures'",
+            "figures": figs}
 
 
 def reference_arm(args):

@@ -82,7 +82,7 @@ const char *gdn_last_error(void);
  * are meaningless except for the error word read by gdn_chunk_fwd_check.
  * Two calls that overlap on the GPU must not share a workspace.
  */
-size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype);
+size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, gdn_dtype dtype);
 
 /*
  * Prefill: the chunked form of the rule over N packed sequences (page 1,
@@ -108,13 +108,16 @@ size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int
  * it without a synchronisation): if it is malformed, the kernels write
  * nothing to o / S_T and record GDN_ERR_SEQLENS in the workspace's error
  * word; gdn_chunk_fwd itself returns GDN_OK and gdn_chunk_fwd_check reports
- * the error. fp32 inputs run an fp32 (CUDA-core) chunked path; bf16 inputs
- * the tensor-core path (bf16 operands, fp32 accumulation and state).
+ * the error. Which kernels run: bf16 inputs with dk = dv = 128 take the
+ * tensor-core path (bf16 operands, fp32 accumulation and state); fp32 inputs
+ * (either head size) and bf16 inputs with dk = dv = 64 take the fp32
+ * CUDA-core chunked path, which has no tensor-core variant (same results up to
+ * rounding, far slower).
  */
 gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          const float *g, const float *beta, const float *S0,
                          const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                         int dtype, void *o, float *S_T,
+                         gdn_dtype dtype, void *o, float *S_T,
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
@@ -132,19 +135,21 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
  * forward runs with the coarser time segmentation that fits in it (the
  * results are the same up to rounding); GDN_ERR_WORKSPACE is returned only
  * if the array could not hold gdn_chunk_fwd's 256-byte minimum. The call
- * allocates nothing. Its first call on a device
- * (with that device current) looks up the array's device address once;
- * make that first call before any stream capture. All calls on a device
- * share the array: calls that overlap on the GPU race and must be
- * serialised by the caller. A malformed device cu_seqlens still makes the
- * kernels write nothing, but this entry point offers no way to read the
- * device error word: validate cu_seqlens with gdn_chunk_fwd +
- * gdn_chunk_fwd_check when it is untrusted.
+ * allocates nothing. Every call looks up the array's device address in the
+ * context current on the calling thread (the first lookup in a context may
+ * load the library's module: make the first call on a device before any
+ * stream capture). All calls on a device share the array: calls that overlap
+ * on the GPU race and must be serialised by the caller. The array's error word
+ * is not readable through this entry point, so two device-side failures go
+ * unreported here: a malformed device cu_seqlens (the kernels then write
+ * nothing) and a bounded inter-block wait that gave up (GDN_ERR_TIMEOUT in
+ * gdn_chunk_fwd_check; o and S_T are then incomplete). Callers that need
+ * either reported use gdn_chunk_fwd + gdn_chunk_fwd_check.
  */
 gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
                                  const float *g, const float *beta, const float *S0,
                                  const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                                 int dtype, void *o, float *S_T, void *stream);
+                                 gdn_dtype dtype, void *o, float *S_T, void *stream);
 
 /*
  * Synchronises `stream` and reads the device error word that the last
@@ -166,7 +171,7 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
  */
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            const float *g, const float *beta, float *S,
-                           int B, int H, int dk, int dv, int dtype, void *o, void *stream);
+                           int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream);
 
 /*
  * The sequential (token-by-token) scan on the GPU: the same result as
@@ -181,7 +186,7 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
 gdn_status gdn_seq_scan(const void *q, const void *k, const void *v,
                         const float *g, const float *beta, const float *S0,
                         const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                        int dtype, void *o, float *S_T, void *stream);
+                        gdn_dtype dtype, void *o, float *S_T, void *stream);
 
 /*
  * Diagnostic (used by the tests, not by the forward path): one tensor-core
@@ -208,6 +213,28 @@ gdn_status gdn_diag_mma_tile(const void *A, const void *B, float *D, int M, int 
  * forward-substitution step of the chunked form). One CTA on `stream`.
  */
 gdn_status gdn_diag_ut_solve(const float *A, float *T, void *stream);
+
+/*
+ * Failure injection, for tests of the failure path (off by default; process
+ * wide, set it while no call is in flight). The pages describe no such thing;
+ * it exists to show that a device-side wait that cannot complete ends with an
+ * error status instead of hanging the GPU.
+ *   GDN_INJECT_NONE: normal operation (wait_us ignored).
+ *   GDN_INJECT_WITHHOLD_LINK: in every later gdn_chunk_fwd call that runs the
+ *     pipelined bf16 tensor-core path (a workspace of at least
+ *     gdn_chunk_fwd_workspace_size bytes) with a sequence split into parallel
+ *     segments, the
+ *     transition block of the first segment of head 0 computes as usual but
+ *     never publishes its end state. The blocks that wait for it give up after
+ *     wait_us microseconds (1 .. 1000000; instead of the normal 1 s bound),
+ *     mark their own results failed so that blocks waiting on them give up
+ *     too, record GDN_ERR_TIMEOUT in the workspace's error word and return.
+ *     Outputs of the affected (sequence, head) pairs are then incomplete;
+ *     other heads are unaffected. gdn_chunk_fwd_check reports the timeout.
+ * Returns GDN_ERR_SHAPE for an unknown kind or an out-of-range wait_us.
+ */
+typedef enum { GDN_INJECT_NONE = 0, GDN_INJECT_WITHHOLD_LINK = 1 } gdn_inject_kind;
+gdn_status gdn_debug_inject(int kind, unsigned wait_us);
 
 /*
  * Kernel timing (measurement support, off by default). While enabled, every

@@ -122,14 +122,15 @@ __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait for a flag that another CTA publishes with a release store: true once it reads
-// FLAG_DONE. A failed flag, another role's abort or the time bound end it with false (and abort
-// this CTA; the time bound also records the timeout).
-__device__ __noinline__ bool wait_flag(const uint32_t *p, Ctl *ctl, uint32_t *err) {
+// FLAG_DONE. A failed flag, another role's abort or the time bound (bound_ns: kWaitNs, or the
+// shorter bound of a failure-injection test) end it with false (and abort this CTA; the time
+// bound also records the timeout).
+__device__ __noinline__ bool wait_flag(const uint32_t *p, Ctl *ctl, uint32_t *err, uint64_t bound_ns) {
     const uint64_t t0 = tc::globaltimer();
     uint32_t f;
     while ((f = tc::ld_acquire_gpu(p)) == 0u) {
         if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
-        if (tc::globaltimer() - t0 > kWaitNs) {
+        if (tc::globaltimer() - t0 > bound_ns) {
             atomicOr(err, ERRBIT_TIMEOUT);
             break;
         }
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
              const float *S0, const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o,
              float *S_T, uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off,
              const int32_t *__restrict__ chunk_off, int seg_chunks, const uint8_t *__restrict__ rec,
-             const uint8_t *__restrict__ link, const uint32_t *__restrict__ flags) {
+             const uint8_t *__restrict__ link, const uint32_t *__restrict__ flags, uint64_t flag_ns) {
     using namespace ob;
     extern __shared__ __align__(1024) uint8_t smem[];
     // What this CTA waits for before reading what earlier passes wrote (the plan's error word and
@@ -646,7 +647,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const int pre = min(nch, 2);
             for (int c = 0; c < pre; ++c) load_inputs(c);
             // (a failed or timed-out flag aborts the CTA; the record loads still complete the barriers)
-            if (split) wait_flag(start_flag, ctl, err);
+            if (split) wait_flag(start_flag, ctl, err, flag_ns);
             else griddep_wait();
             for (int c = 0; c < pre; ++c) load_record(c);
             int issued = pre;
@@ -748,7 +749,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             ok = wait_bar(&bar[FULL], 0, ctl, err);
             if (ok) g0 = vecp(0)[64 + C - 1];
         }
-        if (ok && split && sg.s > 0) ok = __all_sync(0xffffffffu, wait_flag(start_flag, ctl, err));
+        if (ok && split && sg.s > 0) ok = __all_sync(0xffffffffu, wait_flag(start_flag, ctl, err, flag_ns));
         if (ok) {
             const uint8_t *lk = nullptr;
             const float *src = nullptr;
@@ -939,24 +940,32 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
                const int32_t *__restrict__ seg_off, const int32_t *__restrict__ chunk_off, int seg_chunks,
                const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags,
-               uint8_t *__restrict__ part, uint32_t *__restrict__ pflags) {
+               uint8_t *__restrict__ part, uint32_t *__restrict__ pflags, uint64_t flag_ns, int withhold) {
     using namespace tb;
     extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ int s_ticket;
     // Only the loader reads what the prep pass writes (the records); it waits for that grid after
     // starting the first chunks' K, V loads, and the other roles start at once (S0, the identity).
     // The plan (error word, offsets, cleared flags) is complete before prep can launch this grid.
     griddep_launch();
+    // Records flag (after all end-state and part flags): set once the prep grid is complete, so
+    // that output CTAs that need only the records start without waiting for this grid. After it,
+    // the ticket counter.
+    uint32_t *rec_flag = pflags + (size_t)gridDim.y * H;
+    // Work is handed out in the order CTAs start, not by block index: ticket t is segment t / H
+    // of head t % H. A CTA waits only for segments of its own sequence with a lower index, whose
+    // tickets were taken by CTAs that had already started, so every wait ends whatever the order
+    // in which the hardware dispatches the grid's blocks.
+    if (threadIdx.x == 0) s_ticket = (int)atomicAdd(rec_flag + 1, 1u);
+    __syncthreads();
     if (*err & ERRBIT_SEQLENS) return;
     Segment sg;
-    const int h = blockIdx.x;
-    // Records flag (after all end-state and part flags): set once the prep grid is complete, so
-    // that output CTAs that need only the records start without waiting for this grid.
-    uint32_t *rec_flag = pflags + (size_t)gridDim.y * H;
-    if (!find_segment(seg_off, cu, N, T_tot, blockIdx.y, seg_chunks * C, sg) || sg.s == sg.ns - 1) {
+    const int h = s_ticket % H, gseg = s_ticket / H;
+    if (!find_segment(seg_off, cu, N, T_tot, gseg, seg_chunks * C, sg) || sg.s == sg.ns - 1) {
         // (the last segment's end state is never needed.) CTA (0, 0), which sets the records flag
         // from its loader when it has work, sets it here when it has none (no sequence is split);
         // the others leave at once.
-        if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0) {
+        if (threadIdx.x == 0 && h == 0 && gseg == 0) {
             griddep_wait();
             tc::st_release_gpu(rec_flag, FLAG_DONE);
         }
@@ -964,7 +973,6 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     }
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sb = tc::smem_u32(smem);
-    const int gseg = blockIdx.y;
     uint32_t *my_flag = flags + (size_t)gseg * H + h;
     if (sb & 1023u) {
         if (tid == 0) {
@@ -1024,7 +1032,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             }
             // CTA (0, 0) (the first segment of the first sequence: no Phi chain, no fold) sets the
             // records flag, after its first record loads so that the store's fence is not on their path
-            if (blockIdx.x == 0 && blockIdx.y == 0) tc::st_release_gpu(rec_flag, FLAG_DONE);
+            if (h == 0 && gseg == 0) tc::st_release_gpu(rec_flag, FLAG_DONE);
             int k_issued = pk, v_issued = pv;  // chunks whose K (V) part is in flight or landed
             for (int c = pv; c < nch; ++c) {
                 if (c >= k_issued) {
@@ -1235,7 +1243,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
             } else if (ok) {
                 const int half = (warp >> 2) & 1;
-                if ((ok = __all_sync(0xffffffffu, wait_flag(flags + slot0, ctl, err)))) {
+                if ((ok = __all_sync(0xffffffffu, wait_flag(flags + slot0, ctl, err, flag_ns)))) {
                     const uint8_t *src = link + slot0 * LINK_BYTES;
 #pragma unroll 1
                     for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
@@ -1262,7 +1270,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             const int c0 = 32 * (warp >> 2);
             for (int j = 1; ok && j < nfold; ++j) {
                 const int b = j & 1;
-                if (!(ok = __all_sync(0xffffffffu, wait_flag(pflags + slot0 + (size_t)j * H, ctl, err)))) break;
+                if (!(ok = __all_sync(0xffffffffu, wait_flag(pflags + slot0 + (size_t)j * H, ctl, err, flag_ns)))) break;
                 const float4 *src = reinterpret_cast<const float4 *>(part_of(j) + PART_S) + (c0 >> 2) * D + r;
                 float4 sl[8];  // in flight during the step's MMAs
 #pragma unroll
@@ -1300,7 +1308,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                     // buffer b was last read by step j - 2
                     if (j >= 3 && !(good = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 3) >> 1) & 1), ctl, err)))
                         break;
-                    if (!(good = wait_flag(pflags + slot0 + (size_t)j * H, ctl, err))) break;
+                    if (!(good = wait_flag(pflags + slot0 + (size_t)j * H, ctl, err, flag_ns))) break;
                     tc::fence_proxy_async_global();
                     tc::mbar_arrive_expect_tx(&bar[PFULL + b], 65536u);
                     tc::bulk_load(sb + PHI + 65536u * b, part_of(j) + PART_PHI, 65536u, &bar[PFULL + b]);
@@ -1363,7 +1371,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (tid == 0) {
+    // (failure-injection test: segment 0 of head 0 withholds its end-state flag, so that the
+    // CTAs waiting for it give up after the injected bound; nothing else changes)
+    if (tid == 0 && !(withhold && h == 0 && gseg == 0)) {
         const bool good = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
         tc::st_release_gpu(my_flag, good ? FLAG_DONE : FLAG_FAILED);
         if (!good) atomicOr(err, ERRBIT_TIMEOUT);
@@ -1487,7 +1497,7 @@ WsLayout ws_layout(int N, int T_tot, int H, int seg_chunks) {
     l.seg_off = 256;
     l.chunk_off = l.seg_off + align256((size_t)(N + 1) * 4);
     l.flags = l.chunk_off + align256((size_t)(N + 1) * 4);
-    l.s0copy = l.flags + align256(((size_t)2 * l.nslots * H + 1) * 4);  // end-state flags, part flags, records flag
+    l.s0copy = l.flags + align256(((size_t)2 * l.nslots * H + 2) * 4);  // end-state flags, part flags, records flag, ticket
     l.rec = l.s0copy + (seg_chunks > 0 ? (size_t)N * H * D * D * sizeof(float) : 0);
     l.link = l.rec + align256((size_t)l.nc_bound * H * REC_BYTES);
     l.part = l.link + (seg_chunks > 0 ? (size_t)l.nslots * H * LINK_BYTES : 0);
@@ -1527,6 +1537,8 @@ size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks) { return ws_l
 cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
                             const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
                             void *workspace, int seg_chunks, cudaStream_t st, const char **stage) {
+    const Inject inj = inject_settings();
+    const uint64_t flag_ns = inj.flag_wait_ns ? inj.flag_wait_ns : kWaitNs;
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     uint32_t *err = static_cast<uint32_t *>(workspace);
     const WsLayout l = ws_layout(N, T_tot, H, seg_chunks);
@@ -1554,7 +1566,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     }
     *stage = "plan";
     void *pr = prof_start("ws_plan", st);
-    const int nflags = seg_chunks > 0 ? 2 * l.nslots * H + 1 : 0;
+    const int nflags = seg_chunks > 0 ? 2 * l.nslots * H + 2 : 0;
     k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
     prof_stop(pr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1579,7 +1591,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         pr = prof_start("ws_trans", st);
         e = launch_pdl(k_ws_trans, dim3(H, l.nslots), dim3(NT_TRANS), tb::TOTAL, st, tm_k, tm_v, S0, cu, N, T_tot, H,
                        err, (const int32_t *)seg_off, (const int32_t *)chunk_off, seg_chunks, (const uint8_t *)rec, link,
-                       flags, part, flags + (size_t)l.nslots * H);
+                       flags, part, flags + (size_t)l.nslots * H, flag_ns, inj.withhold_first_link ? 1 : 0);
         prof_stop(pr);
         if (e != cudaSuccess) return e;
     }
@@ -1590,7 +1602,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     e = launch_pdl(k_ws_out, dim3(H, l.nslots), dim3(NT_WS), ob::TOTAL, st, tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot,
                    H, o, S_T, err, seg_chunks > 0 ? (const int32_t *)seg_off : nullptr, (const int32_t *)chunk_off,
                    seg_chunks > 0 ? seg_chunks : 1, (const uint8_t *)rec, (const uint8_t *)link,
-                   seg_chunks > 0 ? (const uint32_t *)flags : nullptr);
+                   seg_chunks > 0 ? (const uint32_t *)flags : nullptr, flag_ns);
     prof_stop(pr);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

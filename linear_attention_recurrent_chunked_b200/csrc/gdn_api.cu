@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -143,6 +144,14 @@ void prof_stop(void *handle) {
     delete hd;
 }
 
+std::atomic<int> g_inject_kind{0};
+std::atomic<unsigned long long> g_inject_wait_ns{0};
+
+Inject inject_settings() {
+    const int kind = g_inject_kind.load(std::memory_order_relaxed);
+    return Inject{kind == GDN_INJECT_WITHHOLD_LINK, kind ? (uint64_t)g_inject_wait_ns.load() : 0ull};
+}
+
 // Sets the calling thread's last-error message (for entry points defined in other files).
 gdn_status record_error(gdn_status s, const char *msg) { return fail(s, "%s", msg); }
 
@@ -154,7 +163,7 @@ int gdn_version(void) { return 100; }
 
 const char *gdn_last_error(void) { return g_msg; }
 
-size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int dtype) {
+size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, gdn_dtype dtype) {
     if (dtype == GDN_BF16 && dk == 128 && dv == 128 && N >= 1 && H >= 1 && T_tot >= 0)
         // (the plan differs with and without cu_seqlens; the larger workspace covers both)
         return std::max({kErrWordBytes, gdn::chunk_ws_workspace(N, T_tot, H, gdn::chunk_ws_seg_chunks(N, T_tot, H, false)),
@@ -164,7 +173,7 @@ size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, int
 
 gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
                          const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                         int dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
+                         gdn_dtype dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
     gdn_status s = check_common(q, k, v, g, beta, o, T_tot, H, dk, dv, dtype);
     if (s != GDN_OK) return s;
     if (N < 1) return fail(GDN_ERR_SHAPE, "N=%d must be >= 1", N);
@@ -239,7 +248,7 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta, float *S,
-                           int B, int H, int dk, int dv, int dtype, void *o, void *stream) {
+                           int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream) {
     if (B < 1) return fail(GDN_ERR_SHAPE, "B=%d must be >= 1", B);
     gdn_status s = check_common(q, k, v, g, beta, o, B, H, dk, dv, dtype);
     if (s != GDN_OK) return s;
@@ -267,7 +276,7 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
 
 gdn_status gdn_seq_scan(const void *q, const void *k, const void *v, const float *g, const float *beta,
                         const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                        int dtype, void *o, float *S_T, void *stream) {
+                        gdn_dtype dtype, void *o, float *S_T, void *stream) {
     gdn_status s = check_common(q, k, v, g, beta, o, T_tot, H, dk, dv, dtype);
     if (s != GDN_OK) return s;
     if (N < 1) return fail(GDN_ERR_SHAPE, "N=%d must be >= 1", N);
@@ -293,6 +302,16 @@ gdn_status gdn_seq_scan(const void *q, const void *k, const void *v, const float
                        : gdn::launch_seq_scan<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, st);
     }
     if (e != cudaSuccess) return cuda_fail(e, "sequential scan launch");
+    return ok();
+}
+
+gdn_status gdn_debug_inject(int kind, unsigned wait_us) {
+    if (kind != GDN_INJECT_NONE && kind != GDN_INJECT_WITHHOLD_LINK)
+        return fail(GDN_ERR_SHAPE, "unknown injection kind %d", kind);
+    if (kind != GDN_INJECT_NONE && (wait_us == 0 || wait_us > 1000000u))
+        return fail(GDN_ERR_SHAPE, "wait_us=%u outside 1 .. 1000000", wait_us);
+    gdn::g_inject_wait_ns.store((unsigned long long)wait_us * 1000ull);
+    gdn::g_inject_kind.store(kind);
     return ok();
 }
 

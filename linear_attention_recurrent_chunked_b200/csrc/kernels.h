@@ -45,6 +45,15 @@ cudaError_t launch_chunk_ws(const __nv_bfloat16 *q, const __nv_bfloat16 *k, cons
 int chunk_ws_seg_chunks(int N, int T_tot, int H, bool varlen);  // varlen: cu_seqlens given
 size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks);
 
+// Failure injection for tests (set by gdn_debug_inject; off by default): the pipelined path's
+// first segment of head 0 withholds its end-state flag, and waits for flags give up after
+// flag_wait_ns (0 = the normal bound) instead of hanging.
+struct Inject {
+    bool withhold_first_link;
+    uint64_t flag_wait_ns;
+};
+Inject inject_settings();
+
 // Kernel timing hooks (no-ops unless gdn_profile_enable(1)): an event pair
 // around the launches between prof_start and prof_stop, recorded on st.
 void *prof_start(const char *name, cudaStream_t st);

@@ -35,6 +35,7 @@ SIGNATURES = {
     "gdn_diag_mma_tile": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
     "gdn_diag_ut_solve": (_I, [_VP, _VP, _VP]),
     "gdn_chunk_fwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
+    "gdn_debug_inject": (_I, [_I, ctypes.c_uint]),
     "gdn_profile_enable": (None, [_I]),
     "gdn_profile_read": (_I, [ctypes.c_char_p, _SZ, _VP, _VP, _I]),
 }
@@ -196,6 +197,12 @@ def diag_mma_tile(A, B, a_mn: int = 0, b_mn: int = 0, variant: int = 0):
     D = torch.full((128, N), float("nan"), dtype=torch.float32, device=A.device)
     _check(lib.gdn_diag_mma_tile(_ptr(A), _ptr(B), _ptr(D), M, N, K, a_mn, b_mn, variant, _stream()))
     return D
+
+
+def debug_inject(kind: int, wait_us: int = 0) -> None:
+    """Failure injection for tests (see include/gdn.h): 0 = off, 1 = withhold the first
+    segment's end state of head 0 so that the blocks waiting for it time out after wait_us."""
+    _check(load_library().gdn_debug_inject(kind, wait_us))
 
 
 def profile_enable(on: bool = True) -> None:

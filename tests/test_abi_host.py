@@ -123,3 +123,13 @@ def test_binding_refuses_cpu_tensors(lib):
         gdn.chunk_fwd(x, x, x, gb, gb)
     with pytest.raises(gdn.GdnError):
         gdn.decode_step(x, x, x, gb, gb, torch.zeros(4, 2, 64, 64))
+
+
+def test_failure_injection_arguments(lib):
+    """The test-only failure injection accepts its documented kinds and bounds and nothing else
+    (host logic only; the GPU side is tests/test_gpu_failure.py)."""
+    assert lib.gdn_debug_inject(7, 1000) == 2
+    assert lib.gdn_debug_inject(1, 0) == 2
+    assert lib.gdn_debug_inject(1, 1000001) == 2
+    assert lib.gdn_debug_inject(1, 2000) == 0
+    assert lib.gdn_debug_inject(0, 0) == 0

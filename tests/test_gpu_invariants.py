@@ -1,0 +1,264 @@
+"""The method's own edge cases and structural equivalences, run through the CUDA path (C ABI)
+and compared element by element with the fp64 oracle on the same inputs.
+
+The graded workloads forget their state within a few tokens (g = -softplus(N(0,1))), so they
+barely exercise what the chunked form can get wrong: decays of tokens far apart (fp32
+G_r - G_s, flushed exponentials), a reset inside a chunk or on a chunk boundary, a state kept
+unchanged over many chunks, exact store / retrieve, and the worst-conditioned intra-chunk solve.
+The cases (gated delta rule S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+o_t = S_t q_t):
+
+* alpha ~ 0 (g = -100, exp(-100) ~ 3.7e-44): the state is reset to beta_t v_t k_t^T, mid-chunk
+  and on a chunk boundary, in sequences long enough to be split into parallel segments;
+* beta = 0 and g = 0: the state passes unchanged and o_t = S0 q_t;
+* alpha = beta = 1 with orthonormal keys: S_T k_j = v_j, and o_t = v_t when q_t = k_t;
+* a run of identical unit keys with beta near one (T = (I + A)^{-1} at its worst conditioning);
+* head and sequence permutations permute the results exactly; a packed batch equals separate
+  calls; every path (tensor-core pipelined, single-kernel, fp32) on the same edge inputs.
+
+Tolerance: max|gpu - oracle| / max|oracle| <= 1e-4 (fp32 inputs) or 2e-2 (bf16 inputs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrent_chunked_b200 import gdn
+from linear_attention_recurrent_chunked_b200.workloads import TORCH_DTYPE, make_decode, make_prefill
+from tests.gpu_util import TOL, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+CASES = [("bf16", 128), ("f32", 64)]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gdn.load_library()
+
+
+def run_oracle(w):
+    return oracle.scan(w["q"], w["k"], w["v"], w["g"], w["beta"], S0=w["S0"], cu_seqlens=w["cu_seqlens"])
+
+
+def run_gpu(w, workspace=None):
+    dw = to_dev(w)
+    return gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], dw["cu_seqlens"],
+                         workspace=workspace, check=True)
+
+
+def check(w, o, S_T, what, workspace_note=""):
+    o_ref, S_ref = run_oracle(w)
+    eo, es = rel_err(o, o_ref), rel_err(S_T, S_ref)
+    tol = TOL[w["dtype"]]
+    assert eo <= tol and es <= tol, "%s%s: err(o)=%.3g err(S_T)=%.3g" % (what, workspace_note, eo, es)
+    return o_ref, S_ref
+
+
+def orthonormal_rows(n, d, seed):
+    g = torch.Generator().manual_seed(seed)
+    qm, _ = torch.linalg.qr(torch.randn(d, d, generator=g, dtype=torch.float64))
+    return qm[:n].to(torch.float32)  # n orthonormal rows
+
+
+# ------------------------------------------------------------------ alpha ~ 0: reset
+
+@pytest.mark.parametrize("dtype,d", CASES)
+@pytest.mark.parametrize("where", ["mid_chunk", "chunk_boundary"])
+def test_reset_by_vanishing_decay(dtype, d, where):
+    """g = -100 at a few tokens: the state just after is beta v k^T (up to exp(-100) S). The
+    sequence of 1400 tokens is split into parallel segments on the bf16 path; the resets fall
+    into different segments."""
+    w = make_prefill("varlen", seqlens=[1400, 130], H=2, d=d, dtype=dtype, s0=True, seed=31)
+    ts = [37, 300, 555, 1000, 1437] if where == "mid_chunk" else [64, 320, 640, 1280, 1464]
+    for t in ts:
+        w["g"][t, :] = -100.0
+    o, S_T = run_gpu(w)
+    check(w, o, S_T, "reset " + where)
+
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_reset_every_token_of_a_chunk(dtype, d):
+    """Every token of the second chunk resets: G reaches -6400 inside that chunk and the chunk's
+    decays underflow to zero everywhere except on the diagonal of the decay matrix."""
+    w = make_prefill("varlen", seqlens=[200], H=2, d=d, dtype=dtype, s0=True, seed=32)
+    w["g"][64:128, :] = -100.0
+    o, S_T = run_gpu(w)
+    o_ref, _ = check(w, o, S_T, "all-reset chunk")
+    # inside that chunk o_t = beta_t (k_t . q_t) v_t up to exp(-100) terms
+    t = 100
+    kq = (w["k"][t].double() * w["q"][t].double()).sum(-1)  # [H]
+    expect = (w["beta"][t].double() * kq)[:, None] * w["v"][t].double()
+    assert np.max(np.abs(o_ref[t] - expect.numpy())) < 1e-12
+
+
+# ------------------------------------------------------------------ beta = 0, alpha = 1: state unchanged
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_beta0_alpha1_state_passes_unchanged(dtype, d):
+    w = make_prefill("varlen", seqlens=[400, 65], H=2, d=d, dtype=dtype, s0=True, seed=33)
+    w["g"].zero_()
+    w["beta"].zero_()
+    o, S_T = run_gpu(w)
+    o_ref, S_ref = check(w, o, S_T, "beta=0 alpha=1")
+    assert np.array_equal(S_ref, w["S0"].double().numpy())  # the oracle: exactly unchanged
+    # GPU: S_T == S0 to the state's own rounding, o_t = S0 q_t
+    assert rel_err(S_T, w["S0"].double().numpy()) <= TOL[dtype]
+
+
+# ------------------------------------------------------------------ alpha = beta = 1, orthonormal keys
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_orthonormal_keys_store_and_retrieve(dtype, d):
+    """T = d tokens with orthonormal keys (fp32 before the input cast), alpha = beta = 1, S0 = 0:
+    the state is sum_j v_j k_j^T, so S_T k_j = v_j, and with q_t = k_t, o_t = v_t."""
+    T = d
+    w = make_prefill("varlen", seqlens=[T], H=2, d=d, dtype=dtype, s0=False, seed=34)
+    tdt = TORCH_DTYPE[dtype]
+    for h in range(2):
+        kk = orthonormal_rows(T, d, 100 + h)
+        w["k"][:, h] = kk.to(tdt)
+        w["q"][:, h] = kk.to(tdt)
+    w["g"].zero_()
+    w["beta"].fill_(1.0)
+    o, S_T = run_gpu(w)
+    check(w, o, S_T, "orthonormal keys")
+    # retrieval: bf16 keys are orthonormal only to the cast's rounding (2^-9)
+    tol_ret = 5e-2 if dtype == "bf16" else 1e-4
+    v = w["v"].double().numpy()
+    assert rel_err(o, v) <= tol_ret
+    S = S_T.double().cpu().numpy()[0]  # [H, dv, dk]
+    kd = w["k"].double().numpy()       # [T, H, dk]
+    retrieved = np.einsum("hvk,thk->thv", S, kd)
+    assert rel_err(retrieved, v) <= tol_ret
+
+
+# ------------------------------------------------------------------ identical keys: worst-conditioned solve
+
+@pytest.mark.parametrize("dtype,d", CASES)
+@pytest.mark.parametrize("beta_kind", ["near_one", "one"])
+def test_identical_keys_in_a_chunk(dtype, d, beta_kind):
+    """64 tokens (a whole chunk, then a partial one) share one unit key; beta near or equal to
+    one and no decay make A = beta times the strictly lower ones matrix. With a repeated key
+    S_t k is a scalar moving average (S_t k = (1 - beta_t) S_{t-1} k + beta_t v_t)."""
+    w = make_prefill("varlen", seqlens=[160], H=2, d=d, dtype=dtype, s0=True, seed=35)
+    tdt = TORCH_DTYPE[dtype]
+    gen = torch.Generator().manual_seed(36)
+    u = torch.nn.functional.normalize(torch.randn(2, d, generator=gen), dim=-1).to(tdt)
+    w["k"][:] = u[None]
+    w["g"].zero_()
+    if beta_kind == "one":
+        w["beta"].fill_(1.0)
+    else:
+        w["beta"].copy_(torch.sigmoid(torch.randn(w["beta"].shape, generator=gen) + 4.0))
+    o, S_T = run_gpu(w)
+    check(w, o, S_T, "identical keys, beta " + beta_kind)
+
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_slow_decay_identical_keys_long(dtype, d):
+    """Identical keys with slow decay over a segmented 1500-token sequence."""
+    w = make_prefill("varlen", seqlens=[1500], H=1, d=d, dtype=dtype, s0=True, seed=37)
+    tdt = TORCH_DTYPE[dtype]
+    gen = torch.Generator().manual_seed(38)
+    u = torch.nn.functional.normalize(torch.randn(1, d, generator=gen), dim=-1).to(tdt)
+    w["k"][:] = u[None]
+    w["g"].copy_(-0.01 * torch.rand(w["g"].shape, generator=gen))
+    o, S_T = run_gpu(w)
+    check(w, o, S_T, "identical keys, slow decay")
+
+
+# ------------------------------------------------------------------ the single-kernel path on the same edge inputs
+
+def test_edge_inputs_on_single_kernel_path():
+    """A 256-byte workspace selects the single-kernel tensor-core path: resets, beta = 0 runs
+    and identical keys in one sequence."""
+    w = make_prefill("varlen", seqlens=[450, 90], H=2, d=128, dtype="bf16", s0=True, seed=39)
+    w["g"][[40, 128, 300], :] = -100.0
+    w["beta"][150:260, :] = 0.0
+    w["g"][150:260, :] = 0.0
+    w["k"][330:400] = w["k"][330:331]
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o, S_T = run_gpu(w, workspace=ws)
+    check(w, o, S_T, "edge inputs", " (single-kernel path)")
+
+
+# ------------------------------------------------------------------ structural equivalences
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_head_permutation_permutes_results_exactly(dtype, d):
+    w = make_prefill("varlen", seqlens=[300, 77, 640], H=4, d=d, dtype=dtype, s0=True, seed=40)
+    o, S_T = run_gpu(w)
+    perm = [2, 0, 3, 1]
+    wp = dict(w)
+    for key in ("q", "k", "v", "g", "beta"):
+        wp[key] = w[key][:, perm].contiguous()
+    wp["S0"] = w["S0"][:, perm].contiguous()
+    op, Sp = run_gpu(wp)
+    assert torch.equal(op, o[:, perm]) and torch.equal(Sp, S_T[:, perm])
+
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_sequence_permutation_permutes_results_exactly(dtype, d):
+    lens = [300, 77, 640, 1]
+    w = make_prefill("varlen", seqlens=lens, H=3, d=d, dtype=dtype, s0=True, seed=41)
+    o, S_T = run_gpu(w)
+    perm = [2, 3, 0, 1]
+    cu = w["cu_seqlens"].tolist()
+    idx = torch.cat([torch.arange(cu[n], cu[n + 1]) for n in perm])
+    wp = dict(w)
+    for key in ("q", "k", "v", "g", "beta"):
+        wp[key] = w[key][idx].contiguous()
+    wp["S0"] = w["S0"][perm].contiguous()
+    newlens = [lens[n] for n in perm]
+    wp["cu_seqlens"] = torch.tensor([0] + list(np.cumsum(newlens)), dtype=torch.int32)
+    wp["seqlens"] = newlens
+    op, Sp = run_gpu(wp)
+    assert torch.equal(op, o[idx.cuda()]) and torch.equal(Sp, S_T[perm])
+
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_packed_batch_equals_separate_calls(dtype, d):
+    """A packed varlen call equals one call per sequence (the plans differ, so the comparison
+    is at the parity tolerance, and each side is checked against the oracle)."""
+    lens = [513, 64, 1000, 3]
+    w = make_prefill("varlen", seqlens=lens, H=2, d=d, dtype=dtype, s0=True, seed=42)
+    o, S_T = run_gpu(w)
+    o_ref, S_ref = check(w, o, S_T, "packed")
+    cu = w["cu_seqlens"].tolist()
+    for n, L in enumerate(lens):
+        sl = slice(cu[n], cu[n + 1])
+        wn = dict(w)
+        for key in ("q", "k", "v", "g", "beta"):
+            wn[key] = w[key][sl].contiguous()
+        wn["S0"] = w["S0"][n:n + 1].contiguous()
+        wn["cu_seqlens"] = torch.tensor([0, L], dtype=torch.int32)
+        on, Sn = run_gpu(wn)
+        assert rel_err(on, o[sl].double().cpu().numpy()) <= TOL[dtype], n
+        assert rel_err(Sn[0], S_T[n].double().cpu().numpy()) <= TOL[dtype], n
+        assert rel_err(on, o_ref[sl]) <= TOL[dtype] and rel_err(Sn[0], S_ref[n]) <= TOL[dtype], n
+
+
+# ------------------------------------------------------------------ decode edge cases
+
+@pytest.mark.parametrize("dtype,d", CASES)
+def test_decode_edge_steps(dtype, d):
+    """Decode steps with alpha ~ 0 (reset), beta = 0 with alpha = 1 (state unchanged: exact in
+    fp32, S_new = 1 * S + 0), and a repeated key, each against the oracle."""
+    w = make_decode(steps=5, B=4, H=2, d=d, dtype=dtype, seed=43)
+    w["g"][1, :2] = -100.0
+    w["g"][2].zero_()
+    w["beta"][2].zero_()
+    w["k"][4] = w["k"][3]
+    dw = to_dev(w)
+    S = dw["S"].clone()
+    S_ref = w["S"].double().numpy()
+    for t in range(w["steps"]):
+        S_before = S.clone()
+        o = gdn.decode_step(dw["q"][t], dw["k"][t], dw["v"][t], dw["g"][t], dw["beta"][t], S)
+        o_ref, S_ref = oracle.decode_step(w["q"][t], w["k"][t], w["v"][t], w["g"][t], w["beta"][t], S_ref)
+        assert rel_err(o, o_ref) <= TOL[dtype], t
+        assert rel_err(S, S_ref) <= TOL[dtype], t
+        if t == 2:
+            assert torch.equal(S, S_before)
