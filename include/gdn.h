@@ -121,6 +121,33 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Prefill from the layer's raw inputs: gdn_chunk_fwd with the input
+ * preparation done inside the kernels instead of by the caller. The recurrent
+ * layer of a gated delta network (page 1, abstract, result (i)) normalises its
+ * queries and keys and derives its decay and write strength from gate logits;
+ * the pages name the layer but print none of these steps, so this is the
+ * plain reading of the layer's input contract:
+ *     q_t = q_raw_t / max(||q_raw_t||_2, 1e-12),   k_t likewise (per token, head)
+ *     g_t = -softplus(a_t)  (alpha_t = exp(g_t) = 1 / (1 + exp(a_t)))
+ *     beta_t = sigmoid(b_t) = 1 / (1 + exp(-b_t))
+ * and then the rule exactly as gdn_chunk_fwd. Arguments are gdn_chunk_fwd's
+ * with q_raw, k_raw [T_tot][H][dk] (dtype, any norm) in place of q, k and the
+ * fp32 gate logits a, b [T_tot][H] in place of g, beta. The normalisation and
+ * gates are folded into the passes that read q, k, g and beta anyway: there is
+ * no separate pass over the inputs. bf16 inputs with dk = dv = 128 run only
+ * on the pipelined tensor-core path, whose workspace holds a record per
+ * (chunk, head): gdn_chunk_fwd_workspace_size gives the size of the fastest
+ * plan, a smaller workspace that still holds the records runs without time
+ * segments, and one that does not gives GDN_ERR_WORKSPACE. fp32 inputs and
+ * d = 64 take the fp32 CUDA-core path as in gdn_chunk_fwd.
+ */
+gdn_status gdn_chunk_fwd_raw(const void *q_raw, const void *k_raw, const void *v,
+                             const float *a, const float *b, const float *S0,
+                             const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                             gdn_dtype dtype, void *o, float *S_T,
+                             void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * gdn_chunk_fwd without a caller-provided workspace, for callers that cannot
  * allocate device memory: code running under a memory manager that has
  * already reserved the GPU's memory, plugins whose host application owns
@@ -172,6 +199,16 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            const float *g, const float *beta, float *S,
                            int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream);
+
+/*
+ * Decode from raw inputs: gdn_decode_step with the input preparation of
+ * gdn_chunk_fwd_raw done in the same kernel (q, k normalised, alpha =
+ * exp(-softplus(a)), beta = sigmoid(b)). q_raw, k_raw [B][H][dk] dtype;
+ * a, b [B][H] fp32 gate logits; everything else as gdn_decode_step.
+ */
+gdn_status gdn_decode_step_raw(const void *q_raw, const void *k_raw, const void *v,
+                               const float *a, const float *b, float *S,
+                               int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream);
 
 /*
  * The sequential (token-by-token) scan on the GPU: the same result as

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kSimtThreads) k_chunk_simt(const T *__restrict
                                                              const float *__restrict__ beta, const float *S0,
                                                              const int32_t *__restrict__ cu, int N, int T_tot, int H,
                                                              T *__restrict__ o, float *S_T,
-                                                             const uint32_t *__restrict__ err) {
+                                                             const uint32_t *__restrict__ err, int raw) {
     using Sm = SimtSmem<D, C>;
     constexpr int DP = Sm::DP, CP = Sm::CP;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -74,11 +74,27 @@ __global__ void __launch_bounds__(kSimtThreads) k_chunk_simt(const T *__restrict
             sm.V[r * DP + j] = ok ? Elem<T>::load(v + off) : 0.f;
         }
         if (tid < C) {
+            // raw inputs: g and beta hold the gate logits a, b; g = -softplus(a), beta = sigmoid(b)
             const bool ok = tid < L;
-            sm.G[tid] = ok ? g[(size_t)(c0 + tid) * H + h] : 0.f;
-            sm.beta[tid] = ok ? beta[(size_t)(c0 + tid) * H + h] : 0.f;
+            const float gv = ok ? g[(size_t)(c0 + tid) * H + h] : 0.f;
+            const float bv = ok ? beta[(size_t)(c0 + tid) * H + h] : 0.f;
+            sm.G[tid] = (raw && ok) ? neg_softplus(gv) : gv;
+            sm.beta[tid] = (raw && ok) ? sigmoid_f(bv) : bv;
         }
         __syncthreads();
+        if (raw) {  // raw inputs: L2-normalise the rows of K and Q (one warp per row)
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int rr = warp; rr < 2 * L; rr += kSimtThreads / 32) {
+                float *row = (rr < L ? sm.K : sm.Q) + (rr < L ? rr : rr - L) * DP;
+                float ss = 0.f;
+                for (int j = lane; j < D; j += 32) ss = fmaf(row[j], row[j], ss);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                const float sc = inv_norm(ss);
+                for (int j = lane; j < D; j += 32) row[j] *= sc;
+            }
+            __syncthreads();
+        }
         // ---- G = cumsum(g), gamma, decay to chunk end
         if (tid == 0) {
             float acc = 0.f;
@@ -165,20 +181,21 @@ __global__ void __launch_bounds__(kSimtThreads) k_chunk_simt(const T *__restrict
 template <typename T, int D>
 cudaError_t launch_chunk_simt(const T *q, const T *k, const T *v, const float *g, const float *beta, const float *S0,
                               const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, const uint32_t *err,
-                              cudaStream_t st) {
+                              cudaStream_t st, bool raw) {
     constexpr int C = (D <= 64) ? 64 : 32;
     const size_t smem = sizeof(SimtSmem<D, C>);
     cudaError_t e = cudaFuncSetAttribute(k_chunk_simt<T, D, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(H, N);
-    k_chunk_simt<T, D, C><<<grid, kSimtThreads, smem, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err);
+    k_chunk_simt<T, D, C><<<grid, kSimtThreads, smem, st>>>(q, k, v, g, beta, S0, cu, N, T_tot, H, o, S_T, err,
+                                                            raw ? 1 : 0);
     return cudaGetLastError();
 }
 
 #define GDN_INST(T, D)                                                                                        \
     template cudaError_t launch_chunk_simt<T, D>(const T *, const T *, const T *, const float *, const float *, \
                                                  const float *, const int32_t *, int, int, int, T *, float *,  \
-                                                 const uint32_t *, cudaStream_t);
+                                                 const uint32_t *, cudaStream_t, bool);
 GDN_INST(float, 64)
 GDN_INST(float, 128)
 GDN_INST(__nv_bfloat16, 64)

@@ -162,6 +162,60 @@ __device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, 
     }
 }
 
+// Raw inputs: L2-normalise the 64 rows of a 128-byte-swizzled 64 x 128 bf16 tile in place with
+// 256 threads (t = 0..255): four threads per row, each summing the squares of two 16-byte chunks
+// in each column half (the swizzle only permutes a row's chunks), then scaling them.
+__device__ __forceinline__ void normalise_rows_sw128(uint8_t *tile, int t) {
+    const int r = t >> 2, qd = t & 3;
+    uint4 *p[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p[i] = reinterpret_cast<uint4 *>(tile + (i >> 1) * 8192 + r * 128 + (2 * qd + (i & 1)) * 16);
+    uint4 x[4];
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[i] = *p[i];
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&x[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+            ss = fmaf(a.x, a.x, fmaf(a.y, a.y, ss));
+        }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float sc = inv_norm(ss);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t *w = reinterpret_cast<uint32_t *>(&x[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[j]));
+            w[j] = tc::pack_bf16x2(a.x * sc, a.y * sc);
+        }
+        *p[i] = x[i];
+    }
+}
+
+// Raw inputs: 1 / ||k_r|| of the 64 rows of a swizzled K tile into rn[] (256 threads, as above).
+__device__ __forceinline__ void row_inv_norms_sw128(const uint8_t *tile, float *rn, int t) {
+    const int r = t >> 2, qd = t & 3;
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(tile + (i >> 1) * 8192 + r * 128 + (2 * qd + (i & 1)) * 16);
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(&x);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[j]));
+            ss = fmaf(a.x, a.x, fmaf(a.y, a.y, ss));
+        }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    if (qd == 0) rn[r] = inv_norm(ss);
+}
+
 // T1 = T2 diag(gamma) between two 64 x 64 bf16 tiles (rows r, runs along s; sy = 1024), n threads.
 __device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t, int n) {
     for (int idx = t; idx < 512; idx += n) {
@@ -320,7 +374,8 @@ constexpr uint32_t XS = AT + 64 * AP * 4;           // solve scratch, 32 x XP fp
 constexpr uint32_t REC = XS + 32 * ut::XP * 4;      // record staging (bulk-stored)
 constexpr uint32_t RAW = REC + REC_BYTES;           // raw g, beta of two items: 2 x 512 B
 constexpr uint32_t VS = RAW + 1024;                 // G, gamma, e, beta of the current item (4 x 64 fp32)
-constexpr uint32_t BAR = VS + 1024;                 // K full, mma, TMEM slot
+constexpr uint32_t RN = VS + 1024;                  // 1 / ||k_r|| (raw inputs; 1 otherwise), 64 fp32
+constexpr uint32_t BAR = RN + 256;                  // K full, mma, TMEM slot
 constexpr uint32_t TOTAL = BAR + 64;
 constexpr int CTAS_PER_SM = 4;
 }  // namespace pp
@@ -330,6 +385,7 @@ constexpr int CTAS_PER_SM = 4;
 // g, beta (cp.async) are fetched while the current one runs, and its K tile
 // (TMA) as soon as the current K K^T product has read the single K buffer.
 // Four CTAs share an SM, so that one's solve overlaps another's loads.
+template <bool raw>
 __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
     k_ws_prep(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ g, const float *__restrict__ beta,
               const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
@@ -364,6 +420,8 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         for (int i = 0; i < 3; ++i) tc::mbar_init(&bars[i], 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    float *rnv = reinterpret_cast<float *>(smem + pp::RN);
+    if (tid < C) rnv[tid] = 1.f;  // (raw inputs overwrite it per item)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -445,10 +503,21 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
             cp_async_wait_all();
         }
         __syncthreads();
-        // ---- scalars: G = cumsum(g) (log2 units), gamma, e, beta
+        // ---- scalars: G = cumsum(g) (log2 units), gamma, e, beta. Raw inputs: g = -softplus(a),
+        // beta = sigmoid(b) from the logits, zero past the chunk's valid length L
         const float *graw = reinterpret_cast<const float *>(smem + pp::RAW + b * 512u);
+        int L_item = C;
+        if (raw) {
+            int h_, cs_, gc_;
+            locate(w, h_, cs_, L_item, gc_);
+        }
         if (tid < 32) {
-            const float a = graw[2 * tid] * kLog2e, b2 = a + graw[2 * tid + 1] * kLog2e;
+            float x0 = graw[2 * tid], x1 = graw[2 * tid + 1];
+            if (raw) {
+                x0 = 2 * tid < L_item ? neg_softplus(x0) : 0.f;
+                x1 = 2 * tid + 1 < L_item ? neg_softplus(x1) : 0.f;
+            }
+            const float a = x0 * kLog2e, b2 = a + x1 * kLog2e;
             float sc = b2;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -462,7 +531,11 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         if (tid < C) {
             gam[tid] = ex2(Gl[tid]);
             dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
-            bet[tid] = graw[64 + tid];
+            bet[tid] = raw ? (tid < L_item ? sigmoid_f(graw[64 + tid]) : 0.f) : graw[64 + tid];
+        }
+        if (raw) {  // key norms from the landed K tile (read before the next item's K can be loaded)
+            tc::mbar_wait(&bars[0], (uint32_t)(it & 1));
+            row_inv_norms_sw128(smem + pp::K0, rnv, tid);
         }
         if (fixed && it == 0) {
             griddep_wait();
@@ -488,15 +561,17 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
                 const float y = __shfl_sync(0xffffffffu, x[16 + i], l16);
                 x[i] = hf ? y : x[i];
             }
-            const float Gr = Gl[r], br = bet[r];
+            // (raw inputs: X1 holds raw k_r . k_s, scaled here by 1 / (||k_r|| ||k_s||); otherwise by 1)
+            const float Gr = Gl[r], br = bet[r] * rnv[r];
 #pragma unroll
             for (int i = 0; i < 16; i += 4) {
                 const float4 g4 = *reinterpret_cast<const float4 *>(Gl + c0 + i);
+                const float4 n4 = *reinterpret_cast<const float4 *>(rnv + c0 + i);
                 float4 a;
-                a.x = (c0 + i < r) ? br * ex2(Gr - g4.x) * x[i] : 0.f;
-                a.y = (c0 + i + 1 < r) ? br * ex2(Gr - g4.y) * x[i + 1] : 0.f;
-                a.z = (c0 + i + 2 < r) ? br * ex2(Gr - g4.z) * x[i + 2] : 0.f;
-                a.w = (c0 + i + 3 < r) ? br * ex2(Gr - g4.w) * x[i + 3] : 0.f;
+                a.x = (c0 + i < r) ? br * ex2(Gr - g4.x) * (x[i] * n4.x) : 0.f;
+                a.y = (c0 + i + 1 < r) ? br * ex2(Gr - g4.y) * (x[i + 1] * n4.y) : 0.f;
+                a.z = (c0 + i + 2 < r) ? br * ex2(Gr - g4.z) * (x[i + 2] * n4.z) : 0.f;
+                a.w = (c0 + i + 3 < r) ? br * ex2(Gr - g4.w) * (x[i + 3] * n4.w) : 0.f;
                 *reinterpret_cast<float4 *>(AT + r * AP + c0 + i) = a;
             }
         }
@@ -517,7 +592,9 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
                                 t1.x * b1.x, t1.y * b1.y, t1.z * b1.z, t1.w * b1.w};
             st_run8(sb + pp::REC + REC_T2 + tc::tile_off(r, 8 * j, 128, 1024), x);
         }
-        reinterpret_cast<float *>(smem + pp::REC + REC_VEC)[tid] = vec[tid];
+        // record vectors G, gamma, e and, for raw inputs, 1 / ||k|| in the fourth slot (beta is already
+        // folded into T2 and is not read from the record)
+        reinterpret_cast<float *>(smem + pp::REC + REC_VEC)[tid] = (raw && tid >= 192) ? rnv[tid - 192] : vec[tid];
         tc::fence_smem_to_async();
         __syncthreads();
         if (tid == 0) {
@@ -576,7 +653,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
              const float *S0, const int32_t *__restrict__ cu, int N, int T_tot, int H, bf16 *__restrict__ o,
              float *S_T, uint32_t *__restrict__ err, const int32_t *__restrict__ seg_off,
              const int32_t *__restrict__ chunk_off, int seg_chunks, const uint8_t *__restrict__ rec,
-             const uint8_t *__restrict__ link, const uint32_t *__restrict__ flags, uint64_t flag_ns) {
+             const uint8_t *__restrict__ link, const uint32_t *__restrict__ flags, uint64_t flag_ns, int raw) {
     using namespace ob;
     extern __shared__ __align__(1024) uint8_t smem[];
     // What this CTA waits for before reading what earlier passes wrote (the plan's error word and
@@ -786,8 +863,14 @@ __global__ void __launch_bounds__(NT_WS, 1)
         bool ok = true;
         for (int c = 0; ok && c < nch; ++c) {
             const int b = c & 1;
-            // T1 = T2 diag(gamma) (the previous chunk's W^T, U^T have read T1: WUF was waited below)
+            // T1 = T2 diag(gamma) (the previous chunk's W^T, U^T have read T1: WUF was waited below).
+            // Raw inputs: first normalise K (1 / ||k|| from the record) and Q in place; no MMA reads
+            // this buffer's K or Q before T1R.
             if (!(ok = wait_bar(&bar[FULL + b], full_par(c), ctl, err))) break;
+            if (raw) {
+                scale_rows_sw128(smem + b * BUF + B_K, vecp(c) + 192, t256, 256);
+                normalise_rows_sw128(smem + b * BUF + B_Q, t256);
+            }
             make_t1(smem + T1, smem + b * BUF + B_T2, vecp(c) + 64, t256, 256);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
@@ -940,7 +1023,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
                const int32_t *__restrict__ seg_off, const int32_t *__restrict__ chunk_off, int seg_chunks,
                const uint8_t *__restrict__ rec, uint8_t *__restrict__ link, uint32_t *__restrict__ flags,
-               uint8_t *__restrict__ part, uint32_t *__restrict__ pflags, uint64_t flag_ns, int withhold) {
+               uint8_t *__restrict__ part, uint32_t *__restrict__ pflags, uint64_t flag_ns, int withhold, int raw) {
     using namespace tb;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ int s_ticket;
@@ -1180,6 +1263,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
                        wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err)))
                 break;
+            // raw inputs: normalise K in place (1 / ||k|| from the record) before W^T reads it (T1R)
+            if (raw) scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 192, t128, 128);
             make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
@@ -1536,7 +1621,7 @@ size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks) { return ws_l
 
 cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const float *g, const float *beta,
                             const float *S0, const int32_t *cu, int N, int T_tot, int H, bf16 *o, float *S_T,
-                            void *workspace, int seg_chunks, cudaStream_t st, const char **stage) {
+                            void *workspace, int seg_chunks, cudaStream_t st, const char **stage, bool raw) {
     const Inject inj = inject_settings();
     const uint64_t flag_ns = inj.flag_wait_ns ? inj.flag_wait_ns : kWaitNs;
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
@@ -1574,12 +1659,13 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         // nothing to prepare; the output pass still writes S_T = S0
     } else {
         *stage = "ws_prep";
-        e = cudaFuncSetAttribute(k_ws_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pp::TOTAL);
+        auto prep_kernel = raw ? k_ws_prep<true> : k_ws_prep<false>;
+        e = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pp::TOTAL);
         if (e != cudaSuccess) return e;
         const long items_bound = (long)l.nc_bound * H;
         const int grid = (int)std::max(1L, std::min(items_bound, (long)pp::CTAS_PER_SM * num_sms()));
         pr = prof_start("ws_prep", st);
-        e = launch_pdl(k_ws_prep, dim3(grid), dim3(256), pp::TOTAL, st, tm_k, g, beta, cu, N, T_tot, H, err,
+        e = launch_pdl(prep_kernel, dim3(grid), dim3(256), pp::TOTAL, st, tm_k, g, beta, cu, N, T_tot, H, err,
                        (const int32_t *)chunk_off, rec);
         prof_stop(pr);
         if (e != cudaSuccess) return e;
@@ -1591,7 +1677,8 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         pr = prof_start("ws_trans", st);
         e = launch_pdl(k_ws_trans, dim3(H, l.nslots), dim3(NT_TRANS), tb::TOTAL, st, tm_k, tm_v, S0, cu, N, T_tot, H,
                        err, (const int32_t *)seg_off, (const int32_t *)chunk_off, seg_chunks, (const uint8_t *)rec, link,
-                       flags, part, flags + (size_t)l.nslots * H, flag_ns, inj.withhold_first_link ? 1 : 0);
+                       flags, part, flags + (size_t)l.nslots * H, flag_ns, inj.withhold_first_link ? 1 : 0,
+                       raw ? 1 : 0);
         prof_stop(pr);
         if (e != cudaSuccess) return e;
     }
@@ -1602,7 +1689,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     e = launch_pdl(k_ws_out, dim3(H, l.nslots), dim3(NT_WS), ob::TOTAL, st, tm_q, tm_k, tm_v, tm_o, S0, cu, N, T_tot,
                    H, o, S_T, err, seg_chunks > 0 ? (const int32_t *)seg_off : nullptr, (const int32_t *)chunk_off,
                    seg_chunks > 0 ? seg_chunks : 1, (const uint8_t *)rec, (const uint8_t *)link,
-                   seg_chunks > 0 ? (const uint32_t *)flags : nullptr, flag_ns);
+                   seg_chunks > 0 ? (const uint32_t *)flags : nullptr, flag_ns, raw ? 1 : 0);
     prof_stop(pr);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

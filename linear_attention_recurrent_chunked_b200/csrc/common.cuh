@@ -32,6 +32,14 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
     return make_float4(fa.x, fa.y, fb.x, fb.y);
 }
 
+// Input preparation of the raw-input entry points (the layer's own gates and normalisation):
+// the decay exponent g = -softplus(a) (alpha = exp(g)) of a raw gate logit a, with
+// softplus(a) = max(a, 0) + log(1 + exp(-|a|)); the write strength beta = sigmoid(b); and the
+// factor 1 / max(||x||, 1e-12) that normalises a vector whose squared norm is ss.
+__device__ __forceinline__ float neg_softplus(float a) { return -(fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)))); }
+__device__ __forceinline__ float sigmoid_f(float b) { return 1.f / (1.f + expf(-b)); }
+__device__ __forceinline__ float inv_norm(float ss) { return rsqrtf(fmaxf(ss, 1e-24f)); }
+
 // Sequence bounds from cu_seqlens (device) or equal split, clamped to [0, T_tot].
 __device__ __forceinline__ void seq_bounds(const int32_t *cu, int n, int N, int T_tot, int &t0, int &t1) {
     if (cu) {

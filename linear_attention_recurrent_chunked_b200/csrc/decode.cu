@@ -117,8 +117,11 @@ __device__ __forceinline__ void load_token(const T *qt, const T *kt, const T *vt
     for (int i = 0; i < 4; ++i) vr[i] = Elem<T>::load(vt + rb.row(i));
 }
 
-// grid.x = B*H*(D/64): one CTA per 64 rows of one (b, h) state.
-template <typename T, int D>
+// grid.x = B*H*(D/64): one CTA per 64 rows of one (b, h) state. RAW: q, k arrive unnormalised
+// and g, beta hold the gate logits a, b: q and k are L2-normalised here (their squared norms
+// reduce over the same 8 lanes as the row dot products), alpha = exp(-softplus(a)) and
+// beta = sigmoid(b).
+template <typename T, int D, bool RAW>
 __global__ void __launch_bounds__(kThreads) k_decode_step(const T *__restrict__ q, const T *__restrict__ k,
                                                           const T *__restrict__ v, const float *__restrict__ g,
                                                           const float *__restrict__ beta, float *__restrict__ S,
@@ -131,8 +134,31 @@ __global__ void __launch_bounds__(kThreads) k_decode_step(const T *__restrict__ 
     rb.load(Sh);
     float kc[D / 32][4], qc[D / 32][4], vr[4], out[4];
     load_token<T, D>(q + (size_t)bh * D, k + (size_t)bh * D, v + (size_t)bh * D, rb, kc, qc, vr);
-    const float alpha = expf(g[bh]);
-    rb.step(kc, qc, vr, alpha, beta[bh], out);
+    float alpha, b;
+    if (RAW) {
+        float kk = 0.f, qq = 0.f;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                kk = fmaf(kc[j][c], kc[j][c], kk);
+                qq = fmaf(qc[j][c], qc[j][c], qq);
+            }
+        const float sk = inv_norm(red8(kk)), sq = inv_norm(red8(qq));
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                kc[j][c] *= sk;
+                qc[j][c] *= sq;
+            }
+        alpha = expf(neg_softplus(g[bh]));
+        b = sigmoid_f(beta[bh]);
+    } else {
+        alpha = expf(g[bh]);
+        b = beta[bh];
+    }
+    rb.step(kc, qc, vr, alpha, b, out);
     rb.store(Sh);
     if (rb.part == 0) {
 #pragma unroll
@@ -186,9 +212,12 @@ __global__ void __launch_bounds__(kThreads) k_seq_scan(const T *__restrict__ q, 
 
 template <typename T, int D>
 cudaError_t launch_decode_step(const T *q, const T *k, const T *v, const float *g, const float *beta, float *S,
-                               int B, int H, T *o, cudaStream_t st) {
+                               int B, int H, T *o, cudaStream_t st, bool raw) {
     const int grid = B * H * (D / kRowsPerCta);
-    k_decode_step<T, D><<<grid, kThreads, 0, st>>>(q, k, v, g, beta, S, o);
+    if (raw)
+        k_decode_step<T, D, true><<<grid, kThreads, 0, st>>>(q, k, v, g, beta, S, o);
+    else
+        k_decode_step<T, D, false><<<grid, kThreads, 0, st>>>(q, k, v, g, beta, S, o);
     return cudaGetLastError();
 }
 
@@ -202,7 +231,7 @@ cudaError_t launch_seq_scan(const T *q, const T *k, const T *v, const float *g, 
 
 #define GDN_INST(T, D)                                                                                         \
     template cudaError_t launch_decode_step<T, D>(const T *, const T *, const T *, const float *, const float *, \
-                                                  float *, int, int, T *, cudaStream_t);                     \
+                                                  float *, int, int, T *, cudaStream_t, bool);               \
     template cudaError_t launch_seq_scan<T, D>(const T *, const T *, const T *, const float *, const float *,    \
                                                const float *, const int32_t *, int, int, int, T *, float *,   \
                                                cudaStream_t);

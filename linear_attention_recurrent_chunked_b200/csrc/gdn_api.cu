@@ -171,9 +171,10 @@ size_t gdn_chunk_fwd_workspace_size(int N, int T_tot, int H, int dk, int dv, gdn
     return kErrWordBytes;
 }
 
-gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
-                         const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
-                         gdn_dtype dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
+static gdn_status chunk_fwd_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                 const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                                 gdn_dtype dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream,
+                                 bool raw) {
     gdn_status s = check_common(q, k, v, g, beta, o, T_tot, H, dk, dv, dtype);
     if (s != GDN_OK) return s;
     if (N < 1) return fail(GDN_ERR_SHAPE, "N=%d must be >= 1", N);
@@ -200,10 +201,14 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
         if (ws_bytes >= gdn::chunk_ws_workspace(N, T_tot, H, use_seg)) {
             e = gdn::launch_chunk_ws(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                                      static_cast<const __nv_bfloat16 *>(v), g, beta, S0, cu_seqlens, N, T_tot, H,
-                                     static_cast<__nv_bfloat16 *>(o), S_T, workspace, use_seg, st, &stage);
+                                     static_cast<__nv_bfloat16 *>(o), S_T, workspace, use_seg, st, &stage, raw);
             if (e != cudaSuccess) return cuda_fail(e, stage);
             return ok();
         }
+        if (raw)
+            return fail(GDN_ERR_WORKSPACE,
+                        "raw inputs need the pipelined path: workspace of %zu bytes given, at least %zu needed",
+                        ws_bytes, gdn::chunk_ws_workspace(N, T_tot, H, 0));
         e = gdn::launch_chunk_tc(static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
                                  static_cast<const __nv_bfloat16 *>(v), g, beta, S0, cu_seqlens, N, T_tot, H,
                                  static_cast<__nv_bfloat16 *>(o), S_T, workspace, ws_bytes, st, &stage);
@@ -220,18 +225,32 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const floa
         const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
                     *vf = static_cast<const float *>(v);
         float *of = static_cast<float *>(o);
-        e = (dk == 64) ? gdn::launch_chunk_simt<float, 64>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st)
-                       : gdn::launch_chunk_simt<float, 128>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st);
+        e = (dk == 64) ? gdn::launch_chunk_simt<float, 64>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st, raw)
+                       : gdn::launch_chunk_simt<float, 128>(qf, kf, vf, g, beta, S0, cu_seqlens, N, T_tot, H, of, S_T, err, st, raw);
     } else {
         const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k),
                             *vb = static_cast<const __nv_bfloat16 *>(v);
         __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
         e = (dk == 64)
-                ? gdn::launch_chunk_simt<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st)
-                : gdn::launch_chunk_simt<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st);
+                ? gdn::launch_chunk_simt<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st, raw)
+                : gdn::launch_chunk_simt<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S0, cu_seqlens, N, T_tot, H, ob, S_T, err, st, raw);
     }
     if (e != cudaSuccess) return cuda_fail(e, "chunked forward launch");
     return ok();
+}
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                         const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                         gdn_dtype dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, S0, cu_seqlens, N, T_tot, H, dk, dv, dtype, o, S_T, workspace, ws_bytes,
+                          stream, false);
+}
+
+gdn_status gdn_chunk_fwd_raw(const void *q_raw, const void *k_raw, const void *v, const float *a, const float *b,
+                             const float *S0, const int32_t *cu_seqlens, int N, int T_tot, int H, int dk, int dv,
+                             gdn_dtype dtype, void *o, float *S_T, void *workspace, size_t ws_bytes, void *stream) {
+    return chunk_fwd_impl(q_raw, k_raw, v, a, b, S0, cu_seqlens, N, T_tot, H, dk, dv, dtype, o, S_T, workspace,
+                          ws_bytes, stream, true);
 }
 
 gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *stream) {
@@ -247,8 +266,9 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
     return ok();
 }
 
-gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta, float *S,
-                           int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream) {
+static gdn_status decode_step_impl(const void *q, const void *k, const void *v, const float *g, const float *beta,
+                                   float *S, int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream,
+                                   bool raw) {
     if (B < 1) return fail(GDN_ERR_SHAPE, "B=%d must be >= 1", B);
     gdn_status s = check_common(q, k, v, g, beta, o, B, H, dk, dv, dtype);
     if (s != GDN_OK) return s;
@@ -261,17 +281,27 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const fl
         const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
                     *vf = static_cast<const float *>(v);
         float *of = static_cast<float *>(o);
-        e = (dk == 64) ? gdn::launch_decode_step<float, 64>(qf, kf, vf, g, beta, S, B, H, of, st)
-                       : gdn::launch_decode_step<float, 128>(qf, kf, vf, g, beta, S, B, H, of, st);
+        e = (dk == 64) ? gdn::launch_decode_step<float, 64>(qf, kf, vf, g, beta, S, B, H, of, st, raw)
+                       : gdn::launch_decode_step<float, 128>(qf, kf, vf, g, beta, S, B, H, of, st, raw);
     } else {
         const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(q), *kb = static_cast<const __nv_bfloat16 *>(k),
                             *vb = static_cast<const __nv_bfloat16 *>(v);
         __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
-        e = (dk == 64) ? gdn::launch_decode_step<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S, B, H, ob, st)
-                       : gdn::launch_decode_step<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S, B, H, ob, st);
+        e = (dk == 64) ? gdn::launch_decode_step<__nv_bfloat16, 64>(qb, kb, vb, g, beta, S, B, H, ob, st, raw)
+                       : gdn::launch_decode_step<__nv_bfloat16, 128>(qb, kb, vb, g, beta, S, B, H, ob, st, raw);
     }
     if (e != cudaSuccess) return cuda_fail(e, "decode step launch");
     return ok();
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v, const float *g, const float *beta, float *S,
+                           int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream) {
+    return decode_step_impl(q, k, v, g, beta, S, B, H, dk, dv, dtype, o, stream, false);
+}
+
+gdn_status gdn_decode_step_raw(const void *q_raw, const void *k_raw, const void *v, const float *a, const float *b,
+                               float *S, int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream) {
+    return decode_step_impl(q_raw, k_raw, v, a, b, S, B, H, dk, dv, dtype, o, stream, true);
 }
 
 gdn_status gdn_seq_scan(const void *q, const void *k, const void *v, const float *g, const float *beta,

@@ -10,7 +10,7 @@ namespace gdn {
 
 template <typename T, int D>
 cudaError_t launch_decode_step(const T *q, const T *k, const T *v, const float *g, const float *beta, float *S,
-                               int B, int H, T *o, cudaStream_t st);
+                               int B, int H, T *o, cudaStream_t st, bool raw = false);
 
 template <typename T, int D>
 cudaError_t launch_seq_scan(const T *q, const T *k, const T *v, const float *g, const float *beta, const float *S0,
@@ -19,7 +19,7 @@ cudaError_t launch_seq_scan(const T *q, const T *k, const T *v, const float *g, 
 template <typename T, int D>
 cudaError_t launch_chunk_simt(const T *q, const T *k, const T *v, const float *g, const float *beta, const float *S0,
                               const int32_t *cu, int N, int T_tot, int H, T *o, float *S_T, const uint32_t *err,
-                              cudaStream_t st);
+                              cudaStream_t st, bool raw = false);
 
 // Tensor-core chunked forward, bf16 inputs, dk = dv = 128. Launches the
 // validation / plan, the optional transition pass and the output pass;
@@ -38,10 +38,12 @@ size_t chunk_tc_workspace(int N, int T_tot, int H, int seg_chunks);
 // plan, the parallel prep pass (decay scalars and UT solve of every chunk),
 // the transition pass with its links (seg_chunks > 0 only) and the output
 // pass. Needs chunk_ws_workspace(N, T_tot, H, seg_chunks) bytes of workspace.
+// raw: q, k are unnormalised and g, beta hold the gate logits a, b (g = -softplus(a),
+// beta = sigmoid(b)); the normalisation and gates are applied inside the passes.
 cudaError_t launch_chunk_ws(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v, const float *g,
                             const float *beta, const float *S0, const int32_t *cu, int N, int T_tot, int H,
                             __nv_bfloat16 *o, float *S_T, void *workspace, int seg_chunks, cudaStream_t st,
-                            const char **stage);
+                            const char **stage, bool raw = false);
 int chunk_ws_seg_chunks(int N, int T_tot, int H, bool varlen);  // varlen: cu_seqlens given
 size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks);
 

@@ -29,6 +29,8 @@ SIGNATURES = {
     "gdn_last_error": (ctypes.c_char_p, []),
     "gdn_chunk_fwd_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "gdn_chunk_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "gdn_chunk_fwd_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
+    "gdn_decode_step_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_chunk_fwd_check": (_I, [_VP, _SZ, _VP]),
     "gdn_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_seq_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
@@ -131,6 +133,46 @@ def chunk_fwd(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = Non
     if check:
         _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
     return o, S_T
+
+
+def chunk_fwd_raw(q_raw, k_raw, v, a, b, S0=None, cu_seqlens=None, N: Optional[int] = None, o=None, S_T=None,
+                  workspace=None, check: bool = False):
+    """Chunked prefill from raw inputs (see include/gdn.h): q_raw, k_raw [T,H,dk] of any norm,
+    v [T,H,dv]; a, b [T,H] fp32 gate logits (g = -softplus(a), beta = sigmoid(b)); the rest as
+    chunk_fwd. The normalisation and gates run inside the library's kernels."""
+    lib = load_library()
+    _need_cuda(q_raw, k_raw, v, a, b, S0, cu_seqlens, o, S_T, workspace)
+    T_tot, H, dk = q_raw.shape
+    dv = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N = S0.shape[0] if S0 is not None else 1
+    if o is None:
+        o = torch.empty((T_tot, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    if S_T is None:
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q_raw.device)
+    dt = _DTYPE.get(q_raw.dtype, 99)
+    need = int(lib.gdn_chunk_fwd_workspace_size(N, T_tot, H, dk, dv, dt))
+    ws = workspace if workspace is not None else _workspace(need, q_raw.device)
+    _check(lib.gdn_chunk_fwd_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a), _ptr(b), _ptr(S0), _ptr(cu_seqlens),
+                                 N, T_tot, H, dk, dv, dt, _ptr(o), _ptr(S_T), _ptr(ws), ws.numel(), _stream()))
+    if check:
+        _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
+    return o, S_T
+
+
+def decode_step_raw(q_raw, k_raw, v, a, b, S, o=None):
+    """One decode step from raw inputs (q, k normalised and gates applied in the kernel)."""
+    lib = load_library()
+    _need_cuda(q_raw, k_raw, v, a, b, S, o)
+    B, H, dk = q_raw.shape
+    dv = v.shape[2]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q_raw.dtype, device=q_raw.device)
+    _check(lib.gdn_decode_step_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a), _ptr(b), _ptr(S), B, H, dk, dv,
+                                   _DTYPE.get(q_raw.dtype, 99), _ptr(o), _stream()))
+    return o
 
 
 def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = None, o=None, S_T=None):

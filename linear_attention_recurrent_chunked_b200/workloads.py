@@ -23,7 +23,9 @@ L2-normalised over the head dimension in fp32 (x / max(||x||, 1e-12)) and
 then cast to the input dtype (round to nearest even); g = -softplus(N(0,1))
 (natural-log decay, alpha = exp(g)); beta = sigmoid(N(0,1)); both fp32.
 Draw order from one ``torch.Generator().manual_seed(seed)``: [varlen lengths],
-q, k, v, g, beta, S0. ``stress=True`` replaces the decays by slow ones
+q, k, v, g, beta, S0. The same draws before normalisation and activation (q_raw,
+k_raw in the input dtype; gate logits a, b with g = -softplus(a), beta =
+sigmoid(b)) are returned too, for the entry points that take raw inputs. ``stress=True`` replaces the decays by slow ones
 (g ~ -U(0, 0.01)) and pushes beta towards one (sigmoid(N(0,1) + 3)), so the
 state carries information across thousands of tokens.
 """
@@ -73,11 +75,17 @@ def _unit(x: torch.Tensor) -> torch.Tensor:
     return F.normalize(x, p=2.0, dim=-1, eps=1e-12)
 
 
-def draw_tokens(gen: torch.Generator, shape_qk, shape_v, shape_gate, dtype: str, stress: bool = False):
-    """q, k, v, g, beta in the draw order above. Returns CPU tensors."""
+def draw_tokens(gen: torch.Generator, shape_qk, shape_v, shape_gate, dtype: str, stress: bool = False,
+                raw_out: Optional[dict] = None):
+    """q, k, v, g, beta in the draw order above. Returns CPU tensors. If ``raw_out`` is a dict,
+    it also receives the same draws before normalisation and activation: q_raw, k_raw (the N(0,1)
+    draws cast to the input dtype), a and b (the fp32 gate logits, so that g = -softplus(a) and
+    beta = sigmoid(b); the stress recipe has no such logits and gives none)."""
     tdt = TORCH_DTYPE[dtype]
-    q = _unit(torch.randn(shape_qk, generator=gen, dtype=torch.float32)).to(tdt)
-    k = _unit(torch.randn(shape_qk, generator=gen, dtype=torch.float32)).to(tdt)
+    q32 = torch.randn(shape_qk, generator=gen, dtype=torch.float32)
+    k32 = torch.randn(shape_qk, generator=gen, dtype=torch.float32)
+    q = _unit(q32).to(tdt)
+    k = _unit(k32).to(tdt)
     v = torch.randn(shape_v, generator=gen, dtype=torch.float32).to(tdt)
     g_raw = torch.randn(shape_gate, generator=gen, dtype=torch.float32)
     b_raw = torch.randn(shape_gate, generator=gen, dtype=torch.float32)
@@ -87,6 +95,9 @@ def draw_tokens(gen: torch.Generator, shape_qk, shape_v, shape_gate, dtype: str,
     else:
         g = -F.softplus(g_raw)
         beta = torch.sigmoid(b_raw)
+        if raw_out is not None:
+            raw_out.update(q_raw=q32.to(tdt).contiguous(), k_raw=k32.to(tdt).contiguous(), a=g_raw.contiguous(),
+                           b=b_raw.contiguous())
     return q.contiguous(), k.contiguous(), v.contiguous(), g.contiguous(), beta.contiguous()
 
 
@@ -115,12 +126,13 @@ def make_prefill(cfg, seed: int = 0, stress: bool = False, seqlens: Optional[Lis
     seqlens = [int(x) for x in seqlens]
     N = len(seqlens)
     T_tot = sum(seqlens)
-    q, k, v, g, beta = draw_tokens(gen, (T_tot, H, d), (T_tot, H, d), (T_tot, H), dtype, stress)
+    raw = {}
+    q, k, v, g, beta = draw_tokens(gen, (T_tot, H, d), (T_tot, H, d), (T_tot, H), dtype, stress, raw)
     S0 = (0.02 * torch.randn((N, H, d, d), generator=gen, dtype=torch.float32)).contiguous() if s0 else None
     cu = torch.zeros(N + 1, dtype=torch.int32)
     cu[1:] = torch.cumsum(torch.tensor(seqlens, dtype=torch.int64), 0).to(torch.int32)
     return dict(name=cfg.name, dtype=dtype, N=N, H=H, d=d, T_tot=T_tot, seqlens=seqlens,
-                q=q, k=k, v=v, g=g, beta=beta, S0=S0, cu_seqlens=cu)
+                q=q, k=k, v=v, g=g, beta=beta, S0=S0, cu_seqlens=cu, **raw)
 
 
 def make_decode(cfg: Decode = DECODE, seed: int = 0, steps: Optional[int] = None, B: Optional[int] = None,
@@ -134,7 +146,8 @@ def make_decode(cfg: Decode = DECODE, seed: int = 0, steps: Optional[int] = None
     d = cfg.d if d is None else d
     dtype = cfg.dtype if dtype is None else dtype
     gen = torch.Generator().manual_seed(seed)
-    q, k, v, g, beta = draw_tokens(gen, (steps, B, H, d), (steps, B, H, d), (steps, B, H), dtype, stress)
+    raw = {}
+    q, k, v, g, beta = draw_tokens(gen, (steps, B, H, d), (steps, B, H, d), (steps, B, H), dtype, stress, raw)
     S = (0.02 * torch.randn((B, H, d, d), generator=gen, dtype=torch.float32)).contiguous()
     return dict(name=cfg.name, dtype=dtype, B=B, H=H, d=d, steps=steps,
-                q=q, k=k, v=v, g=g, beta=beta, S=S)
+                q=q, k=k, v=v, g=g, beta=beta, S=S, **raw)
