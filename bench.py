@@ -352,6 +352,31 @@ def gpu_arm(args):
         for name in ("prefill_10k", "varlen"):
             _, _, _, e = prefill_entry(name, max(5, args.steps // 2), args.warmup)
             result[name] = e
+        # input preparation fused into the kernels (raw q, k and gate logits) against the caller
+        # preparing the inputs with torch on the GPU (a separate pass over q, k, g, beta) first
+        import torch.nn.functional as F
+        for name in ("prefill_2k", "prefill_10k"):
+            w = make_prefill(name, seed=0)
+            t = dev_inputs(w)
+            o = torch.empty_like(t["v"])
+            S_T = torch.empty((w["N"], w["H"], w["d"], w["d"]), dtype=torch.float32, device=dev)
+            fused = lambda: gdn.chunk_fwd_raw(t["q_raw"], t["k_raw"], t["v"], t["a"], t["b"], t["S0"],
+                                              t["cu_seqlens"], o=o, S_T=S_T)
+
+            def separate():
+                q = F.normalize(t["q_raw"].float(), dim=-1).to(t["q_raw"].dtype)
+                k = F.normalize(t["k_raw"].float(), dim=-1).to(t["k_raw"].dtype)
+                gdn.chunk_fwd(q, k, t["v"], -F.softplus(t["a"]), torch.sigmoid(t["b"]), t["S0"], t["cu_seqlens"],
+                              o=o, S_T=S_T)
+
+            ms_f = statistics.mean(time_steps(fused, max(5, args.steps // 2), args.warmup))
+            ms_s = statistics.mean(time_steps(separate, max(5, args.steps // 2), args.warmup))
+            result[name]["from_raw_inputs"] = {
+                "fused_ms": ms_f, "torch_prep_then_chunk_fwd_ms": ms_s,
+                "fused_tokens_per_s": w["T_tot"] / (ms_f * 1e-3),
+                "note": "raw q, k (unnormalised) and gate logits a, b: g = -softplus(a), beta = sigmoid(b); "
+                        "fused = gdn_chunk_fwd_raw, separate = torch normalise/softplus/sigmoid on the GPU, "
+                        "then gdn_chunk_fwd"}
         # GPU sequential scan comparator (the pages' chunked-vs-sequential ratio)
         for name in ("prefill_2k", "prefill_10k"):
             w = make_prefill(name, seed=0)
@@ -409,25 +434,30 @@ def decode_entry(args, torch, gdn, dev, dist, pk, make_decode):
     w = make_decode(seed=0)
     steps = w["steps"]
     q, k, v, g, beta = (w[x].to(dev) for x in ("q", "k", "v", "g", "beta"))
+    q_raw, k_raw, a, b = (w[x].to(dev) for x in ("q_raw", "k_raw", "a", "b"))
     sets = [w["S"].to(dev) for _ in range(4)]
     o = torch.empty_like(v)
     nbytes = decode_bytes(w["B"], w["H"], w["d"])
 
-    def run(state_sets):
+    def run(state_sets, raw=False):
         for t in range(steps):
-            gdn.decode_step(q[t], k[t], v[t], g[t], beta[t], state_sets[t % len(state_sets)], o=o[t])
+            if raw:  # raw q, k and gate logits: normalisation and gates inside the decode kernel
+                gdn.decode_step_raw(q_raw[t], k_raw[t], v[t], a[t], b[t], state_sets[t % len(state_sets)], o=o[t])
+            else:
+                gdn.decode_step(q[t], k[t], v[t], g[t], beta[t], state_sets[t % len(state_sets)], o=o[t])
 
     out = {}
-    for label, ss in (("l2_cold_4sets", sets), ("l2_resident_1set", sets[:1])):
+    for label, ss, raw in (("l2_cold_4sets", sets, False), ("l2_resident_1set", sets[:1], False),
+                           ("raw_inputs_l2_cold_4sets", sets, True)):
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            run(ss)  # warm-up outside capture
+            run(ss, raw)  # warm-up outside capture
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            run(ss)
+            run(ss, raw)
         for _ in range(max(3, args.warmup)):
             graph.replay()
         torch.cuda.synchronize()
