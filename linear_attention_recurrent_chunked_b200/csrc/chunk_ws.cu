@@ -743,26 +743,34 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            // base descriptors; every operand below is one of these plus a byte offset
+            const tc::Desc dq = tc::split_desc(tc::make_desc_sw128(sb + B_Q, 16, 1024));      // Q, K-major
+            const tc::Desc dk = tc::split_desc(tc::make_desc_sw128(sb + B_K, 16, 1024));      // K, K-major
+            const tc::Desc dkm = tc::split_desc(tc::make_desc_sw128(sb + B_K, 8192, 1024));   // K, MN-major
+            const tc::Desc dvm = tc::split_desc(tc::make_desc_sw128(sb + B_V, 8192, 1024));   // V, MN-major
+            const tc::Desc dt1 = tc::split_desc(tc::make_desc(sb + T1, 1024, 128));
+            const tc::Desc dt2 = tc::split_desc(tc::make_desc(sb + B_T2, 1024, 128));
+            const tc::Desc ds = tc::split_desc(tc::make_desc(sb + S, 2048, 128));
+            const tc::Desc dw = tc::split_desc(tc::make_desc(sb + W, 128, 2048));
+            const tc::Desc ddl = tc::split_desc(tc::make_desc(sb + DL, 2048, 128));
+            const tc::Desc dp = tc::split_desc(tc::make_desc(sb + P, 1024, 128));
             // X1 = Q K^T (rows 64..127 of the A operand read the next 64 rows of the buffer; never used)
             auto issue_x1 = [&](int c) {
-                const uint32_t bb = buf(c);
+                const uint32_t bo = (uint32_t)(c & 1) * BUF;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    tc::mma_bf16(tm + TM_X1, tc::make_desc_sw128(bb + B_Q + off, 16, 1024),
-                                 tc::make_desc_sw128(bb + B_K + off, 16, 1024), id_kk64, kk > 0);
+                    const uint32_t off = bo + (kk >> 2) * 8192 + (kk & 3) * 32;
+                    tc::mma_bf16_off(tm + TM_X1, dq, off, dk, off, id_kk64, kk > 0);
                 }
                 tc::mma_commit(&bar[X1F]);
             };
             // W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views of the K and V tiles)
             auto issue_wu = [&](int c) {
-                const uint32_t bb = buf(c);
+                const uint32_t bo = (uint32_t)(c & 1) * BUF;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024),
-                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                    tc::mma_bf16(tm + TM_U, tc::make_desc_sw128(bb + B_V + kk * 2048, 8192, 1024),
-                                 tc::make_desc(bb + B_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_WT, dkm, bo + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_U, dvm, bo + kk * 2048, dt2, bo + kk * 2048, id_mk64, kk > 0);
                 }
                 tc::mma_commit(&bar[WUF]);
             };
@@ -774,27 +782,24 @@ __global__ void __launch_bounds__(NT_WS, 1)
             }
             for (int c = 0; ok && c < nch; ++c) {
                 const int b = c & 1;
-                const uint32_t par = (uint32_t)(c & 1), bb = buf(c);
+                const uint32_t par = (uint32_t)(c & 1), bo = (uint32_t)b * BUF;
                 if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
                 // Delta^T = U^T + S (-W)^T, accumulated onto U^T; then O1 = S Q^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_U, tc::make_desc(sb + S + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
+                    tc::mma_bf16_off(tm + TM_U, ds, kk * 4096, dw, kk * 256, id_km64, 1);
                 tc::mma_commit(&bar[M3]);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_O1 + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(bb + B_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_kk64,
-                                 kk > 0);
+                    tc::mma_bf16_off(tm + TM_O1 + 64 * b, ds, kk * 4096, dq, bo + (kk >> 2) * 8192 + (kk & 3) * 32,
+                                     id_kk64, kk > 0);
                 // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K)
                 if (!(ok = wait_bar(&bar[DLR], par, ctl, err) && wait_bar(&bar[PR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(bb + B_K + kk * 2048, 8192, 1024), id_km128, 1);
+                    tc::mma_bf16_off(tm + TM_S, ddl, kk * 4096, dkm, bo + kk * 2048, id_km128, 1);
                 tc::mma_commit(&bar[M4S]);
                 tc::mma_commit(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
                 // the next chunk's W^T, U^T and X1
@@ -811,8 +816,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_O2, tc::make_desc(sb + DL + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + P + b * 8192 + kk * 2048, 1024, 128), id_kk64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_O2, ddl, kk * 4096, dp, b * 8192 + kk * 2048, id_kk64, kk > 0);
                 tc::mma_commit(&bar[M4O]);
             }
         }
@@ -1137,6 +1141,10 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         // ---------------------------------------------------------------- W issuer: W^T = K^T T1^T, U^T = V^T T2^T
         if (lane == 0 && nch > 0) {
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
+            const tc::Desc dkm = tc::split_desc(tc::make_desc_sw128(sb + KRING + KS_K, 8192, 1024));
+            const tc::Desc dvm = tc::split_desc(tc::make_desc_sw128(sb + VRING + VS_V, 8192, 1024));
+            const tc::Desc dt1 = tc::split_desc(tc::make_desc(sb + T1, 1024, 128));
+            const tc::Desc dt2 = tc::split_desc(tc::make_desc(sb + VRING + VS_T2, 1024, 128));
             bool ok = true;
             for (int c = 0; ok && c < nch; ++c) {
                 // W^T(c - 1) read by prep (WR), the U^T buffer's Delta_S^T of chunk c - 2 read (DSR),
@@ -1148,13 +1156,12 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                            wait_bar(&bar[T1R], (uint32_t)(c & 1), ctl, err)))
                     break;
                 tc::fence_after_sync();
-                const uint32_t kt = sb + kslot(c) + KS_K, vs = sb + vslot(c);
+                const uint32_t ko = (uint32_t)(c % 3) * KSLOT, vo = (uint32_t)(c & 1) * VSLOT;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16(tm + TM_WT, tc::make_desc_sw128(kt + kk * 2048, 8192, 1024),
-                                 tc::make_desc(sb + T1 + kk * 2048, 1024, 128), id_mk64, kk > 0);
-                    tc::mma_bf16(tm + TM_U + 64 * (c & 1), tc::make_desc_sw128(vs + VS_V + kk * 2048, 8192, 1024),
-                                 tc::make_desc(vs + VS_T2 + kk * 2048, 1024, 128), id_mk64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_WT, dkm, ko + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_U + 64 * (c & 1), dvm, vo + kk * 2048, dt2, vo + kk * 2048, id_mk64,
+                                     kk > 0);
                 }
                 tc::mma_commit(&bar[WUF]);
                 tc::mma_commit(&bar[EMPTYV + (c & 1)]);
@@ -1165,17 +1172,20 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         if (lane == 0 && nch > 0) {
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            const tc::Desc ds = tc::split_desc(tc::make_desc(sb + S, 2048, 128));
+            const tc::Desc dw = tc::split_desc(tc::make_desc(sb + W, 128, 2048));
+            const tc::Desc dts = tc::split_desc(tc::make_desc(sb + DTS, 2048, 128));
+            const tc::Desc dkm = tc::split_desc(tc::make_desc_sw128(sb + KRING + KS_K, 8192, 1024));
             bool ok = true;
             for (int c = 0; ok && c < nch; ++c) {
                 const int b = c & 1;
-                const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
+                const uint32_t par = (uint32_t)(c & 1), ko = (uint32_t)(c % 3) * KSLOT;
                 // Delta_S^T = U^T + S (-W)^T, accumulated onto U^T (W^T, U^T are complete: prep saw WUF before WR)
                 if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_U + 64 * b, tc::make_desc(sb + S + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, 1);
+                    tc::mma_bf16_off(tm + TM_U + 64 * b, ds, kk * 4096, dw, kk * 256, id_km64, 1);
                 tc::mma_commit(&bar[M3S]);
                 // S <- gamma_C S + Delta_S^T (diag(e) K)
                 if (!(ok = wait_bar(&bar[DSR + b], (uint32_t)((c >> 1) & 1), ctl, err) &&
@@ -1184,8 +1194,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_S, tc::make_desc(sb + DTS + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
+                    tc::mma_bf16_off(tm + TM_S, dts, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
                 tc::mma_commit(&bar[M4S]);
                 tc::mma_commit(&bar[EMPTYK + c % 3]);
             }
@@ -1195,16 +1204,19 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         if (lane == 0 && nch > 0 && has_x) {
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+            const tc::Desc dx = tc::split_desc(tc::make_desc(sb + X, 2048, 128));
+            const tc::Desc dw = tc::split_desc(tc::make_desc(sb + W, 128, 2048));
+            const tc::Desc dtx = tc::split_desc(tc::make_desc(sb + DTX, 2048, 128));
+            const tc::Desc dkm = tc::split_desc(tc::make_desc_sw128(sb + KRING + KS_K, 8192, 1024));
             bool ok = true;
             for (int c = 0; ok && c < nch; ++c) {
-                const uint32_t par = (uint32_t)(c & 1), kt = sb + kslot(c) + KS_K;
+                const uint32_t par = (uint32_t)(c & 1), ko = (uint32_t)(c % 3) * KSLOT;
                 // X (-W)^T
                 if (!(ok = wait_bar(&bar[XR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16(tm + TM_DX, tc::make_desc(sb + X + kk * 4096, 2048, 128),
-                                 tc::make_desc(sb + W + kk * 256, 128, 2048), id_km64, kk > 0);
+                    tc::mma_bf16_off(tm + TM_DX, dx, kk * 4096, dw, kk * 256, id_km64, kk > 0);
                 tc::mma_commit(&bar[M3X]);
                 // X <- gamma_C X + X (-W)^T diag(e) K
                 if (!(ok = wait_bar(&bar[DXR], par, ctl, err) &&
@@ -1213,8 +1225,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16(tm + TM_X, tc::make_desc(sb + DTX + kk * 4096, 2048, 128),
-                                 tc::make_desc_sw128(kt + kk * 2048, 8192, 1024), id_km128, 1);
+                    tc::mma_bf16_off(tm + TM_X, dtx, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
                 tc::mma_commit(&bar[M4X]);
                 tc::mma_commit(&bar[EMPTYK + c % 3]);
             }

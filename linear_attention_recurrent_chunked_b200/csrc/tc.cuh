@@ -102,6 +102,28 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// A shared-memory descriptor as its two 32-bit words. The start-address field is the low 14 bits
+// (address / 16) and every operand tile here lies below 256 KB of shared memory, so the descriptor
+// of (base + off) for a 16-byte multiple off is the base descriptor with off / 16 added to its low
+// word: an MMA loop then needs one integer add per operand instead of rebuilding the descriptor.
+struct Desc {
+    uint32_t lo, hi;
+};
+__device__ __forceinline__ Desc split_desc(uint64_t d) { return Desc{(uint32_t)d, (uint32_t)(d >> 32)}; }
+
+// D[tmem] (+)= A * B^T with both descriptors given as base + byte offset.
+__device__ __forceinline__ void mma_bf16_off(uint32_t d_tmem, Desc a, uint32_t a_off, Desc b, uint32_t b_off,
+                                             uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+        "mov.b64 ad, {%1, %2};\n\t"
+        "mov.b64 bd, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a.lo + (a_off >> 4)), "r"(a.hi), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on the mbarrier when all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))
