@@ -388,6 +388,7 @@ def gpu_arm(args):
             result[name]["seq_scan_ms"] = statistics.mean(ts)
             result[name]["chunked_over_sequential"] = statistics.mean(ts) / result[name]["ms_per_step"]
         result["decode"] = decode_entry(args, torch, gdn, dev, dist, pk, make_decode)
+        result["projection"] = projection_entry(args, torch, gdn, dev, dist, pk, time_steps)
 
     # ---------------- JSON line
     main = result["prefill_2k"]
@@ -426,6 +427,37 @@ def gpu_arm(args):
     if dist is not None:
         dist.barrier(device_ids=[dev.index])
         dist.destroy_process_group()
+
+
+def projection_entry(args, torch, gdn, dev, dist, pk, time_steps):
+    """The int8-weight input projection of the layer (x [T, 1024] -> q, k, v, a, b with H = 16,
+    d = 128: N = 6176 channels) at the prefill sizes (tensor-bound: flops over the measured dense
+    bf16 peak) and at the decode size T = 64 (one token for each of the 64 sequences: bound by
+    reading the int8 weights; bytes over the measured HBM bandwidth). L2 flushed before each step."""
+    from linear_attention_recurrent_chunked_b200.workloads import make_projection
+    out = {}
+    for T in (2048, 10240, 64):
+        p = make_projection(T, seed=0)
+        x, w, sc = p["x"].to(dev), p["w"].to(dev), p["scale"].to(dev)
+        H, dk, dv, D, N = p["H"], p["dk"], p["dv"], p["D"], p["N"]
+        bufs = gdn.proj_w8(x, w, sc, H, dk, dv)
+        fn = lambda: gdn.proj_w8(x, w, sc, H, dk, dv, out=bufs)
+        ms = max_over_ranks(dist, statistics.mean(time_steps(fn, max(5, args.steps // 2), args.warmup)), dev)
+        gdn.proj_w8(x, w, sc, H, dk, dv, out=bufs, check=True)
+        flops = 2.0 * T * D * N
+        nbytes = T * D * 2 + N * D + N * 4 + T * (2 * H * dk + H * dv) * 2 + 2 * T * H * 4
+        tflops = flops / (ms * 1e-3) / 1e12
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        entry = {"T": T, "D": D, "N": N, "ms": ms, "tflops": tflops, "GB_per_s": gbs,
+                 "algorithmic_flops": flops, "algorithmic_bytes": nbytes}
+        if flops / nbytes > pk["bf16"] * 1e12 / (pk["hbm"] * 1e9):
+            entry["roofline"] = {"bound": "tensor", "achieved": tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                                 "frac": tflops / pk["bf16"], "peak_source": pk["src"]}
+        else:
+            entry["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                                 "frac": gbs / pk["hbm"], "peak_source": pk["src"]}
+        out["T%d" % T] = entry
+    return out
 
 
 def decode_entry(args, torch, gdn, dev, dist, pk, make_decode):

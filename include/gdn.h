@@ -211,6 +211,30 @@ gdn_status gdn_decode_step_raw(const void *q_raw, const void *k_raw, const void 
                                int B, int H, int dk, int dv, gdn_dtype dtype, void *o, void *stream);
 
 /*
+ * Input projection of the recurrent layer with int8 weights. The pages' system
+ * keeps its language-model weights as 8-bit codes dequantised for the
+ * projections (page 1, abstract; page 2, "Resumen Tecnico", the GEMM item);
+ * this is that projection for the recurrent layer, producing exactly the raw
+ * inputs gdn_chunk_fwd_raw / gdn_decode_step_raw take:
+ *     y[t][n] = scale[n] * sum_j x[t][j] w[n][j]        (fp32 accumulation)
+ * with output channels in the order q (H dk), k (H dk), v (H dv), a (H), b (H),
+ * head-major inside each, N = H (2 dk + dv) + 2 H. The int8 codes are exact in
+ * bf16: the product runs on the tensor cores with bf16 operands and the scale
+ * is applied to the fp32 result, so the weights cross HBM as int8 and the
+ * dequantisation is exact. The pages do not fix a quantisation scheme; this one
+ * is symmetric with one scale per output channel.
+ *   x [T][D] bf16 (D a positive multiple of 64); w [N][D] int8; scale [N] fp32;
+ *   q_raw, k_raw [T][H][dk] bf16; v [T][H][dv] bf16; a, b [T][H] fp32
+ *   (outputs, rounded to nearest even for bf16); H dk and H dv multiples of 8.
+ *   workspace, ws_bytes: >= 256 bytes of device memory for the error word
+ *   (gdn_chunk_fwd_check reads it: GDN_ERR_TIMEOUT if a bounded wait gave up).
+ * Pointers 16-byte aligned (a, b: 4). Runs one persistent kernel on `stream`.
+ */
+gdn_status gdn_proj_w8(const void *x, const int8_t *w, const float *scale, int T, int D, int H, int dk,
+                       int dv, void *q_raw, void *k_raw, void *v, float *a, float *b,
+                       void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * The sequential (token-by-token) scan on the GPU: the same result as
  * gdn_chunk_fwd, computed one token at a time with the decode step's row
  * update. It is the comparator for the chunked path's speed-up (page 1,

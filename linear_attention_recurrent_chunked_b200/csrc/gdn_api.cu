@@ -335,6 +335,31 @@ gdn_status gdn_seq_scan(const void *q, const void *k, const void *v, const float
     return ok();
 }
 
+gdn_status gdn_proj_w8(const void *x, const int8_t *w, const float *scale, int T, int D, int H, int dk, int dv,
+                       void *q_raw, void *k_raw, void *v, float *a, float *b, void *workspace, size_t ws_bytes,
+                       void *stream) {
+    if (T < 0 || D < 64 || D % 64 != 0 || H < 1 || dk < 1 || dv < 1 || (H * dk) % 8 != 0 || (H * dv) % 8 != 0)
+        return fail(GDN_ERR_SHAPE, "T=%d D=%d H=%d dk=%d dv=%d unsupported (D a positive multiple of 64, H dk and "
+                    "H dv multiples of 8)", T, D, H, dk, dv);
+    if ((double)T * D >= 2.0e9 || (double)H * (2 * dk + dv) >= 1.0e6) return fail(GDN_ERR_SHAPE, "sizes overflow");
+    if (T > 0 && (!x || !w || !scale || !q_raw || !k_raw || !v || !a || !b))
+        return fail(GDN_ERR_NULL, "x, w, scale and every output are required");
+    const void *p16[] = {x, w, scale, q_raw, k_raw, v};
+    for (const void *p : p16)
+        if (misaligned(p)) return fail(GDN_ERR_ALIGN, "pointer %p is not 16-byte aligned", p);
+    if ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 3u)
+        return fail(GDN_ERR_ALIGN, "a and b must be 4-byte aligned");
+    if (!workspace || ws_bytes < kErrWordBytes)
+        return fail(GDN_ERR_WORKSPACE, "workspace of at least %zu bytes (the error word) needed", kErrWordBytes);
+    const char *stage = "";
+    const cudaError_t e = gdn::launch_proj_w8(
+        static_cast<const __nv_bfloat16 *>(x), w, scale, T, D, H, dk, dv, static_cast<__nv_bfloat16 *>(q_raw),
+        static_cast<__nv_bfloat16 *>(k_raw), static_cast<__nv_bfloat16 *>(v), a, b, static_cast<uint32_t *>(workspace),
+        static_cast<cudaStream_t>(stream), &stage);
+    if (e != cudaSuccess) return cuda_fail(e, stage);
+    return ok();
+}
+
 gdn_status gdn_debug_inject(int kind, unsigned wait_us) {
     if (kind != GDN_INJECT_NONE && kind != GDN_INJECT_WITHHOLD_LINK)
         return fail(GDN_ERR_SHAPE, "unknown injection kind %d", kind);

@@ -47,6 +47,13 @@ cudaError_t launch_chunk_ws(const __nv_bfloat16 *q, const __nv_bfloat16 *k, cons
 int chunk_ws_seg_chunks(int N, int T_tot, int H, bool varlen);  // varlen: cu_seqlens given
 size_t chunk_ws_workspace(int N, int T_tot, int H, int seg_chunks);
 
+// Input projection with int8 weights (W8A16 on the tensor cores): y = x (diag(scale) w)^T split
+// into q, k, v (bf16) and the gate logits a, b (fp32). x [T][D] bf16 (D % 64 == 0), w [N][D] int8,
+// N = H (2 dk + dv) + 2 H; err is the error word (reset here).
+cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float *scale, int T, int D, int H, int dk,
+                           int dv, __nv_bfloat16 *q, __nv_bfloat16 *k, __nv_bfloat16 *v, float *a, float *b,
+                           uint32_t *err, cudaStream_t st, const char **stage);
+
 // Failure injection for tests (set by gdn_debug_inject; off by default): the pipelined path's
 // first segment of head 0 withholds its end-state flag, and waits for flags give up after
 // flag_wait_ns (0 = the normal bound) instead of hanging.

@@ -1,0 +1,352 @@
+// Input projection of the recurrent layer with int8 weights, on the sm_100a tensor cores.
+//
+// The pages' system keeps the language model's weights as 8-bit codes that are dequantised for
+// the projections (page 1, abstract: int8 weights dequantised once; page 2, "Resumen Tecnico",
+// the GEMM item). For the recurrent layer the projection turns hidden states x [T][D] into the
+// layer's raw inputs: q, k, v (H heads of dk, dk, dv values, bf16) and the gate logits a, b
+// (one per head, fp32), with one weight matrix of N = H (2 dk + dv) + 2 H output channels stored
+// as int8 codes w[n][j] and one fp32 scale per channel:
+//
+//     y[t][n] = scale[n] * sum_j x[t][j] w[n][j]
+//
+// Columns in the order q, k, v, a, b (head-major inside each), written straight into the
+// layouts gdn_chunk_fwd_raw / gdn_decode_step_raw read. The int8 codes are exact in bf16, so the
+// product runs on bf16 operands with fp32 accumulation and the scale is applied to the fp32
+// result: the dequantisation is exact and the weights cross HBM as int8 (half the bytes of bf16).
+//
+// One persistent CTA per SM walks output tiles of 128 tokens x 256 channels (K steps of 64):
+//   loader    (1 thread)   TMA: x tile (bf16, 128-byte swizzle) and int8 weight tile, 4-deep ring
+//   convert   (4 warps)    int8 tile -> bf16 K-major 128-byte-swizzled operand tile, 2-deep ring
+//   MMA       (1 thread)   4 tcgen05.mma (M=128, N=256, K=16) per K step into a TMEM accumulator
+//                          (two accumulators of 256 columns: one tile's epilogue overlaps the next)
+//   epilogue  (4 warps)    TMEM -> fp32 registers -> * scale -> bf16 / fp32 rows in global memory
+// Every wait is bounded in time; a timeout sets the error word and all roles leave their loops.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace gdn {
+namespace {
+
+using bf16_t = __nv_bfloat16;
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int NSTAGE = 4, NBSLOT = 2;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB bf16 x tile
+constexpr uint32_t W8_BYTES = BN * BK;      // 16 KB int8 weight tile
+constexpr uint32_t B_BYTES = BN * BK * 2;   // 32 KB bf16 weight tile
+constexpr uint32_t OFF_A = 0;
+constexpr uint32_t OFF_W8 = OFF_A + NSTAGE * A_BYTES;
+constexpr uint32_t OFF_B = OFF_W8 + NSTAGE * W8_BYTES;
+constexpr uint32_t OFF_BAR = OFF_B + NBSLOT * B_BYTES;
+enum {
+    FULL = 0,                    // [4] x and w8 of a stage landed (loader arrive + bytes)
+    EMPTY = FULL + NSTAGE,       // [4] stage free: MMA commit (x read) + converters (w8 read)
+    BFULL = EMPTY + NSTAGE,      // [2] bf16 weight tile written (128 converter threads)
+    BEMPTY = BFULL + NBSLOT,     // [2] bf16 weight tile read by the MMAs (commit)
+    AFULL = BEMPTY + NBSLOT,     // [2] accumulator complete (commit)
+    AEMPTY = AFULL + 2,          // [2] accumulator read out (128 epilogue threads)
+    FIN = AEMPTY + 2,            // every MMA of the CTA done (drained before TMEM is freed)
+    NBAR = FIN + 1
+};
+constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
+constexpr uint32_t SMEM_TOTAL = OFF_CTL + 16 + 1024;  // + alignment slack
+constexpr int NTHREADS = 320;                           // 10 warps
+constexpr int W_LOAD = 0, W_MMA = 1;                    // converters: warps 2-5; epilogue: warps 6-9
+__host__ __device__ constexpr uint32_t bar_count(int i) {
+    return (i >= EMPTY && i < EMPTY + NSTAGE) ? 129u : (i >= BFULL && i < BFULL + NBSLOT) ? 128u
+           : (i >= AEMPTY && i < AEMPTY + 2) ? 128u : 1u;
+}
+
+struct Ctl {
+    uint32_t tmem, abort;
+};
+
+__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    if (tc::mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = tc::globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (tc::mbar_try_wait(bar, parity)) return true;
+        if ((i & 15u) == 0) {
+            if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
+            if (tc::globaltimer() - t0 > kWaitNs) {
+                if (err) atomicOr(err, ERRBIT_TIMEOUT);
+                *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+                return false;
+            }
+        }
+    }
+}
+__device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = tc::globaltimer();
+    while (!tc::mbar_try_wait(bar, parity))
+        if (tc::globaltimer() - t0 > kWaitNs) return;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint64_t *mbar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(tc::smem_u32(mbar))
+        : "memory");
+}
+
+// Where output column n goes: region 0..4 = q, k, v (bf16 [T][width]), a, b (fp32 [T][H]).
+struct Route {
+    int Hdk, Hdv, H, N;
+};
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    k_proj_w8(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+              const float *__restrict__ scale, int T, int D, Route rt, bf16_t *__restrict__ q, bf16_t *__restrict__ k,
+              bf16_t *__restrict__ v, float *__restrict__ ga, float *__restrict__ gb, uint32_t *__restrict__ err) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = tc::smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);  // 1024-byte aligned for the swizzle
+    const uint32_t sb = tc::smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + OFF_CTL);
+    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
+    if (tid == 32) {
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
+        ctl->abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tm = ctl->tmem;
+    const int mt = (T + BM - 1) / BM, nt = (rt.N + BN - 1) / BN, ksteps = D / BK;
+    const int ntiles = mt * nt;
+
+    if (warp == W_LOAD) {
+        if (lane == 0) {
+            int it = 0, issued = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+                const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = it % NSTAGE;
+                    if (it >= NSTAGE && !(ok = wait_bar(&bar[EMPTY + s], (uint32_t)(((it / NSTAGE) - 1) & 1), ctl, err)))
+                        break;
+                    tc::mbar_arrive_expect_tx(&bar[FULL + s], A_BYTES + W8_BYTES);
+                    tma_load_2d(sb + OFF_A + s * A_BYTES, &tm_x, &bar[FULL + s], ks * BK, m0);
+                    tma_load_2d(sb + OFF_W8 + s * W8_BYTES, &tm_w, &bar[FULL + s], ks * BK, n0);
+                    issued = it + 1;
+                }
+            }
+            for (int j = std::max(0, issued - NSTAGE); j < issued; ++j)
+                drain_bar(&bar[FULL + j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
+        }
+    } else if (warp == W_MMA) {
+        if (lane == 0) {
+            const uint32_t idesc = tc::make_idesc_bf16(BM, BN, 0, 0);
+            const tc::Desc da = tc::split_desc(tc::make_desc_sw128(sb + OFF_A, 16, 1024));
+            const tc::Desc db = tc::split_desc(tc::make_desc_sw128(sb + OFF_B, 16, 1024));
+            int it = 0, ti = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
+                const int acc = ti & 1;
+                if (ti >= 2 && !(ok = wait_bar(&bar[AEMPTY + acc], (uint32_t)(((ti >> 1) - 1) & 1), ctl, err))) break;
+                tc::fence_after_sync();
+                for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                    const int s = it % NSTAGE, bs = it % NBSLOT;
+                    if (!(ok = wait_bar(&bar[FULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
+                               wait_bar(&bar[BFULL + bs], (uint32_t)((it / NBSLOT) & 1), ctl, err)))
+                        break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        tc::mma_bf16_off(tm + acc * BN, da, s * A_BYTES + kk * 32, db, bs * B_BYTES + kk * 32, idesc,
+                                         (ks > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&bar[EMPTY + s]);
+                    tc::mma_commit(&bar[BEMPTY + bs]);
+                }
+                if (ok) tc::mma_commit(&bar[AFULL + acc]);
+            }
+            tc::mma_commit(&bar[FIN]);
+            drain_bar(&bar[FIN], 0);
+        }
+    } else if (warp < 6) {
+        // ---------------------------------------------------------------- convert (128 threads)
+        const int t = tid - 64;
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+            for (int ks = 0; ks < ksteps; ++ks, ++it) {
+                const int s = it % NSTAGE, bs = it % NBSLOT;
+                ok = wait_bar(&bar[FULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
+                     (it < NBSLOT || wait_bar(&bar[BEMPTY + bs], (uint32_t)(((it / NBSLOT) - 1) & 1), ctl, err));
+                if (!(ok = __all_sync(0xffffffffu, ok))) break;
+                tc::fence_after_sync();
+                const uint8_t *w8 = smem + OFF_W8 + s * W8_BYTES;
+                uint8_t *bt = smem + OFF_B + bs * B_BYTES;
+                // 16-byte chunk c of the int8 tile (row c / 4, codes 16 (c % 4) ..): consecutive threads read
+                // consecutive chunks; each becomes two 16-byte bf16 chunks of the row's swizzled 128 bytes
+#pragma unroll 2
+                for (int c = t; c < BN * BK / 16; c += 128) {
+                    const int row = c >> 2, q4 = c & 3;
+                    const uint4 raw = *reinterpret_cast<const uint4 *>(w8 + 16 * c);
+                    const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+                    uint32_t o[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int32_t x = (int32_t)wd[j];
+                        o[2 * j] = tc::pack_bf16x2((float)(int8_t)(x & 0xff), (float)(int8_t)((x >> 8) & 0xff));
+                        o[2 * j + 1] = tc::pack_bf16x2((float)(int8_t)((x >> 16) & 0xff), (float)(int8_t)(x >> 24));
+                    }
+                    const uint32_t rbase = (uint32_t)row * 128u, sw = (uint32_t)(row & 7);
+                    *reinterpret_cast<uint4 *>(bt + rbase + (((2u * q4) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4 *>(bt + rbase + (((2u * q4 + 1u) ^ sw) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                tc::fence_smem_to_async();
+                tc::mbar_arrive(&bar[BFULL + bs]);
+                tc::mbar_arrive(&bar[EMPTY + s]);  // this thread's reads of the int8 stage are done
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- epilogue (128 threads)
+        const int row = (warp & 3) * 32 + lane;  // this thread's TMEM lane = token row of the tile
+        const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
+        int ti = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
+            const int acc = ti & 1;
+            const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+            if (!(ok = __all_sync(0xffffffffu, wait_bar(&bar[AFULL + acc], (uint32_t)((ti >> 1) & 1), ctl, err))))
+                break;
+            tc::fence_after_sync();
+            const int t = m0 + row;
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                float x[32];
+                tc::tmem_ld32(tl + acc * BN + c0, x);
+                const int n = n0 + c0;
+                if (t >= T || n >= rt.N) continue;
+                if (n + 32 <= rt.N) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 s4 = __ldg(reinterpret_cast<const float4 *>(scale + n + i));
+                        x[i] *= s4.x; x[i + 1] *= s4.y; x[i + 2] *= s4.z; x[i + 3] *= s4.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] *= (n + i < rt.N) ? __ldg(scale + n + i) : 0.f;
+                }
+                // 32 columns inside one bf16 region: four 16-byte stores; otherwise column by column
+                const int r0 = n < rt.Hdk ? 0 : n < 2 * rt.Hdk ? 1 : n < 2 * rt.Hdk + rt.Hdv ? 2 : 3;
+                const int base = r0 == 0 ? 0 : r0 == 1 ? rt.Hdk : 2 * rt.Hdk;
+                const int width = r0 == 2 ? rt.Hdv : rt.Hdk;
+                if (r0 < 3 && n + 32 <= base + width) {
+                    bf16_t *dst = (r0 == 0 ? q : r0 == 1 ? k : v) + (size_t)t * width + (n - base);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8)
+                        *reinterpret_cast<uint4 *>(dst + i) =
+                            make_uint4(tc::pack_bf16x2(x[i], x[i + 1]), tc::pack_bf16x2(x[i + 2], x[i + 3]),
+                                       tc::pack_bf16x2(x[i + 4], x[i + 5]), tc::pack_bf16x2(x[i + 6], x[i + 7]));
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = n + i;
+                        if (c >= rt.N) break;
+                        if (c < rt.Hdk) q[(size_t)t * rt.Hdk + c] = __float2bfloat16_rn(x[i]);
+                        else if (c < 2 * rt.Hdk) k[(size_t)t * rt.Hdk + c - rt.Hdk] = __float2bfloat16_rn(x[i]);
+                        else if (c < 2 * rt.Hdk + rt.Hdv) v[(size_t)t * rt.Hdv + c - 2 * rt.Hdk] = __float2bfloat16_rn(x[i]);
+                        else if (c < 2 * rt.Hdk + rt.Hdv + rt.H) ga[(size_t)t * rt.H + c - 2 * rt.Hdk - rt.Hdv] = x[i];
+                        else gb[(size_t)t * rt.H + c - 2 * rt.Hdk - rt.Hdv - rt.H] = x[i];
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(&bar[AEMPTY + acc]);
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tc::tmem_dealloc(tm, 512);
+}
+
+}  // namespace
+}  // namespace gdn
+
+namespace gdn {
+namespace {
+
+cudaError_t encode_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                      uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    if (!encode) return cudaErrorNotSupported;
+    const cuuint64_t dims[2] = {inner, std::max<uint64_t>(outer, 1)};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+int sm_count() {
+    static int n = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    });
+    return n;
+}
+
+}  // namespace
+
+cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float *scale, int T, int D, int H, int dk,
+                           int dv, __nv_bfloat16 *q, __nv_bfloat16 *k, __nv_bfloat16 *v, float *a, float *b,
+                           uint32_t *err, cudaStream_t st, const char **stage) {
+    cudaError_t e;
+    *stage = "error word reset";
+    if ((e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+    const int N = H * (2 * dk + dv) + 2 * H;
+    if (T == 0) return cudaSuccess;
+    CUtensorMap tm_x, tm_w;
+    *stage = "TMA descriptor encoding";
+    if ((e = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, BK, BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+        return e;
+    if ((e = encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)D, (uint64_t)N, (uint64_t)D, BK, BN,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+        return e;
+    *stage = "proj_w8";
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(k_proj_w8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_TOTAL);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    const long tiles = (long)((T + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = (int)std::min<long>(tiles, sm_count());
+    void *pr = prof_start("proj_w8", st);
+    k_proj_w8<<<grid, NTHREADS, SMEM_TOTAL, st>>>(tm_x, tm_w, scale, T, D, Route{H * dk, H * dv, H, N}, q, k, v, a,
+                                                   b, err);
+    prof_stop(pr);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

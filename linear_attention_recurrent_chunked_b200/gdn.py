@@ -32,6 +32,7 @@ SIGNATURES = {
     "gdn_chunk_fwd_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
     "gdn_decode_step_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_chunk_fwd_check": (_I, [_VP, _SZ, _VP]),
+    "gdn_proj_w8": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gdn_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_seq_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
     "gdn_diag_mma_tile": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP]),
@@ -173,6 +174,29 @@ def decode_step_raw(q_raw, k_raw, v, a, b, S, o=None):
     _check(lib.gdn_decode_step_raw(_ptr(q_raw), _ptr(k_raw), _ptr(v), _ptr(a), _ptr(b), _ptr(S), B, H, dk, dv,
                                    _DTYPE.get(q_raw.dtype, 99), _ptr(o), _stream()))
     return o
+
+
+def proj_w8(x, w, scale, H: int, dk: int, dv: int, out=None, workspace=None, check: bool = False):
+    """Input projection with int8 weights (see include/gdn.h): x [T, D] bf16, w [N, D] int8,
+    scale [N] fp32, N = H (2 dk + dv) + 2 H. Returns (q_raw [T,H,dk], k_raw [T,H,dk], v [T,H,dv]
+    bf16, a [T,H], b [T,H] fp32); ``out`` may pass those five tensors to write into."""
+    lib = load_library()
+    _need_cuda(x, w, scale, workspace)
+    T, D = x.shape
+    dev = x.device
+    if out is None:
+        out = (torch.empty((T, H, dk), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, H, dk), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, H, dv), dtype=torch.bfloat16, device=dev),
+               torch.empty((T, H), dtype=torch.float32, device=dev),
+               torch.empty((T, H), dtype=torch.float32, device=dev))
+    _need_cuda(*out)
+    ws = workspace if workspace is not None else _workspace(256, dev)
+    _check(lib.gdn_proj_w8(_ptr(x), _ptr(w), _ptr(scale), T, D, H, dk, dv, *[_ptr(t) for t in out], _ptr(ws),
+                           ws.numel(), _stream()))
+    if check:
+        _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
+    return out
 
 
 def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = None, o=None, S_T=None):

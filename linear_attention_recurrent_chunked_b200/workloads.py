@@ -151,3 +151,17 @@ def make_decode(cfg: Decode = DECODE, seed: int = 0, steps: Optional[int] = None
     S = (0.02 * torch.randn((B, H, d, d), generator=gen, dtype=torch.float32)).contiguous()
     return dict(name=cfg.name, dtype=dtype, B=B, H=H, d=d, steps=steps,
                 q=q, k=k, v=v, g=g, beta=beta, S=S, **raw)
+
+
+def make_projection(T: int, D: int = 1024, H: int = 16, dk: int = 128, dv: int = 128, seed: int = 0):
+    """Inputs of the int8-weight input projection: hidden states x [T, D] ~ N(0, 1) in bf16, and a
+    weight matrix W [N, D] ~ N(0, 1/D) (N = H (2 dk + dv) + 2 H output channels) quantised
+    symmetrically per output channel to int8 codes w and fp32 scales (scale = max|W_n| / 127,
+    w = round(W / scale)). Draw order: x, then W. Returns CPU tensors x, w, scale and the sizes."""
+    gen = torch.Generator().manual_seed(seed)
+    N = H * (2 * dk + dv) + 2 * H
+    x = torch.randn((T, D), generator=gen, dtype=torch.float32).to(torch.bfloat16).contiguous()
+    W = torch.randn((N, D), generator=gen, dtype=torch.float32) / float(D) ** 0.5
+    scale = (W.abs().amax(dim=1) / 127.0).clamp_min(1e-12)
+    w = torch.round(W / scale[:, None]).clamp(-127, 127).to(torch.int8).contiguous()
+    return dict(x=x, w=w, scale=scale.contiguous(), T=T, D=D, H=H, dk=dk, dv=dv, N=N)
