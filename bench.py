@@ -644,7 +644,13 @@ def case_arm(args):
     dev = torch.device("cuda", 0)
     gdn.load_library()
     n = args.warmup + args.steps
-    if args.case == "decode":
+    if args.case.startswith("proj_"):  # proj_<T>: the int8-weight input projection for T tokens
+        from linear_attention_recurrent_chunked_b200.workloads import make_projection
+        p = make_projection(int(args.case[5:]), seed=0)
+        x, w, sc = p["x"].to(dev), p["w"].to(dev), p["scale"].to(dev)
+        for _ in range(n):
+            gdn.proj_w8(x, w, sc, p["H"], p["dk"], p["dv"])
+    elif args.case == "decode":
         w = make_decode(seed=0)
         t = {k: w[k].to(dev) for k in ("q", "k", "v", "g", "beta", "S")}
         for i in range(n):
@@ -671,7 +677,7 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="main workload only (no 10k/varlen/decode/scan extras)")
     ap.add_argument("--case", default=None,
                     help="profiling mode: run only WARMUP+STEPS calls of one workload (prefill_2k, prefill_10k, "
-                         "varlen, tiny, decode, scan_2k) and print nothing but a one-line summary")
+                         "varlen, tiny, decode, scan_2k, proj_<T>) and print nothing but a one-line summary")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -143,15 +143,16 @@ __device__ __noinline__ bool wait_flag(const uint32_t *p, Ctl *ctl, uint32_t *er
 __device__ __forceinline__ uint32_t lane_base(uint32_t tm, int warp) { return tm + ((uint32_t)((warp & 3) * 32) << 16); }
 
 // Scale the 64 rows of a 128-byte-swizzled 64 x 128 bf16 tile (two 8 KB column
-// halves) by f[row], in place, with n threads (t = 0..n-1). The swizzle only
-// permutes 16-byte chunks within a row, so a chunk's row is its offset within
-// the half / 128.
-__device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, int t, int n) {
+// halves) by f[row] (times f2[row] if f2 is given), in place, with n threads
+// (t = 0..n-1). The swizzle only permutes 16-byte chunks within a row, so a
+// chunk's row is its offset within the half / 128.
+__device__ __forceinline__ void scale_rows_sw128(uint8_t *tile, const float *f, int t, int n,
+                                                 const float *f2 = nullptr) {
     for (int idx = t; idx < 1024; idx += n) {
         const int row = (idx & 511) >> 3;
         uint4 *p = reinterpret_cast<uint4 *>(tile + 16 * idx);
         uint4 x = *p;
-        const float s = f[row];
+        const float s = f2 ? f[row] * f2[row] : f[row];
         uint32_t *w = reinterpret_cast<uint32_t *>(&x);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -216,8 +217,10 @@ __device__ __forceinline__ void row_inv_norms_sw128(const uint8_t *tile, float *
     if (qd == 0) rn[r] = inv_norm(ss);
 }
 
-// T1 = T2 diag(gamma) between two 64 x 64 bf16 tiles (rows r, runs along s; sy = 1024), n threads.
-__device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t, int n) {
+// T1 = T2 diag(gamma) (times diag(rn) if rn is given: raw inputs, 1 / ||k_s||) between two 64 x 64
+// bf16 tiles (rows r, runs along s; sy = 1024), n threads.
+__device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const float *gam, int t, int n,
+                                        const float *rn = nullptr) {
     for (int idx = t; idx < 512; idx += n) {
         const int s0 = 8 * (idx >> 6);
         uint4 x = *reinterpret_cast<const uint4 *>(t2 + 16 * idx);
@@ -225,7 +228,12 @@ __device__ __forceinline__ void make_t1(uint8_t *t1, const uint8_t *t2, const fl
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&w[j]));
-            w[j] = tc::pack_bf16x2(a.x * gam[s0 + 2 * j], a.y * gam[s0 + 2 * j + 1]);
+            float g0 = gam[s0 + 2 * j], g1 = gam[s0 + 2 * j + 1];
+            if (rn) {
+                g0 *= rn[s0 + 2 * j];
+                g1 *= rn[s0 + 2 * j + 1];
+            }
+            w[j] = tc::pack_bf16x2(a.x * g0, a.y * g1);
         }
         *reinterpret_cast<uint4 *>(t1 + 16 * idx) = x;
     }
@@ -868,14 +876,12 @@ __global__ void __launch_bounds__(NT_WS, 1)
         for (int c = 0; ok && c < nch; ++c) {
             const int b = c & 1;
             // T1 = T2 diag(gamma) (the previous chunk's W^T, U^T have read T1: WUF was waited below).
-            // Raw inputs: first normalise K (1 / ||k|| from the record) and Q in place; no MMA reads
-            // this buffer's K or Q before T1R.
+            // Raw inputs: first normalise Q in place; no MMA reads this buffer's Q before T1R.
             if (!(ok = wait_bar(&bar[FULL + b], full_par(c), ctl, err))) break;
-            if (raw) {
-                scale_rows_sw128(smem + b * BUF + B_K, vecp(c) + 192, t256, 256);
-                normalise_rows_sw128(smem + b * BUF + B_Q, t256);
-            }
-            make_t1(smem + T1, smem + b * BUF + B_T2, vecp(c) + 64, t256, 256);
+            // (raw inputs: the keys' 1 / ||k|| is folded into T1 here, into P's columns and into
+            // diag(e) K below; Q is normalised in place since both of its products read it)
+            if (raw) normalise_rows_sw128(smem + b * BUF + B_Q, t256);
+            make_t1(smem + T1, smem + b * BUF + B_T2, vecp(c) + 64, t256, 256, raw ? vecp(c) + 192 : nullptr);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
             // -W from W^T (all earlier readers of the W tile are covered by WUF: W^T, U^T come after them)
@@ -892,13 +898,17 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 const float Gr = vec[r];
                 float x[32];
                 tc::tmem_ld32(tl + TM_X1 + s0, x);
+                if (raw)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] *= vec[192 + s0 + i];  // raw keys: 1 / ||k_s||
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - vec[s0 + i]) * x[i] : 0.f;
 #pragma unroll
                 for (int i = 0; i < 32; i += 8) st_run8(sb + P + b * 8192 + tc::tile_off(r, s0 + i, 128, 1024), x + i);
             }
             tc::fence_before_sync();
-            scale_rows_sw128(smem + b * BUF + B_K, vec + 128, t256, 256);  // X1 and W^T, U^T have read K
+            scale_rows_sw128(smem + b * BUF + B_K, vec + 128, t256, 256,
+                             raw ? vec + 192 : nullptr);  // X1 and W^T, U^T have read K
             handoff(&bar[PR]);
         }
     } else {
@@ -1274,9 +1284,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
                        wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err)))
                 break;
-            // raw inputs: normalise K in place (1 / ||k|| from the record) before W^T reads it (T1R)
-            if (raw) scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 192, t128, 128);
-            make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128);
+            // (raw inputs: the keys' 1 / ||k|| from the record is folded into T1 and diag(e) K)
+            make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128, raw ? vecp(c) + 192 : nullptr);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
             // -W from W^T, once both chains' products have read the previous -W (other issuers)
@@ -1288,7 +1297,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             tile32_epilogue(sb + W, tl + TM_WT, k, 0, -1.f);
             tile32_epilogue(sb + W, tl + TM_WT + 32, k, 32, -1.f);
             handoff(&bar[WR]);
-            scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 128, t128, 128);  // W^T has read K
+            scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 128, t128, 128,
+                             raw ? vecp(c) + 192 : nullptr);  // W^T has read K
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[KR + (c & 3)]);
         }

@@ -14,11 +14,13 @@
 // product runs on bf16 operands with fp32 accumulation and the scale is applied to the fp32
 // result: the dequantisation is exact and the weights cross HBM as int8 (half the bytes of bf16).
 //
-// One persistent CTA per SM walks output tiles of 128 tokens x 256 channels (K steps of 64):
+// One persistent CTA per SM walks output tiles of 128 tokens x BN channels (BN = 256, or 128 / 64
+// when there are too few tiles to fill the GPU, as for one decode step), K steps of 64:
 //   loader    (1 thread)   TMA: x tile (bf16, 128-byte swizzle) and int8 weight tile, 4-deep ring
-//   convert   (4 warps)    int8 tile -> bf16 K-major 128-byte-swizzled operand tile, 2-deep ring
-//   MMA       (1 thread)   4 tcgen05.mma (M=128, N=256, K=16) per K step into a TMEM accumulator
-//                          (two accumulators of 256 columns: one tile's epilogue overlaps the next)
+//   convert   (8 warps)    int8 tile -> bf16 K-major 128-byte-swizzled operand tile, 3-deep ring
+//                          (exact, on integer and fp32 pipes: codes_to_bf16x4)
+//   MMA       (1 thread)   4 tcgen05.mma (M=128, N=BN, K=16) per K step into a TMEM accumulator
+//                          (two accumulators of BN columns: one tile's epilogue overlaps the next)
 //   epilogue  (4 warps)    TMEM -> fp32 registers -> * scale -> bf16 / fp32 rows in global memory
 // Every wait is bounded in time; a timeout sets the error word and all roles leave their loops.
 #include <cuda.h>
@@ -35,34 +37,36 @@ namespace gdn {
 namespace {
 
 using bf16_t = __nv_bfloat16;
-constexpr int BM = 128, BN = 256, BK = 64;
-constexpr int NSTAGE = 4, NBSLOT = 2;
+constexpr int BM = 128, BK = 64;
+constexpr int NSTAGE = 4, NBSLOT = 3;
 constexpr uint64_t kWaitNs = 1000000000ull;
-constexpr uint32_t A_BYTES = BM * BK * 2;   // 16 KB bf16 x tile
-constexpr uint32_t W8_BYTES = BN * BK;      // 16 KB int8 weight tile
-constexpr uint32_t B_BYTES = BN * BK * 2;   // 32 KB bf16 weight tile
-constexpr uint32_t OFF_A = 0;
-constexpr uint32_t OFF_W8 = OFF_A + NSTAGE * A_BYTES;
-constexpr uint32_t OFF_B = OFF_W8 + NSTAGE * W8_BYTES;
-constexpr uint32_t OFF_BAR = OFF_B + NBSLOT * B_BYTES;
+constexpr int NCONV = 256;                       // converter threads (8 warps)
+constexpr int NTHREADS = 64 + NCONV + 128;       // loader, MMA, converters, epilogue (14 warps)
+constexpr int W_LOAD = 0, W_MMA = 1, W_CONV0 = 2, W_EPI0 = 2 + NCONV / 32;
 enum {
-    FULL = 0,                    // [4] x and w8 of a stage landed (loader arrive + bytes)
-    EMPTY = FULL + NSTAGE,       // [4] stage free: MMA commit (x read) + converters (w8 read)
-    BFULL = EMPTY + NSTAGE,      // [2] bf16 weight tile written (128 converter threads)
-    BEMPTY = BFULL + NBSLOT,     // [2] bf16 weight tile read by the MMAs (commit)
+    FULL = 0,                    // [NSTAGE] x and w8 of a stage landed (loader arrive + bytes)
+    EMPTY = FULL + NSTAGE,       // [NSTAGE] stage free: MMA commit (x read) + every converter (w8 read)
+    BFULL = EMPTY + NSTAGE,      // [NBSLOT] bf16 weight tile written (every converter)
+    BEMPTY = BFULL + NBSLOT,     // [NBSLOT] bf16 weight tile read by the MMAs (commit)
     AFULL = BEMPTY + NBSLOT,     // [2] accumulator complete (commit)
     AEMPTY = AFULL + 2,          // [2] accumulator read out (128 epilogue threads)
     FIN = AEMPTY + 2,            // every MMA of the CTA done (drained before TMEM is freed)
     NBAR = FIN + 1
 };
-constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
-constexpr uint32_t SMEM_TOTAL = OFF_CTL + 16 + 1024;  // + alignment slack
-constexpr int NTHREADS = 320;                           // 10 warps
-constexpr int W_LOAD = 0, W_MMA = 1;                    // converters: warps 2-5; epilogue: warps 6-9
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-    return (i >= EMPTY && i < EMPTY + NSTAGE) ? 129u : (i >= BFULL && i < BFULL + NBSLOT) ? 128u
+    return (i >= EMPTY && i < EMPTY + NSTAGE) ? 1u + NCONV : (i >= BFULL && i < BFULL + NBSLOT) ? (uint32_t)NCONV
            : (i >= AEMPTY && i < AEMPTY + 2) ? 128u : 1u;
 }
+
+// Shared-memory layout for a channel tile of BN (x: 128 x 64 bf16; w8: BN x 64 int8; bf16 weight tile BN x 64).
+template <int BN>
+struct Lay {
+    static constexpr uint32_t A_BYTES = BM * BK * 2, W8_BYTES = BN * BK, B_BYTES = BN * BK * 2;
+    static constexpr uint32_t OFF_A = 0, OFF_W8 = OFF_A + NSTAGE * A_BYTES, OFF_B = OFF_W8 + NSTAGE * W8_BYTES;
+    static constexpr uint32_t OFF_BAR = OFF_B + NBSLOT * B_BYTES, OFF_CTL = OFF_BAR + 8 * NBAR;
+    static constexpr uint32_t TOTAL = OFF_CTL + 16 + 1024;  // + slack for the 1024-byte alignment
+};
+static_assert(Lay<256>::TOTAL <= 232448, "shared memory");
 
 struct Ctl {
     uint32_t tmem, abort;
@@ -97,23 +101,39 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint
         : "memory");
 }
 
+// Four int8 codes (one 32-bit word) as two bf16 pairs, exactly and on full-rate pipes: with
+// u = code + 128 (the word XOR 0x80808080), the fp32 with bit pattern 0x4B000000 | u is 2^23 + u,
+// and subtracting 2^23 + 128 leaves the code exactly. A code needs at most 8 significant bits, so
+// its bf16 is exactly the upper 16 bits of that fp32: a byte permute packs two of them.
+__device__ __forceinline__ void codes_to_bf16x4(uint32_t word, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = word ^ 0x80808080u;
+    const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - 8388736.0f;
+    const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - 8388736.0f;
+    const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652)) - 8388736.0f;
+    const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653)) - 8388736.0f;
+    lo = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
+    hi = __byte_perm(__float_as_uint(f2), __float_as_uint(f3), 0x7632);
+}
+
 // Where output column n goes: region 0..4 = q, k, v (bf16 [T][width]), a, b (fp32 [T][H]).
 struct Route {
     int Hdk, Hdv, H, N;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_proj_w8(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
               const float *__restrict__ scale, int T, int D, Route rt, bf16_t *__restrict__ q, bf16_t *__restrict__ k,
               bf16_t *__restrict__ v, float *__restrict__ ga, float *__restrict__ gb, uint32_t *__restrict__ err) {
+    using L = Lay<BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);  // 1024-byte aligned for the swizzle
     const uint32_t sb = tc::smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-    Ctl *ctl = reinterpret_cast<Ctl *>(smem + OFF_CTL);
-    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
+    Ctl *ctl = reinterpret_cast<Ctl *>(smem + L::OFF_CTL);
+    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 2 * BN < 32 ? 32 : 2 * BN);
     if (tid == 32) {
         for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
         ctl->abort = 0;
@@ -136,20 +156,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const int s = it % NSTAGE;
                     if (it >= NSTAGE && !(ok = wait_bar(&bar[EMPTY + s], (uint32_t)(((it / NSTAGE) - 1) & 1), ctl, err)))
                         break;
-                    tc::mbar_arrive_expect_tx(&bar[FULL + s], A_BYTES + W8_BYTES);
-                    tma_load_2d(sb + OFF_A + s * A_BYTES, &tm_x, &bar[FULL + s], ks * BK, m0);
-                    tma_load_2d(sb + OFF_W8 + s * W8_BYTES, &tm_w, &bar[FULL + s], ks * BK, n0);
+                    tc::mbar_arrive_expect_tx(&bar[FULL + s], L::A_BYTES + L::W8_BYTES);
+                    tma_load_2d(sb + L::OFF_A + s * L::A_BYTES, &tm_x, &bar[FULL + s], ks * BK, m0);
+                    tma_load_2d(sb + L::OFF_W8 + s * L::W8_BYTES, &tm_w, &bar[FULL + s], ks * BK, n0);
                     issued = it + 1;
                 }
             }
-            for (int j = std::max(0, issued - NSTAGE); j < issued; ++j)
+            for (int j = issued > NSTAGE ? issued - NSTAGE : 0; j < issued; ++j)
                 drain_bar(&bar[FULL + j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
         }
     } else if (warp == W_MMA) {
         if (lane == 0) {
             const uint32_t idesc = tc::make_idesc_bf16(BM, BN, 0, 0);
-            const tc::Desc da = tc::split_desc(tc::make_desc_sw128(sb + OFF_A, 16, 1024));
-            const tc::Desc db = tc::split_desc(tc::make_desc_sw128(sb + OFF_B, 16, 1024));
+            const tc::Desc da = tc::split_desc(tc::make_desc_sw128(sb + L::OFF_A, 16, 1024));
+            const tc::Desc db = tc::split_desc(tc::make_desc_sw128(sb + L::OFF_B, 16, 1024));
             int it = 0, ti = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
@@ -164,8 +184,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tc::fence_after_sync();
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        tc::mma_bf16_off(tm + acc * BN, da, s * A_BYTES + kk * 32, db, bs * B_BYTES + kk * 32, idesc,
-                                         (ks > 0 || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16_off(tm + acc * BN, da, s * L::A_BYTES + kk * 32, db, bs * L::B_BYTES + kk * 32,
+                                         idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                     tc::mma_commit(&bar[EMPTY + s]);
                     tc::mma_commit(&bar[BEMPTY + bs]);
                 }
@@ -174,9 +194,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc::mma_commit(&bar[FIN]);
             drain_bar(&bar[FIN], 0);
         }
-    } else if (warp < 6) {
-        // ---------------------------------------------------------------- convert (128 threads)
-        const int t = tid - 64;
+    } else if (warp < W_EPI0) {
+        // ---------------------------------------------------------------- convert (NCONV threads)
+        const int t = tid - 32 * W_CONV0;
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
@@ -186,22 +206,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                      (it < NBSLOT || wait_bar(&bar[BEMPTY + bs], (uint32_t)(((it / NBSLOT) - 1) & 1), ctl, err));
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
                 tc::fence_after_sync();
-                const uint8_t *w8 = smem + OFF_W8 + s * W8_BYTES;
-                uint8_t *bt = smem + OFF_B + bs * B_BYTES;
+                const uint8_t *w8 = smem + L::OFF_W8 + s * L::W8_BYTES;
+                uint8_t *bt = smem + L::OFF_B + bs * L::B_BYTES;
                 // 16-byte chunk c of the int8 tile (row c / 4, codes 16 (c % 4) ..): consecutive threads read
                 // consecutive chunks; each becomes two 16-byte bf16 chunks of the row's swizzled 128 bytes
-#pragma unroll 2
-                for (int c = t; c < BN * BK / 16; c += 128) {
+#pragma unroll
+                for (int c = t; c < BN * BK / 16; c += NCONV) {
                     const int row = c >> 2, q4 = c & 3;
                     const uint4 raw = *reinterpret_cast<const uint4 *>(w8 + 16 * c);
-                    const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
                     uint32_t o[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int32_t x = (int32_t)wd[j];
-                        o[2 * j] = tc::pack_bf16x2((float)(int8_t)(x & 0xff), (float)(int8_t)((x >> 8) & 0xff));
-                        o[2 * j + 1] = tc::pack_bf16x2((float)(int8_t)((x >> 16) & 0xff), (float)(int8_t)(x >> 24));
-                    }
+                    codes_to_bf16x4(raw.x, o[0], o[1]);
+                    codes_to_bf16x4(raw.y, o[2], o[3]);
+                    codes_to_bf16x4(raw.z, o[4], o[5]);
+                    codes_to_bf16x4(raw.w, o[6], o[7]);
                     const uint32_t rbase = (uint32_t)row * 128u, sw = (uint32_t)(row & 7);
                     *reinterpret_cast<uint4 *>(bt + rbase + (((2u * q4) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                     *reinterpret_cast<uint4 *>(bt + rbase + (((2u * q4 + 1u) ^ sw) << 4)) =
@@ -271,7 +288,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tm, 512);
+    if (warp == 0) tc::tmem_dealloc(tm, 2 * BN < 32 ? 32 : 2 * BN);
 }
 
 }  // namespace
@@ -325,27 +342,40 @@ cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float 
     if ((e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
     const int N = H * (2 * dk + dv) + 2 * H;
     if (T == 0) return cudaSuccess;
-    CUtensorMap tm_x, tm_w;
+    CUtensorMap tm_x;
     *stage = "TMA descriptor encoding";
     if ((e = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, BK, BM,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
         return e;
-    if ((e = encode_2d(&tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)D, (uint64_t)N, (uint64_t)D, BK, BN,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
-        return e;
     *stage = "proj_w8";
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(k_proj_w8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_TOTAL);
-    });
-    if (attr_err != cudaSuccess) return attr_err;
-    const long tiles = (long)((T + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int grid = (int)std::min<long>(tiles, sm_count());
-    void *pr = prof_start("proj_w8", st);
-    k_proj_w8<<<grid, NTHREADS, SMEM_TOTAL, st>>>(tm_x, tm_w, scale, T, D, Route{H * dk, H * dv, H, N}, q, k, v, a,
-                                                   b, err);
-    prof_stop(pr);
+    // Channel tile: the widest of 256 / 128 / 64 that still gives every SM a tile (small T, e.g.
+    // one decode step, is bound by reading the weights and needs many CTAs to do so).
+    const long mt = (T + BM - 1) / BM;
+    int bn = 64;
+    for (int cand : {256, 128})
+        if (mt * ((N + cand - 1) / cand) >= sm_count()) {
+            bn = cand;
+            break;
+        }
+    auto launch = [&](auto kernel, int BNv, uint32_t smem_bytes) -> cudaError_t {
+        cudaError_t ea = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+        if (ea != cudaSuccess) return ea;
+        CUtensorMap tm_w2;
+        ea = encode_2d(&tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)D, (uint64_t)N, (uint64_t)D, BK, BNv,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (ea != cudaSuccess) return ea;
+        const long tiles = mt * ((N + BNv - 1) / BNv);
+        const int grid = (int)std::min<long>(tiles, sm_count());
+        void *pr = prof_start("proj_w8", st);
+        kernel<<<grid, NTHREADS, smem_bytes, st>>>(tm_x, tm_w2, scale, T, D, Route{H * dk, H * dv, H, N}, q, k, v,
+                                                    a, b, err);
+        prof_stop(pr);
+        return cudaSuccess;
+    };
+    if (bn == 256) e = launch(k_proj_w8<256>, 256, Lay<256>::TOTAL);
+    else if (bn == 128) e = launch(k_proj_w8<128>, 128, Lay<128>::TOTAL);
+    else e = launch(k_proj_w8<64>, 64, Lay<64>::TOTAL);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
