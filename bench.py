@@ -389,6 +389,7 @@ def gpu_arm(args):
             result[name]["chunked_over_sequential"] = statistics.mean(ts) / result[name]["ms_per_step"]
         result["decode"] = decode_entry(args, torch, gdn, dev, dist, pk, make_decode)
         result["projection"] = projection_entry(args, torch, gdn, dev, dist, pk, time_steps)
+        result["attention"] = attention_entry(args, torch, gdn, dev, dist, pk, time_steps)
 
     # ---------------- JSON line
     main = result["prefill_2k"]
@@ -457,6 +458,28 @@ def projection_entry(args, torch, gdn, dev, dist, pk, time_steps):
             entry["roofline"] = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                                  "frac": gbs / pk["hbm"], "peak_source": pk["src"]}
         out["T%d" % T] = entry
+    return out
+
+
+def attention_entry(args, torch, gdn, dev, dist, pk, time_steps):
+    """The hybrid's causal attention layer (H = 16 heads of d = 128, bf16) at 2k and 10k tokens:
+    device time per call with L2 flushed, and the causal flop count 4 d T (T + 1) / 2 per head
+    (Q K^T and P V over the pairs j <= t) against the measured dense bf16 peak."""
+    from linear_attention_recurrent_chunked_b200.workloads import make_attention
+    out = {}
+    for T in (2048, 10240):
+        w = make_attention([T], H=16, seed=0)
+        q, k, v = w["q"].to(dev), w["k"].to(dev), w["v"].to(dev)
+        o = torch.empty_like(q)
+        fn = lambda: gdn.attn_fwd(q, k, v, None, N=1, o=o)
+        ms = max_over_ranks(dist, statistics.mean(time_steps(fn, max(5, args.steps // 2), args.warmup)), dev)
+        gdn.attn_fwd(q, k, v, None, N=1, o=o, check=True)
+        flops = 4.0 * w["d"] * T * (T + 1) / 2 * w["H"]
+        tflops = flops / (ms * 1e-3) / 1e12
+        out["T%d" % T] = {"T": T, "H": w["H"], "d": w["d"], "ms": ms, "tokens_per_s": T / (ms * 1e-3),
+                          "algorithmic_flops": flops,
+                          "roofline": {"bound": "tensor", "achieved": tflops, "peak": pk["bf16"], "unit": "TFLOP/s",
+                                       "frac": tflops / pk["bf16"], "peak_source": pk["src"]}}
     return out
 
 
@@ -644,7 +667,13 @@ def case_arm(args):
     dev = torch.device("cuda", 0)
     gdn.load_library()
     n = args.warmup + args.steps
-    if args.case.startswith("proj_"):  # proj_<T>: the int8-weight input projection for T tokens
+    if args.case.startswith("attn_"):  # attn_<T>: causal attention over one sequence of T tokens, 16 heads
+        from linear_attention_recurrent_chunked_b200.workloads import make_attention
+        w = make_attention([int(args.case[5:])], H=16, seed=0)
+        q, k, v = w["q"].to(dev), w["k"].to(dev), w["v"].to(dev)
+        for _ in range(n):
+            gdn.attn_fwd(q, k, v, None, N=1)
+    elif args.case.startswith("proj_"):  # proj_<T>: the int8-weight input projection for T tokens
         from linear_attention_recurrent_chunked_b200.workloads import make_projection
         p = make_projection(int(args.case[5:]), seed=0)
         x, w, sc = p["x"].to(dev), p["w"].to(dev), p["scale"].to(dev)

@@ -235,6 +235,30 @@ gdn_status gdn_proj_w8(const void *x, const int8_t *w, const float *scale, int T
                        void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * Causal attention of the hybrid backbone's attention layers. The pages' backbone
+ * interleaves the recurrent layers with causal attention layers, whose O(N^2)
+ * kernel made long-context prefill collapse until it was rewritten as per-head
+ * GEMMs (page 1, abstract: 17x faster prefill at 10k tokens; page 2, "Resumen
+ * Tecnico", the attention rewrite). Per sequence, head h and position t:
+ *     o_t = sum_{j <= t} softmax_j(scale * q_t . k_j) v_j
+ * over the keys of the same sequence (standard scaled dot-product attention with
+ * a causal mask; the pages do not write it out). The scores never leave the
+ * chip: per query tile they live in tensor memory (see the implementation).
+ *   q, k, v, o [T_tot][H][d] bf16, d = 128 (o: output, bf16 rounded to nearest)
+ *   cu_seqlens [N+1] int32 on the device, or NULL for N equal sequences;
+ *     max_len bounds the sequences' lengths (ignored when cu_seqlens is NULL)
+ *   scale > 0, or <= 0 for 1 / sqrt(d)
+ *   workspace, ws_bytes: >= 256 bytes of device memory for the error word
+ *     (gdn_chunk_fwd_check reads it: GDN_ERR_SEQLENS for a malformed device
+ *     cu_seqlens, then nothing is written; GDN_ERR_TIMEOUT for a bounded wait
+ *     that gave up).
+ * Pointers 16-byte aligned. dtype must be GDN_BF16 (GDN_ERR_DTYPE otherwise).
+ */
+gdn_status gdn_attn_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int N,
+                        int T_tot, int H, int d, int max_len, float scale, gdn_dtype dtype, void *o,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * The sequential (token-by-token) scan on the GPU: the same result as
  * gdn_chunk_fwd, computed one token at a time with the decode step's row
  * update. It is the comparator for the chunked path's speed-up (page 1,

@@ -1,6 +1,7 @@
 // C ABI of the library (declared in include/gdn.h): argument validation,
 // error reporting and dispatch to the kernels. Host code only, apart from the
 // small cu_seqlens validation kernel.
+#include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -356,6 +357,34 @@ gdn_status gdn_proj_w8(const void *x, const int8_t *w, const float *scale, int T
         static_cast<const __nv_bfloat16 *>(x), w, scale, T, D, H, dk, dv, static_cast<__nv_bfloat16 *>(q_raw),
         static_cast<__nv_bfloat16 *>(k_raw), static_cast<__nv_bfloat16 *>(v), a, b, static_cast<uint32_t *>(workspace),
         static_cast<cudaStream_t>(stream), &stage);
+    if (e != cudaSuccess) return cuda_fail(e, stage);
+    return ok();
+}
+
+gdn_status gdn_attn_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens, int N, int T_tot,
+                        int H, int d, int max_len, float scale, gdn_dtype dtype, void *o, void *workspace,
+                        size_t ws_bytes, void *stream) {
+    if (dtype != GDN_BF16) return fail(GDN_ERR_DTYPE, "attention takes bf16 inputs only");
+    if (d != 128) return fail(GDN_ERR_SHAPE, "attention head size d=%d unsupported (128)", d);
+    if (N < 1 || H < 1 || T_tot < 0) return fail(GDN_ERR_SHAPE, "N=%d H=%d T=%d out of range", N, H, T_tot);
+    if (!cu_seqlens && T_tot % N != 0)
+        return fail(GDN_ERR_SEQLENS, "cu_seqlens is NULL and T_tot=%d is not a multiple of N=%d", T_tot, N);
+    if (!cu_seqlens) max_len = T_tot / N;
+    if (max_len < 0 || max_len > T_tot) return fail(GDN_ERR_SHAPE, "max_len=%d outside 0 .. T_tot", max_len);
+    if ((double)T_tot * H * d >= 9.0e18 || (double)((max_len + 127) / 128) * H * N >= 2.0e9)
+        return fail(GDN_ERR_SHAPE, "sizes overflow");
+    if (T_tot > 0 && (!q || !k || !v || !o)) return fail(GDN_ERR_NULL, "q, k, v and o are required");
+    const void *ptrs[] = {q, k, v, o, cu_seqlens};
+    for (const void *p : ptrs)
+        if (misaligned(p)) return fail(GDN_ERR_ALIGN, "pointer %p is not 16-byte aligned", p);
+    if (!workspace || ws_bytes < kErrWordBytes)
+        return fail(GDN_ERR_WORKSPACE, "workspace of at least %zu bytes (the error word) needed", kErrWordBytes);
+    if (!(scale > 0.f)) scale = 1.f / sqrtf((float)d);
+    const char *stage = "";
+    const cudaError_t e = gdn::launch_attn_fwd(
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k),
+        static_cast<const __nv_bfloat16 *>(v), cu_seqlens, N, T_tot, H, max_len, scale,
+        static_cast<__nv_bfloat16 *>(o), static_cast<uint32_t *>(workspace), static_cast<cudaStream_t>(stream), &stage);
     if (e != cudaSuccess) return cuda_fail(e, stage);
     return ok();
 }

@@ -54,6 +54,13 @@ cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float 
                            int dv, __nv_bfloat16 *q, __nv_bfloat16 *k, __nv_bfloat16 *v, float *a, float *b,
                            uint32_t *err, cudaStream_t st, const char **stage);
 
+// Causal attention (bf16, d = 128) over packed sequences: o_t = softmax_j<=t(scale q_t . k_j) v_j per
+// head; q, k, v, o [T_tot][H][128]; cu (device, N+1 offsets) or NULL (N equal sequences);
+// max_len = the longest sequence's length (bounds the grid); err = error word.
+cudaError_t launch_attn_fwd(const __nv_bfloat16 *q, const __nv_bfloat16 *k, const __nv_bfloat16 *v,
+                            const int32_t *cu, int N, int T_tot, int H, int max_len, float scale, __nv_bfloat16 *o,
+                            uint32_t *err, cudaStream_t st, const char **stage);
+
 // Failure injection for tests (set by gdn_debug_inject; off by default): the pipelined path's
 // first segment of head 0 withholds its end-state flag, and waits for flags give up after
 // flag_wait_ns (0 = the normal bound) instead of hanging.

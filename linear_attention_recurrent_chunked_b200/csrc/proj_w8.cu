@@ -16,7 +16,8 @@
 //
 // One persistent CTA per SM walks output tiles of 128 tokens x BN channels (BN = 256, or 128 / 64
 // when there are too few tiles to fill the GPU, as for one decode step), K steps of 64:
-//   loader    (1 thread)   TMA: x tile (bf16, 128-byte swizzle) and int8 weight tile, 4-deep ring
+//   loaders   (2 threads)  TMA: x tiles (bf16, 128-byte swizzle) and int8 weight tiles, two 4-deep
+//                          rings, freed by the MMAs and by the converters respectively
 //   convert   (8 warps)    int8 tile -> bf16 K-major 128-byte-swizzled operand tile, 3-deep ring
 //                          (exact, on integer and fp32 pipes: codes_to_bf16x4)
 //   MMA       (1 thread)   4 tcgen05.mma (M=128, N=BN, K=16) per K step into a TMEM accumulator
@@ -41,12 +42,14 @@ constexpr int BM = 128, BK = 64;
 constexpr int NSTAGE = 4, NBSLOT = 3;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int NCONV = 256;                       // converter threads (8 warps)
-constexpr int NTHREADS = 64 + NCONV + 128;       // loader, MMA, converters, epilogue (14 warps)
-constexpr int W_LOAD = 0, W_MMA = 1, W_CONV0 = 2, W_EPI0 = 2 + NCONV / 32;
+constexpr int NTHREADS = 96 + NCONV + 128;       // x loader, MMA, w8 loader, converters, epilogue (15 warps)
+constexpr int W_LOAD = 0, W_MMA = 1, W_LOADW = 2, W_CONV0 = 3, W_EPI0 = 3 + NCONV / 32;
 enum {
-    FULL = 0,                    // [NSTAGE] x and w8 of a stage landed (loader arrive + bytes)
-    EMPTY = FULL + NSTAGE,       // [NSTAGE] stage free: MMA commit (x read) + every converter (w8 read)
-    BFULL = EMPTY + NSTAGE,      // [NBSLOT] bf16 weight tile written (every converter)
+    FULL = 0,                    // [NSTAGE] x tile of a stage landed (x loader arrive + bytes)
+    EMPTY = FULL + NSTAGE,       // [NSTAGE] x stage free (MMA commit)
+    WFULL = EMPTY + NSTAGE,      // [NSTAGE] int8 weight tile landed (w8 loader arrive + bytes)
+    WEMPTY = WFULL + NSTAGE,     // [NSTAGE] int8 stage free (every converter)
+    BFULL = WEMPTY + NSTAGE,     // [NBSLOT] bf16 weight tile written (every converter)
     BEMPTY = BFULL + NBSLOT,     // [NBSLOT] bf16 weight tile read by the MMAs (commit)
     AFULL = BEMPTY + NBSLOT,     // [2] accumulator complete (commit)
     AEMPTY = AFULL + 2,          // [2] accumulator read out (128 epilogue threads)
@@ -54,7 +57,7 @@ enum {
     NBAR = FIN + 1
 };
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-    return (i >= EMPTY && i < EMPTY + NSTAGE) ? 1u + NCONV : (i >= BFULL && i < BFULL + NBSLOT) ? (uint32_t)NCONV
+    return (i >= WEMPTY && i < WEMPTY + NSTAGE) ? (uint32_t)NCONV : (i >= BFULL && i < BFULL + NBSLOT) ? (uint32_t)NCONV
            : (i >= AEMPTY && i < AEMPTY + 2) ? 128u : 1u;
 }
 
@@ -146,24 +149,32 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int mt = (T + BM - 1) / BM, nt = (rt.N + BN - 1) / BN, ksteps = D / BK;
     const int ntiles = mt * nt;
 
-    if (warp == W_LOAD) {
+    if (warp == W_LOAD || warp == W_LOADW) {
+        // two loader threads: the x ring is freed by the MMAs, the int8 ring by the converters, so the
+        // weight tiles (and their conversion) can run ahead of the products
         if (lane == 0) {
+            const bool wl = warp == W_LOADW;
+            uint64_t *full = &bar[wl ? WFULL : FULL], *empty = &bar[wl ? WEMPTY : EMPTY];
             int it = 0, issued = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
                 const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
                 for (int ks = 0; ks < ksteps; ++ks, ++it) {
                     const int s = it % NSTAGE;
-                    if (it >= NSTAGE && !(ok = wait_bar(&bar[EMPTY + s], (uint32_t)(((it / NSTAGE) - 1) & 1), ctl, err)))
+                    if (it >= NSTAGE && !(ok = wait_bar(&empty[s], (uint32_t)(((it / NSTAGE) - 1) & 1), ctl, err)))
                         break;
-                    tc::mbar_arrive_expect_tx(&bar[FULL + s], L::A_BYTES + L::W8_BYTES);
-                    tma_load_2d(sb + L::OFF_A + s * L::A_BYTES, &tm_x, &bar[FULL + s], ks * BK, m0);
-                    tma_load_2d(sb + L::OFF_W8 + s * L::W8_BYTES, &tm_w, &bar[FULL + s], ks * BK, n0);
+                    if (wl) {
+                        tc::mbar_arrive_expect_tx(&full[s], L::W8_BYTES);
+                        tma_load_2d(sb + L::OFF_W8 + s * L::W8_BYTES, &tm_w, &full[s], ks * BK, n0);
+                    } else {
+                        tc::mbar_arrive_expect_tx(&full[s], L::A_BYTES);
+                        tma_load_2d(sb + L::OFF_A + s * L::A_BYTES, &tm_x, &full[s], ks * BK, m0);
+                    }
                     issued = it + 1;
                 }
             }
             for (int j = issued > NSTAGE ? issued - NSTAGE : 0; j < issued; ++j)
-                drain_bar(&bar[FULL + j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
+                drain_bar(&full[j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
         }
     } else if (warp == W_MMA) {
         if (lane == 0) {
@@ -202,7 +213,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
             for (int ks = 0; ks < ksteps; ++ks, ++it) {
                 const int s = it % NSTAGE, bs = it % NBSLOT;
-                ok = wait_bar(&bar[FULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
+                ok = wait_bar(&bar[WFULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
                      (it < NBSLOT || wait_bar(&bar[BEMPTY + bs], (uint32_t)(((it / NBSLOT) - 1) & 1), ctl, err));
                 if (!(ok = __all_sync(0xffffffffu, ok))) break;
                 tc::fence_after_sync();
@@ -226,7 +237,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 tc::fence_smem_to_async();
                 tc::mbar_arrive(&bar[BFULL + bs]);
-                tc::mbar_arrive(&bar[EMPTY + s]);  // this thread's reads of the int8 stage are done
+                tc::mbar_arrive(&bar[WEMPTY + s]);  // this thread's reads of the int8 stage are done
             }
         }
     } else {

@@ -124,6 +124,18 @@ __device__ __forceinline__ void mma_bf16_off(uint32_t d_tmem, Desc a, uint32_t a
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B^T with B given as base descriptor + byte offset (A layout as mma_bf16_ts).
+__device__ __forceinline__ void mma_bf16_ts_off(uint32_t d_tmem, uint32_t a_tmem, Desc b, uint32_t b_off,
+                                                uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on the mbarrier when all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))

@@ -32,6 +32,7 @@ SIGNATURES = {
     "gdn_chunk_fwd_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP, _SZ, _VP]),
     "gdn_decode_step_raw": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_chunk_fwd_check": (_I, [_VP, _SZ, _VP]),
+    "gdn_attn_fwd": (_I, [_VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, ctypes.c_float, _I, _VP, _VP, _SZ, _VP]),
     "gdn_proj_w8": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "gdn_decode_step": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _VP, _VP]),
     "gdn_seq_scan": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _VP, _VP, _VP]),
@@ -197,6 +198,31 @@ def proj_w8(x, w, scale, H: int, dk: int, dv: int, out=None, workspace=None, che
     if check:
         _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
     return out
+
+
+def attn_fwd(q, k, v, cu_seqlens=None, N: Optional[int] = None, max_len: Optional[int] = None,
+             scale: float = 0.0, o=None, workspace=None, check: bool = False):
+    """Causal attention (see include/gdn.h): q, k, v [T, H, 128] bf16; cu_seqlens [N+1] int32
+    (device) or None (N equal sequences, N from ``N``, else 1); max_len bounds the sequence
+    lengths (required with cu_seqlens); scale <= 0 means 1 / sqrt(128). Returns o [T, H, 128]."""
+    lib = load_library()
+    _need_cuda(q, k, v, cu_seqlens, o, workspace)
+    T_tot, H, d = q.shape
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+        if max_len is None:
+            raise GdnError(2, "max_len is required with cu_seqlens")
+    else:
+        N = 1 if N is None else N
+        max_len = T_tot // N
+    if o is None:
+        o = torch.empty_like(q)
+    ws = workspace if workspace is not None else _workspace(256, q.device)
+    _check(lib.gdn_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), N, T_tot, H, d, max_len, float(scale),
+                            _DTYPE.get(q.dtype, 99), _ptr(o), _ptr(ws), ws.numel(), _stream()))
+    if check:
+        _check(lib.gdn_chunk_fwd_check(_ptr(ws), ws.numel(), _stream()))
+    return o
 
 
 def chunk_fwd_noalloc(q, k, v, g, beta, S0=None, cu_seqlens=None, N: Optional[int] = None, o=None, S_T=None):

@@ -165,3 +165,16 @@ def make_projection(T: int, D: int = 1024, H: int = 16, dk: int = 128, dv: int =
     scale = (W.abs().amax(dim=1) / 127.0).clamp_min(1e-12)
     w = torch.round(W / scale[:, None]).clamp(-127, 127).to(torch.int8).contiguous()
     return dict(x=x, w=w, scale=scale.contiguous(), T=T, D=D, H=H, dk=dk, dv=dv, N=N)
+
+
+def make_attention(seqlens: List[int], H: int = 16, d: int = 128, seed: int = 0):
+    """Inputs of the causal attention layer over packed sequences: q, k, v [T, H, d] ~ N(0, 1) in
+    bf16 (draw order q, k, v), cu_seqlens [N+1] int32, and the sizes."""
+    gen = torch.Generator().manual_seed(seed)
+    T = int(sum(seqlens))
+    q, k, v = (torch.randn((T, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16).contiguous()
+               for _ in range(3))
+    cu = torch.zeros(len(seqlens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(seqlens, dtype=torch.int64), 0).to(torch.int32)
+    return dict(q=q, k=k, v=v, cu_seqlens=cu, seqlens=[int(x) for x in seqlens], T=T, H=H, d=d,
+                N=len(seqlens), max_len=max(seqlens) if seqlens else 0)
