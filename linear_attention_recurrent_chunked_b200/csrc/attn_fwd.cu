@@ -225,13 +225,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     s[64 + i] = c[i];
                 }
             }
-            const int kbase = j * TK;  // key position of column 0 within the sequence
-            float mt = -INFINITY;
+            // row maximum of the raw scores (the causal mask only cuts the diagonal key tile), in eight
+            // independent partial maxima so that the reduction is not one 128-long dependent chain
+            float pm[8];
 #pragma unroll
-            for (int i = 0; i < 128; ++i) {
-                s[i] = (kbase + i <= qpos) ? s[i] * sc : -INFINITY;
-                mt = fmaxf(mt, s[i]);
+            for (int u = 0; u < 8; ++u) pm[u] = -INFINITY;
+            if (j == qi) {
+                const int lim = qpos - j * TK;  // key columns beyond this row's position are masked
+#pragma unroll
+                for (int i = 0; i < 128; ++i) {
+                    s[i] = (i <= lim) ? s[i] : -INFINITY;
+                    pm[i & 7] = fmaxf(pm[i & 7], s[i]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 128; ++i) pm[i & 7] = fmaxf(pm[i & 7], s[i]);
             }
+            const float mt = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                   fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * sc;
             // lazy rescale: a new reference maximum only when this tile's exceeds it by more than kRescale
             float alpha = 1.f;
             const bool grow = mt > m_ref + kRescale;
@@ -254,20 +265,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tc::tmem_st32(tl + TM_O + c0, u);
                 }
             }
-            // P = 2^(s - m_ref) as bf16 pairs over the first 64 columns of the score buffer
-            float ls = 0.f;
+            // P = 2^(s sc - m_ref) (one FFMA and one MUFU.EX2 per score; masked scores give 0) as bf16 pairs
+            // over the first 64 columns of the score buffer; the row sum in eight partial sums
+            float ps[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < 128; c0 += 64) {
                 uint32_t u[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const float p0 = chunk::ex2(s[c0 + 2 * i] - m_ref), p1 = chunk::ex2(s[c0 + 2 * i + 1] - m_ref);
-                    ls += p0 + p1;
+                    const float p0 = chunk::ex2(fmaf(s[c0 + 2 * i], sc, -m_ref));
+                    const float p1 = chunk::ex2(fmaf(s[c0 + 2 * i + 1], sc, -m_ref));
+                    ps[i & 7] += p0 + p1;
                     u[i] = tc::pack_bf16x2(p0, p1);
                 }
                 tc::tmem_st32(tl + TM_S + b * 128 + c0 / 2, u);
             }
-            l += ls;
+            l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             tc::tmem_st_wait();
             tc::fence_before_sync();
             tc::mbar_arrive(&bar[PREADY + b]);
