@@ -13,8 +13,11 @@
 // One CTA per (query tile of 128 positions, head, sequence), the largest tiles dispatched
 // first; roles:
 //   loader   (1 thread)  TMA: the Q tile once, K and V tiles of 128 keys into 2-deep rings
-//   MMA      (1 thread)  S_j = Q K_j^T (M=128, N=128, K=128) into one of two TMEM score buffers,
-//                        two tiles ahead; O += P_j V_j (A = P_j in TMEM) once the softmax is done
+//   MMA      (1 warp)    S_j = Q K_j^T (M=128, N=128, K=128) into one of three TMEM score buffers,
+//                        two tiles ahead; O += P_j V_j (A = P_j in TMEM) once the softmax is done.
+//                        A product writing a buffer is issued only after the O += P V that read
+//                        the buffer's previous P has completed: a later tcgen05.mma is not ordered
+//                        after an earlier one's tensor-memory operand reads.
 //   softmax  (4 warps)   one query row per thread: scores * scale in log2 units, causal mask,
 //                        row max and sum, P = 2^(s - m) as bf16 pairs written over the score
 //                        buffer; O is rescaled (read, scaled, written back in TMEM) only when a
@@ -40,18 +43,20 @@ enum {
     VFULL = 3,    // [2]
     KEMPTY = 5,   // [2] S_j has read K_j (commit)
     VEMPTY = 7,   // [2] PV_j has read V_j (commit)
-    SFULL = 9,    // [2] S_j complete (commit)
-    PREADY = 11,  // [2] P_j written over its score buffer, O rescaled (128 softmax threads)
-    OV = 13,      // O += P_j V_j complete (commit; one phase per key tile)
-    FIN = 14,     // every MMA of the CTA done
-    NBAR = 15
+    SFULL = 9,    // [3] S_j complete (commit), per score buffer
+    PREADY = 12,  // [3] P_j written over its score buffer, O rescaled (128 softmax threads)
+    PVD = 15,     // [3] O += P_j V_j has read the buffer's P (commit)
+    OV = 18,      // O += P_j V_j complete (commit; one phase per key tile)
+    FIN = 19,     // every MMA of the CTA done
+    NBAR = 20
 };
 constexpr uint32_t OFF_CTL = OFF_BAR + 8 * NBAR;
 constexpr uint32_t SMEM_TOTAL = OFF_CTL + 16 + 1024;
 constexpr int NTHREADS = 192;  // loader warp, MMA warp, 4 softmax warps
 constexpr int W_LOAD = 0, W_MMA = 1;
-// TMEM columns: score buffers S0, S1 (P_j overwrites the first 64 columns of its buffer), O
-constexpr uint32_t TM_S = 0, TM_O = 256;
+// TMEM columns: score buffers S0, S1, S2 (tile j in buffer j % 3; P_j overwrites the first 64
+// columns of its buffer), O
+constexpr uint32_t TM_S = 0, TM_O = 384;
 
 struct Ctl {
     uint32_t tmem, abort;
@@ -71,6 +76,11 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, 
             }
         }
     }
+}
+// wait_bar for a warp that issues MMAs as a whole (tc::*_w): every lane waits (converged), so that
+// the warp stays converged for the elected issue.
+__device__ __forceinline__ bool wait_bar_w(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, ctl, err));
 }
 __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = tc::globaltimer();
@@ -120,7 +130,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + OFF_CTL);
     if (warp == 0) tc::tmem_alloc(&ctl->tmem, 512);
     if (tid == 32) {
-        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i == PREADY || i == PREADY + 1) ? 128u : 1u);
+        for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], (i >= PREADY && i < PREADY + 3) ? 128u : 1u);
         ctl->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -157,7 +167,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int j = issued_v > 2 ? issued_v - 2 : 0; j < issued_v; ++j) drain_bar(&bar[VFULL + (j & 1)], (j >> 1) & 1);
         }
     } else if (warp == W_MMA) {
-        if (lane == 0) {
+        {  // the whole warp, lane 0 issuing
             const uint32_t id_s = tc::make_idesc_bf16(TQ, TK, 0, 0);  // Q K^T: both K-major
             const uint32_t id_o = tc::make_idesc_bf16(TQ, D, 0, 1);   // P V: V MN-major
             const tc::Desc dq = tc::split_desc(tc::make_desc_sw128(sb + OFF_Q, 16, 1024));
@@ -168,38 +178,43 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                    tc::mma_bf16_off(tm + TM_S + (j & 1) * 128, dq, off, dk, kb + off, id_s, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_S + (j % 3) * 128, dq, off, dk, kb + off, id_s, kk > 0);
                 }
-                tc::mma_commit(&bar[SFULL + (j & 1)]);
-                tc::mma_commit(&bar[KEMPTY + (j & 1)]);
+                tc::mma_commit_w(&bar[SFULL + j % 3]);
+                tc::mma_commit_w(&bar[KEMPTY + (j & 1)]);
             };
-            bool ok = wait_bar(&bar[QFULL], 0, ctl, err);
+            bool ok = wait_bar_w(&bar[QFULL], 0, ctl, err);
             for (int j = 0; ok && j < 2 && j < nk; ++j) {
-                if (!(ok = wait_bar(&bar[KFULL + j], 0, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[KFULL + j], 0, ctl, err))) break;
                 tc::fence_after_sync();
                 issue_s(j);
             }
             for (int j = 0; ok && j < nk; ++j) {
-                const int b = j & 1;
-                if (!(ok = wait_bar(&bar[PREADY + b], (uint32_t)((j >> 1) & 1), ctl, err) &&
-                           wait_bar(&bar[VFULL + b], (uint32_t)((j >> 1) & 1), ctl, err)))
+                const int b = j & 1, b3 = j % 3;
+                if (!(ok = wait_bar_w(&bar[PREADY + b3], (uint32_t)((j / 3) & 1), ctl, err) &&
+                           wait_bar_w(&bar[VFULL + b], (uint32_t)((j >> 1) & 1), ctl, err)))
                     break;
                 tc::fence_after_sync();
                 // O += P_j V_j: A = P_j (bf16 pairs in the score buffer's first 64 columns), B = V_j (MN-major)
 #pragma unroll
                 for (int kk = 0; kk < TK / 16; ++kk)
-                    tc::mma_bf16_ts_off(tm + TM_O, tm + TM_S + b * 128 + 8 * kk, dv,
+                    tc::mma_bf16_ts_off_w(tm + TM_O, tm + TM_S + b3 * 128 + 8 * kk, dv,
                                         b * TILE + kk * 2048, id_o, (j > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&bar[OV]);
-                tc::mma_commit(&bar[VEMPTY + b]);
+                tc::mma_commit_w(&bar[OV]);
+                tc::mma_commit_w(&bar[VEMPTY + b]);
+                tc::mma_commit_w(&bar[PVD + b3]);
                 if (j + 2 < nk) {
-                    if (!(ok = wait_bar(&bar[KFULL + b], (uint32_t)(((j + 2) >> 1) & 1), ctl, err))) break;
+                    // S_{j+2} goes to buffer (j + 2) % 3, whose last P (tile j - 1) must have been read
+                    if (!(ok = wait_bar_w(&bar[KFULL + b], (uint32_t)(((j + 2) >> 1) & 1), ctl, err) &&
+                               (j == 0 || wait_bar_w(&bar[PVD + (j + 2) % 3], (uint32_t)(((j - 1) / 3) & 1), ctl, err))))
+                        break;
                     tc::fence_after_sync();
                     issue_s(j + 2);
                 }
             }
-            tc::mma_commit(&bar[FIN]);
-            drain_bar(&bar[FIN], 0);
+            tc::mma_commit_w(&bar[FIN]);
+            if (lane == 0) drain_bar(&bar[FIN], 0);
+            __syncwarp();
         }
     } else {
         // ---------------------------------------------------------------- softmax (one query row per thread)
@@ -210,8 +225,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float m_ref = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; ok && j < nk; ++j) {
-            const int b = j & 1;
-            if (!(ok = __all_sync(0xffffffffu, wait_bar(&bar[SFULL + b], (uint32_t)((j >> 1) & 1), ctl, err))))
+            const int b = j % 3;
+            if (!(ok = __all_sync(0xffffffffu, wait_bar(&bar[SFULL + b], (uint32_t)((j / 3) & 1), ctl, err))))
                 break;
             tc::fence_after_sync();
             float s[128];

@@ -114,6 +114,11 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, 
         }
     }
 }
+// wait_bar for a warp that issues MMAs as a whole (tc::*_w): every lane waits (converged), so that
+// the warp stays converged for the elected issue.
+__device__ __forceinline__ bool wait_bar_w(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, ctl, err));
+}
 // Time-bounded wait that ignores the abort flag (used to drain copies in flight before exit).
 __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = tc::globaltimer();
@@ -746,7 +751,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0 && nch > 0) {
+        if (nch > 0) {  // the whole warp, lane 0 issuing
             const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
@@ -768,21 +773,21 @@ __global__ void __launch_bounds__(NT_WS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = bo + (kk >> 2) * 8192 + (kk & 3) * 32;
-                    tc::mma_bf16_off(tm + TM_X1, dq, off, dk, off, id_kk64, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_X1, dq, off, dk, off, id_kk64, kk > 0);
                 }
-                tc::mma_commit(&bar[X1F]);
+                tc::mma_commit_w(&bar[X1F]);
             };
             // W^T = K^T T1^T, U^T = V^T T2^T (A operands: MN-major views of the K and V tiles)
             auto issue_wu = [&](int c) {
                 const uint32_t bo = (uint32_t)(c & 1) * BUF;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16_off(tm + TM_WT, dkm, bo + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
-                    tc::mma_bf16_off(tm + TM_U, dvm, bo + kk * 2048, dt2, bo + kk * 2048, id_mk64, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_WT, dkm, bo + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_U, dvm, bo + kk * 2048, dt2, bo + kk * 2048, id_mk64, kk > 0);
                 }
-                tc::mma_commit(&bar[WUF]);
+                tc::mma_commit_w(&bar[WUF]);
             };
-            bool ok = wait_bar(&bar[FULL], 0, ctl, err) && wait_bar(&bar[T1R], 0, ctl, err);
+            bool ok = wait_bar_w(&bar[FULL], 0, ctl, err) && wait_bar_w(&bar[T1R], 0, ctl, err);
             if (ok) {
                 tc::fence_after_sync();
                 issue_wu(0);
@@ -791,41 +796,41 @@ __global__ void __launch_bounds__(NT_WS, 1)
             for (int c = 0; ok && c < nch; ++c) {
                 const int b = c & 1;
                 const uint32_t par = (uint32_t)(c & 1), bo = (uint32_t)b * BUF;
-                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[SR], par, ctl, err) && wait_bar_w(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
                 // Delta^T = U^T + S (-W)^T, accumulated onto U^T; then O1 = S Q^T
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_U, ds, kk * 4096, dw, kk * 256, id_km64, 1);
-                tc::mma_commit(&bar[M3]);
+                    tc::mma_bf16_off_w(tm + TM_U, ds, kk * 4096, dw, kk * 256, id_km64, 1);
+                tc::mma_commit_w(&bar[M3]);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_O1 + 64 * b, ds, kk * 4096, dq, bo + (kk >> 2) * 8192 + (kk & 3) * 32,
+                    tc::mma_bf16_off_w(tm + TM_O1 + 64 * b, ds, kk * 4096, dq, bo + (kk >> 2) * 8192 + (kk & 3) * 32,
                                      id_kk64, kk > 0);
                 // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K)
-                if (!(ok = wait_bar(&bar[DLR], par, ctl, err) && wait_bar(&bar[PR], par, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[DLR], par, ctl, err) && wait_bar_w(&bar[PR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_S, ddl, kk * 4096, dkm, bo + kk * 2048, id_km128, 1);
-                tc::mma_commit(&bar[M4S]);
-                tc::mma_commit(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
+                    tc::mma_bf16_off_w(tm + TM_S, ddl, kk * 4096, dkm, bo + kk * 2048, id_km128, 1);
+                tc::mma_commit_w(&bar[M4S]);
+                tc::mma_commit_w(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
                 // the next chunk's W^T, U^T and X1
                 if (c + 1 < nch) {
-                    if (!(ok = wait_bar(&bar[FULL + (b ^ 1)], full_par(c + 1), ctl, err) &&
-                               wait_bar(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
+                    if (!(ok = wait_bar_w(&bar[FULL + (b ^ 1)], full_par(c + 1), ctl, err) &&
+                               wait_bar_w(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
                         break;
                     tc::fence_after_sync();
                     issue_wu(c + 1);
                     issue_x1(c + 1);
                 }
                 // O2 = Delta^T P^T (after the output warps have read the previous O2)
-                if (c >= 1 && !(ok = wait_bar(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err))) break;
+                if (c >= 1 && !(ok = wait_bar_w(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_O2, ddl, kk * 4096, dp, b * 8192 + kk * 2048, id_kk64, kk > 0);
-                tc::mma_commit(&bar[M4O]);
+                    tc::mma_bf16_off_w(tm + TM_O2, ddl, kk * 4096, dp, b * 8192 + kk * 2048, id_kk64, kk > 0);
+                tc::mma_commit_w(&bar[M4O]);
             }
         }
     } else if (warp < 8) {
@@ -962,9 +967,10 @@ __global__ void __launch_bounds__(NT_WS, 1)
         }
         if (v == 0) tc::bulk_wait_all();
     }
-    if (warp == W_MMA && lane == 0) {
-        tc::mma_commit(&bar[FIN]);
-        drain_bar(&bar[FIN], 0);
+    if (warp == W_MMA) {
+        tc::mma_commit_w(&bar[FIN]);
+        if (lane == 0) drain_bar(&bar[FIN], 0);
+        __syncwarp();
     }
     if (split && tid == 0) griddep_wait();  // complete only after the transition grid (the stream's next work reuses the workspace)
     tc::fence_before_sync();
@@ -1149,7 +1155,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         }
     } else if (warp == W_WMMA) {
         // ---------------------------------------------------------------- W issuer: W^T = K^T T1^T, U^T = V^T T2^T
-        if (lane == 0 && nch > 0) {
+        if (nch > 0) {  // the whole warp, lane 0 issuing
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const tc::Desc dkm = tc::split_desc(tc::make_desc_sw128(sb + KRING + KS_K, 8192, 1024));
             const tc::Desc dvm = tc::split_desc(tc::make_desc_sw128(sb + VRING + VS_V, 8192, 1024));
@@ -1159,27 +1165,27 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             for (int c = 0; ok && c < nch; ++c) {
                 // W^T(c - 1) read by prep (WR), the U^T buffer's Delta_S^T of chunk c - 2 read (DSR),
                 // this chunk's K, V, T2 and T1 in place
-                if (c >= 1 && !(ok = wait_bar(&bar[WR], (uint32_t)((c - 1) & 1), ctl, err))) break;
-                if (c >= 2 && !(ok = wait_bar(&bar[DSR + (c & 1)], (uint32_t)(((c - 2) >> 1) & 1), ctl, err))) break;
-                if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
-                           wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err) &&
-                           wait_bar(&bar[T1R], (uint32_t)(c & 1), ctl, err)))
+                if (c >= 1 && !(ok = wait_bar_w(&bar[WR], (uint32_t)((c - 1) & 1), ctl, err))) break;
+                if (c >= 2 && !(ok = wait_bar_w(&bar[DSR + (c & 1)], (uint32_t)(((c - 2) >> 1) & 1), ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
+                           wait_bar_w(&bar[FULLV + (c & 1)], vpar(c), ctl, err) &&
+                           wait_bar_w(&bar[T1R], (uint32_t)(c & 1), ctl, err)))
                     break;
                 tc::fence_after_sync();
                 const uint32_t ko = (uint32_t)(c % 3) * KSLOT, vo = (uint32_t)(c & 1) * VSLOT;
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    tc::mma_bf16_off(tm + TM_WT, dkm, ko + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
-                    tc::mma_bf16_off(tm + TM_U + 64 * (c & 1), dvm, vo + kk * 2048, dt2, vo + kk * 2048, id_mk64,
+                    tc::mma_bf16_off_w(tm + TM_WT, dkm, ko + kk * 2048, dt1, kk * 2048, id_mk64, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_U + 64 * (c & 1), dvm, vo + kk * 2048, dt2, vo + kk * 2048, id_mk64,
                                      kk > 0);
                 }
-                tc::mma_commit(&bar[WUF]);
-                tc::mma_commit(&bar[EMPTYV + (c & 1)]);
+                tc::mma_commit_w(&bar[WUF]);
+                tc::mma_commit_w(&bar[EMPTYV + (c & 1)]);
             }
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------------- S issuer
-        if (lane == 0 && nch > 0) {
+        if (nch > 0) {  // the whole warp, lane 0 issuing
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
             const tc::Desc ds = tc::split_desc(tc::make_desc(sb + S, 2048, 128));
@@ -1191,27 +1197,27 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 const int b = c & 1;
                 const uint32_t par = (uint32_t)(c & 1), ko = (uint32_t)(c % 3) * KSLOT;
                 // Delta_S^T = U^T + S (-W)^T, accumulated onto U^T (W^T, U^T are complete: prep saw WUF before WR)
-                if (!(ok = wait_bar(&bar[SR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[SR], par, ctl, err) && wait_bar_w(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_U + 64 * b, ds, kk * 4096, dw, kk * 256, id_km64, 1);
-                tc::mma_commit(&bar[M3S]);
+                    tc::mma_bf16_off_w(tm + TM_U + 64 * b, ds, kk * 4096, dw, kk * 256, id_km64, 1);
+                tc::mma_commit_w(&bar[M3S]);
                 // S <- gamma_C S + Delta_S^T (diag(e) K)
-                if (!(ok = wait_bar(&bar[DSR + b], (uint32_t)((c >> 1) & 1), ctl, err) &&
-                           wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                if (!(ok = wait_bar_w(&bar[DSR + b], (uint32_t)((c >> 1) & 1), ctl, err) &&
+                           wait_bar_w(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
                     break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_S, dts, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
-                tc::mma_commit(&bar[M4S]);
-                tc::mma_commit(&bar[EMPTYK + c % 3]);
+                    tc::mma_bf16_off_w(tm + TM_S, dts, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
+                tc::mma_commit_w(&bar[M4S]);
+                tc::mma_commit_w(&bar[EMPTYK + c % 3]);
             }
         }
     } else if (warp == W_XMMA) {
         // ---------------------------------------------------------------- X issuer (segments with a Phi chain)
-        if (lane == 0 && nch > 0 && has_x) {
+        if (nch > 0 && has_x) {  // the whole warp, lane 0 issuing
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
             const tc::Desc dx = tc::split_desc(tc::make_desc(sb + X, 2048, 128));
@@ -1222,22 +1228,22 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             for (int c = 0; ok && c < nch; ++c) {
                 const uint32_t par = (uint32_t)(c & 1), ko = (uint32_t)(c % 3) * KSLOT;
                 // X (-W)^T
-                if (!(ok = wait_bar(&bar[XR], par, ctl, err) && wait_bar(&bar[WR], par, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[XR], par, ctl, err) && wait_bar_w(&bar[WR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_DX, dx, kk * 4096, dw, kk * 256, id_km64, kk > 0);
-                tc::mma_commit(&bar[M3X]);
+                    tc::mma_bf16_off_w(tm + TM_DX, dx, kk * 4096, dw, kk * 256, id_km64, kk > 0);
+                tc::mma_commit_w(&bar[M3X]);
                 // X <- gamma_C X + X (-W)^T diag(e) K
-                if (!(ok = wait_bar(&bar[DXR], par, ctl, err) &&
-                           wait_bar(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                if (!(ok = wait_bar_w(&bar[DXR], par, ctl, err) &&
+                           wait_bar_w(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
                     break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16_off(tm + TM_X, dtx, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
-                tc::mma_commit(&bar[M4X]);
-                tc::mma_commit(&bar[EMPTYK + c % 3]);
+                    tc::mma_bf16_off_w(tm + TM_X, dtx, kk * 4096, dkm, ko + kk * 2048, id_km128, 1);
+                tc::mma_commit_w(&bar[M4X]);
+                tc::mma_commit_w(&bar[EMPTYK + c % 3]);
             }
         }
     } else if (warp < 16) {
@@ -1424,27 +1430,26 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                     if (last[b]) drain_bar(&bar[PFULL + b], (uint32_t)(((last[b] - 1) >> 1) & 1));
             }
         } else if (warp == W_MMA) {
-            if (lane == 0 && ok) {
+            if (__all_sync(0xffffffffu, ok)) {  // the whole warp, lane 0 issuing
                 const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
                 for (int j = 1; j <= nfold; ++j) {
                     const int b = j & 1;
                     const bool own = j == nfold;
-                    if (!(j == 1 ? wait_bar(&bar[A1R], 0, ctl, err)
-                                 : wait_bar(&bar[AREADY], (uint32_t)((j - 2) & 1), ctl, err)))
+                    if (!(j == 1 ? wait_bar_w(&bar[A1R], 0, ctl, err)
+                                 : wait_bar_w(&bar[AREADY], (uint32_t)((j - 2) & 1), ctl, err)))
                         break;
-                    if (!wait_bar(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
+                    if (!wait_bar_w(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
                     tc::fence_after_sync();
-                    const uint32_t d = tm + (own ? TM_S : TM_D), phi = sb + PHI + 65536u * b;
+                    const uint32_t d = tm + (own ? TM_S : TM_D);
+                    const tc::Desc dph = tc::split_desc(tc::make_desc(sb + PHI + 65536u * b, 128, 2048));
 #pragma unroll 1
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t ah = tm + TM_A + 16 * kk, al = ah + 8;
-                        const uint64_t bh = tc::make_desc(phi + kk * 256, 128, 2048);
-                        const uint64_t bl = tc::make_desc(phi + 32768 + kk * 256, 128, 2048);
-                        tc::mma_bf16_ts(d, ah, bh, id_km128, (own || kk > 0) ? 1u : 0u);
-                        tc::mma_bf16_ts(d, ah, bl, id_km128, 1);
-                        tc::mma_bf16_ts(d, al, bh, id_km128, 1);
+                        tc::mma_bf16_ts_off_w(d, ah, dph, kk * 256, id_km128, (own || kk > 0) ? 1u : 0u);
+                        tc::mma_bf16_ts_off_w(d, ah, dph, 32768 + kk * 256, id_km128, 1);
+                        tc::mma_bf16_ts_off_w(d, al, dph, kk * 256, id_km128, 1);
                     }
-                    tc::mma_commit(&bar[MDONE + b]);
+                    tc::mma_commit_w(&bar[MDONE + b]);
                 }
             }
         }
@@ -1463,17 +1468,11 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         }
         __threadfence();
     }
-    if (warp == W_MMA && lane == 0) {
-        tc::mma_commit(&bar[FIN]);
-        drain_bar(&bar[FIN], 0);
-    }
-    if (warp == W_XMMA && lane == 0) {
-        tc::mma_commit(&bar[FINX]);
-        drain_bar(&bar[FINX], 0);
-    }
-    if (warp == W_WMMA && lane == 0) {
-        tc::mma_commit(&bar[FINW]);
-        drain_bar(&bar[FINW], 0);
+    if (warp == W_MMA || warp == W_XMMA || warp == W_WMMA) {
+        uint64_t *fin = &bar[warp == W_MMA ? FIN : warp == W_XMMA ? FINX : FINW];
+        tc::mma_commit_w(fin);
+        if (lane == 0) drain_bar(fin, 0);
+        __syncwarp();
     }
     tc::fence_before_sync();
     __syncthreads();

@@ -39,17 +39,22 @@ namespace {
 
 using bf16_t = __nv_bfloat16;
 constexpr int BM = 128, BK = 64;
-constexpr int NSTAGE = 4, NBSLOT = 3;
+constexpr int NBSLOT = 3;
+// ring depth of the x and int8 stages: deeper for the narrow tiles of small T, where each CTA's
+// K loop is a chain of load latencies rather than of products
+template <int BN>
+constexpr int nstage() { return BN >= 256 ? 4 : BN >= 128 ? 6 : 8; }
+constexpr int NSTAGE_MAX = 8;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int NCONV = 256;                       // converter threads (8 warps)
 constexpr int NTHREADS = 96 + NCONV + 128;       // x loader, MMA, w8 loader, converters, epilogue (15 warps)
 constexpr int W_LOAD = 0, W_MMA = 1, W_LOADW = 2, W_CONV0 = 3, W_EPI0 = 3 + NCONV / 32;
 enum {
-    FULL = 0,                    // [NSTAGE] x tile of a stage landed (x loader arrive + bytes)
-    EMPTY = FULL + NSTAGE,       // [NSTAGE] x stage free (MMA commit)
-    WFULL = EMPTY + NSTAGE,      // [NSTAGE] int8 weight tile landed (w8 loader arrive + bytes)
-    WEMPTY = WFULL + NSTAGE,     // [NSTAGE] int8 stage free (every converter)
-    BFULL = WEMPTY + NSTAGE,     // [NBSLOT] bf16 weight tile written (every converter)
+    FULL = 0,                        // [stages] x tile of a stage landed (x loader arrive + bytes)
+    EMPTY = FULL + NSTAGE_MAX,       // [stages] x stage free (MMA commit)
+    WFULL = EMPTY + NSTAGE_MAX,      // [stages] int8 weight tile landed (w8 loader arrive + bytes)
+    WEMPTY = WFULL + NSTAGE_MAX,     // [stages] int8 stage free (every converter)
+    BFULL = WEMPTY + NSTAGE_MAX,     // [NBSLOT] bf16 weight tile written (every converter)
     BEMPTY = BFULL + NBSLOT,     // [NBSLOT] bf16 weight tile read by the MMAs (commit)
     AFULL = BEMPTY + NBSLOT,     // [2] accumulator complete (commit)
     AEMPTY = AFULL + 2,          // [2] accumulator read out (128 epilogue threads)
@@ -57,19 +62,20 @@ enum {
     NBAR = FIN + 1
 };
 __host__ __device__ constexpr uint32_t bar_count(int i) {
-    return (i >= WEMPTY && i < WEMPTY + NSTAGE) ? (uint32_t)NCONV : (i >= BFULL && i < BFULL + NBSLOT) ? (uint32_t)NCONV
+    return (i >= WEMPTY && i < WEMPTY + NSTAGE_MAX) ? (uint32_t)NCONV : (i >= BFULL && i < BFULL + NBSLOT) ? (uint32_t)NCONV
            : (i >= AEMPTY && i < AEMPTY + 2) ? 128u : 1u;
 }
 
 // Shared-memory layout for a channel tile of BN (x: 128 x 64 bf16; w8: BN x 64 int8; bf16 weight tile BN x 64).
 template <int BN>
 struct Lay {
+    static constexpr int NSTAGE = nstage<BN>();
     static constexpr uint32_t A_BYTES = BM * BK * 2, W8_BYTES = BN * BK, B_BYTES = BN * BK * 2;
     static constexpr uint32_t OFF_A = 0, OFF_W8 = OFF_A + NSTAGE * A_BYTES, OFF_B = OFF_W8 + NSTAGE * W8_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_B + NBSLOT * B_BYTES, OFF_CTL = OFF_BAR + 8 * NBAR;
     static constexpr uint32_t TOTAL = OFF_CTL + 16 + 1024;  // + slack for the 1024-byte alignment
 };
-static_assert(Lay<256>::TOTAL <= 232448, "shared memory");
+static_assert(Lay<256>::TOTAL <= 232448 && Lay<128>::TOTAL <= 232448 && Lay<64>::TOTAL <= 232448, "shared memory");
 
 struct Ctl {
     uint32_t tmem, abort;
@@ -89,6 +95,11 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, 
             }
         }
     }
+}
+// wait_bar for a warp that issues MMAs as a whole (tc::*_w): every lane waits (converged), so that
+// the warp stays converged for the elected issue.
+__device__ __forceinline__ bool wait_bar_w(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    return __all_sync(0xffffffffu, wait_bar(bar, parity, ctl, err));
 }
 __device__ __noinline__ void drain_bar(uint64_t *bar, uint32_t parity) {
     const uint64_t t0 = tc::globaltimer();
@@ -129,6 +140,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const float *__restrict__ scale, int T, int D, Route rt, bf16_t *__restrict__ q, bf16_t *__restrict__ k,
               bf16_t *__restrict__ v, float *__restrict__ ga, float *__restrict__ gb, uint32_t *__restrict__ err) {
     using L = Lay<BN>;
+    constexpr int NSTAGE = L::NSTAGE;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = tc::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024u - (raw_base & 1023u)) & 1023u);  // 1024-byte aligned for the swizzle
@@ -177,7 +189,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 drain_bar(&full[j % NSTAGE], (uint32_t)((j / NSTAGE) & 1));
         }
     } else if (warp == W_MMA) {
-        if (lane == 0) {
+        {  // the whole warp, lane 0 issuing
             const uint32_t idesc = tc::make_idesc_bf16(BM, BN, 0, 0);
             const tc::Desc da = tc::split_desc(tc::make_desc_sw128(sb + L::OFF_A, 16, 1024));
             const tc::Desc db = tc::split_desc(tc::make_desc_sw128(sb + L::OFF_B, 16, 1024));
@@ -185,25 +197,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
                 const int acc = ti & 1;
-                if (ti >= 2 && !(ok = wait_bar(&bar[AEMPTY + acc], (uint32_t)(((ti >> 1) - 1) & 1), ctl, err))) break;
+                if (ti >= 2 && !(ok = wait_bar_w(&bar[AEMPTY + acc], (uint32_t)(((ti >> 1) - 1) & 1), ctl, err))) break;
                 tc::fence_after_sync();
                 for (int ks = 0; ks < ksteps; ++ks, ++it) {
                     const int s = it % NSTAGE, bs = it % NBSLOT;
-                    if (!(ok = wait_bar(&bar[FULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
-                               wait_bar(&bar[BFULL + bs], (uint32_t)((it / NBSLOT) & 1), ctl, err)))
+                    if (!(ok = wait_bar_w(&bar[FULL + s], (uint32_t)((it / NSTAGE) & 1), ctl, err) &&
+                               wait_bar_w(&bar[BFULL + bs], (uint32_t)((it / NBSLOT) & 1), ctl, err)))
                         break;
                     tc::fence_after_sync();
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk)
-                        tc::mma_bf16_off(tm + acc * BN, da, s * L::A_BYTES + kk * 32, db, bs * L::B_BYTES + kk * 32,
+                        tc::mma_bf16_off_w(tm + acc * BN, da, s * L::A_BYTES + kk * 32, db, bs * L::B_BYTES + kk * 32,
                                          idesc, (ks > 0 || kk > 0) ? 1u : 0u);
-                    tc::mma_commit(&bar[EMPTY + s]);
-                    tc::mma_commit(&bar[BEMPTY + bs]);
+                    tc::mma_commit_w(&bar[EMPTY + s]);
+                    tc::mma_commit_w(&bar[BEMPTY + bs]);
                 }
-                if (ok) tc::mma_commit(&bar[AFULL + acc]);
+                if (ok) tc::mma_commit_w(&bar[AFULL + acc]);
             }
-            tc::mma_commit(&bar[FIN]);
-            drain_bar(&bar[FIN], 0);
+            tc::mma_commit_w(&bar[FIN]);
+            if (lane == 0) drain_bar(&bar[FIN], 0);
+            __syncwarp();
         }
     } else if (warp < W_EPI0) {
         // ---------------------------------------------------------------- convert (NCONV threads)

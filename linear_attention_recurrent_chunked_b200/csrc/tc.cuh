@@ -136,6 +136,44 @@ __device__ __forceinline__ void mma_bf16_ts_off(uint32_t d_tmem, uint32_t a_tmem
         : "memory");
 }
 
+// Warp-issued forms: all 32 lanes of a warp execute the call with the same operands and the lane
+// that elect.sync picks (the same lane every time the whole warp executes it) issues the
+// instruction. The operands are
+// then warp-uniform, so they stay in uniform registers; an MMA issued from a single thread
+// under a lane test instead moves every operand to the uniform datapath per instruction, which
+// measured about 60 cycles per tcgen05.mma on B200 against 25-45 cycles issued this way.
+// A warp that issues this way must also commit this way (a commit tracks its own thread's MMAs).
+__device__ __forceinline__ void mma_bf16_off_w(uint32_t d_tmem, Desc a, uint32_t a_off, Desc b, uint32_t b_off,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 ad, bd;\n\t"
+        "mov.b64 ad, {%1, %2};\n\t"
+        "mov.b64 bd, {%3, %4};\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %5, p;\n\t}" ::"r"(d_tmem),
+        "r"(a.lo + (a_off >> 4)), "r"(a.hi), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_off_w(uint32_t d_tmem, uint32_t a_tmem, Desc b, uint32_t b_off,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t *mbar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(mbar))
+        : "memory");
+}
+
 // Arrive (once) on the mbarrier when all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))
