@@ -182,7 +182,11 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
  * Synchronises `stream` and reads the device error word that the last
  * gdn_chunk_fwd on this workspace wrote: GDN_OK, GDN_ERR_SEQLENS or
  * GDN_ERR_TIMEOUT (a bounded inter-block wait gave up; outputs are then
- * incomplete). The word is reset by every gdn_chunk_fwd call.
+ * incomplete). The word is reset by every gdn_chunk_fwd call. On a timeout
+ * of the pipelined path, gdn_last_error() names the first wait that gave up
+ * (the mbarrier's shared-memory address and awaited parity, or the flag's
+ * word offset in the workspace, with the block and thread), a diagnostic for
+ * whoever changes the kernels.
  */
 gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *stream);
 

@@ -97,6 +97,16 @@ struct Ctl {
     uint32_t abort;  // set by the first role that gives up
 };
 
+// The first wait of a call that runs out of time records where, after the error word (the plan
+// kernel clears these words): err[1] = 1 + the mbarrier's shared-memory address, or bit 30 + the
+// flag's word offset from the error word; err[2] = blockIdx.y << 16 | blockIdx.x; err[3] =
+// threadIdx.x | the awaited parity << 16.
+__device__ __forceinline__ void record_timeout_site(uint32_t *err, uint32_t what, uint32_t parity) {
+    if (atomicCAS(err + 1, 0u, what) == 0u) {
+        err[2] = (blockIdx.y << 16) | blockIdx.x;
+        err[3] = threadIdx.x | (parity << 16);
+    }
+}
 // Bounded wait for the phase `parity` of an mbarrier. Gives up when another
 // role has aborted, or after kWaitNs (then it records the timeout and aborts).
 __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
@@ -108,6 +118,7 @@ __device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, 
             if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
             if (tc::globaltimer() - t0 > kWaitNs) {
                 atomicOr(err, ERRBIT_TIMEOUT);
+                record_timeout_site(err, 1u + tc::smem_u32(bar), parity);
                 *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
                 return false;
             }
@@ -137,6 +148,7 @@ __device__ __noinline__ bool wait_flag(const uint32_t *p, Ctl *ctl, uint32_t *er
         if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
         if (tc::globaltimer() - t0 > bound_ns) {
             atomicOr(err, ERRBIT_TIMEOUT);
+            record_timeout_site(err, (1u << 30) | (uint32_t)(p - err), 0u);
             break;
         }
         __nanosleep(32);
@@ -1499,6 +1511,7 @@ __global__ void __launch_bounds__(256) k_ws_plan(const int32_t *__restrict__ cu,
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     griddep_launch();  // the prep kernel may launch now; it waits for this grid to complete
     if (tid == 0) bad = 0;
+    if (tid < 3) err[1 + tid] = 0u;  // timeout site record
     for (int i = tid; i < nflags; i += 256) flags[i] = 0u;
     __syncthreads();
     // thread tid owns sequences [n0, n1)

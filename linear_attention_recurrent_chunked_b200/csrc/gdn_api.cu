@@ -257,12 +257,26 @@ gdn_status gdn_chunk_fwd_raw(const void *q_raw, const void *k_raw, const void *v
 gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *stream) {
     if (!workspace || ws_bytes < sizeof(uint32_t)) return fail(GDN_ERR_WORKSPACE, "workspace missing");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint32_t word = 0;
-    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st);
+    // the error word, then (pipelined path) where the first timed-out wait was: the barrier's
+    // shared-memory address + 1 or bit 30 + a flag's word offset, the block, the thread and parity
+    uint32_t w[4] = {0, 0, 0, 0};
+    const size_t n = ws_bytes >= sizeof(w) ? sizeof(w) : sizeof(uint32_t);
+    cudaError_t e = cudaMemcpyAsync(w, workspace, n, cudaMemcpyDeviceToHost, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    const uint32_t word = w[0];
     if (word & gdn::ERRBIT_SEQLENS) return fail(GDN_ERR_SEQLENS, "cu_seqlens is not 0 = c0 <= c1 <= ... <= cN = T_tot");
-    if (word & gdn::ERRBIT_TIMEOUT) return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    if (word & gdn::ERRBIT_TIMEOUT) {
+        if (w[1] & (1u << 30))
+            return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up (first: flag word %u, block (%u, %u), thread %u)",
+                        w[1] & 0x3FFFFFFFu, w[2] & 0xFFFFu, w[2] >> 16, w[3] & 0xFFFFu);
+        if (w[1])
+            return fail(GDN_ERR_TIMEOUT,
+                        "a bounded device-side wait gave up (first: mbarrier at shared address %u, parity %u, block "
+                        "(%u, %u), thread %u)",
+                        w[1] - 1u, w[3] >> 16, w[2] & 0xFFFFu, w[2] >> 16, w[3] & 0xFFFFu);
+        return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
+    }
     if (word & gdn::ERRBIT_INTERNAL) return fail(GDN_ERR_CUDA, "internal: misaligned shared-memory base, nothing written");
     return ok();
 }

@@ -44,10 +44,13 @@ def test_withheld_link_times_out_reports_and_recovers():
         gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], dw["cu_seqlens"], o=o, S_T=S_T,
                       workspace=ws)
         status = lib.gdn_chunk_fwd_check(_p(ws), ws.numel(), stream)
+        message = lib.gdn_last_error()  # (the next successful call clears it)
         elapsed = time.perf_counter() - t0
     finally:
         gdn.debug_inject(0, 0)
-    assert status == 8, (status, lib.gdn_last_error())  # GDN_ERR_TIMEOUT
+    assert status == 8, (status, message)  # GDN_ERR_TIMEOUT
+    # the message names the first wait that gave up: a wait for the withheld end-state flag
+    assert b"flag word" in message, message
     assert elapsed < 5.0, elapsed  # the waits gave up after the injected bound, not after 1 s each
     o_ref, S_ref = oracle.scan(w["q"], w["k"], w["v"], w["g"], w["beta"], S0=w["S0"], cu_seqlens=w["cu_seqlens"])
     # head 1 never waits for head 0: its outputs and final state are complete and correct
