@@ -72,10 +72,10 @@ constexpr uint32_t REC_VEC = 8192;  // G (log2 units), gamma, e, beta: 4 x 64 fp
 constexpr uint32_t REC_BYTES = 9216;
 // ---- published segment end state: bf16 hi and lo tiles, rows v, runs along k (sx = 128, sy = 2048)
 constexpr uint32_t LINK_BYTES = 65536;
-// ---- published part of a segment after the first (S_end = S_in Phi + S_loc): Phi as bf16 hi and lo
-// tiles in the B-operand layout of the link step (rows k, runs along k'; sx = 128, sy = 2048), then
-// S_loc in fp32 as [k / 4][v][4] (one 16-byte group per TMEM lane and column quad, so that a warp's
-// 32 lanes touch 512 contiguous bytes)
+// ---- published part of a segment after the first (S_end = S_in Phi + S_loc): Phi as the fold's
+// tf32 B operand (fp32 rounded to tf32; K-major rows k', 128-byte swizzle, four 16 KB K groups of 32
+// values of k), then S_loc in fp32 as [k / 4][v][4] (one 16-byte group per TMEM lane and column
+// quad, so that a warp's 32 lanes touch 512 contiguous bytes)
 constexpr uint32_t PART_PHI = 0, PART_S = 65536, PART_BYTES = 131072;
 constexpr uint32_t FLAG_DONE = 1u, FLAG_FAILED = 2u;
 
@@ -342,24 +342,8 @@ __device__ __forceinline__ void state_init64(uint32_t s_tile, uint32_t tl_s, int
     tc::tmem_st_wait();
 }
 
-// bf16 hi / lo split of 32 values of row `row` into two tiles (sx = 128, sy = 2048)
-// in shared memory (hi at base, lo at base + 32 KB).
-__device__ __forceinline__ void st_split32(uint32_t base, int row, int c0, const float *x) {
-#pragma unroll
-    for (int i = 0; i < 32; i += 8) {
-        float hi[8], lo[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            hi[j] = __bfloat162float(__float2bfloat16_rn(x[i + j]));
-            lo[j] = x[i + j] - hi[j];
-        }
-        st_run8(base + tc::tile_off(row, c0 + i, 128, 2048), hi);
-        st_run8(base + 32768 + tc::tile_off(row, c0 + i, 128, 2048), lo);
-    }
-}
-
-// The same split into global memory (hi at base, lo at base + 32 KB; same byte layout, so that a
-// bulk copy reproduces the shared-memory tiles).
+// bf16 hi / lo split of 32 values of row `row` into global memory: two tiles (sx = 128, sy = 2048),
+// hi at base, lo at base + 32 KB.
 __device__ __forceinline__ void st_split32_global(uint8_t *base, int row, int c0, const float *x) {
 #pragma unroll
     for (int i = 0; i < 32; i += 8) {
@@ -1008,11 +992,10 @@ constexpr uint32_t DTX = DTS + 16384;
 constexpr uint32_t BAR = DTX + 16384;
 constexpr uint32_t TOTAL = BAR + 320;
 // link phase (after the chunk loop every tile is free)
-constexpr uint32_t PHI = 0;  // two buffers: Phi_j hi | lo as B operands (rows k, runs along k'; sy = 2048)
-// TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T;
-// in the link phase the fold's product P takes TM_D and its A operand split(S_end(j)) TM_A: for K
-// step kk (16 values of k), 8 columns of bf16 pairs hi then 8 of lo, at TM_A + 16 kk
-constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448, TM_D = 256, TM_A = 384;
+constexpr uint32_t PHI = 0;  // two buffers: Phi_j as a tf32 B operand (K-major rows k', 128-byte swizzle; 64 KB)
+// TMEM columns: S_loc, X, U^T (two buffers, Delta_S^T accumulated onto them), W^T, X (-W)^T; in the
+// link phase the fold's end states F(j) take columns 256 and 384 in turn (see fbuf)
+constexpr uint32_t TM_S = 0, TM_X = 128, TM_U = 256, TM_WT = 384, TM_DX = 448;
 // Three MMA issuers: S chain, X chain, and the W issuer (the next chunk's W^T, U^T).
 // A barrier that both issuers (or an issuer and a role that can run a chunk ahead) wait for is
 // kept in several copies indexed by the chunk, so that no waiter can see it a whole phase later.
@@ -1031,19 +1014,20 @@ enum {
     FINX = 27,  // the same for the X issuer
     FINW = 28,  // the same for the W issuer
     // link phase, fold step j (buffer j & 1 where there are two)
-    A1R = 29,     // the first step's A is in TM_A (S warps, 256)
-    AREADY = 30,  // split(S_end(j)) is in TM_A and P has been read (S and X warps, 512)
-    PFULL = 31,   // [2] Phi_j landed
-    MDONE = 33,   // [2] the step's MMAs are done
-    NBAR = 35
+    A1R = 29,     // F(0), the first segment's end state, is in TMEM (S warps, 256)
+    AREADY = 30,  // [2] F(j) holds S_loc(j) (S and X warps, 512)
+    PUBD = 32,    // the part has been read out of TMEM (X warps, 256)
+    PFULL = 33,   // [2] Phi_j landed
+    MDONE = 35,   // [2] the step's MMAs are done
+    NBAR = 37
 };
 // (EMPTYK takes a commit from each issuer: count 2 with an X chain, 1 without.)
 __device__ __forceinline__ constexpr uint32_t bar_count(int i, bool has_x) {
     return (i >= EMPTYK && i < EMPTYK + 3)                                  ? (has_x ? 2u : 1u)
            : (i >= T1R && i < KR + 4)                                       ? 128u
            : (i >= SR && i <= DXR)                                          ? 256u
-           : (i == A1R)                                                     ? 256u
-           : (i == AREADY)                                                  ? 512u
+           : (i == A1R || i == PUBD)                                        ? 256u
+           : (i == AREADY || i == AREADY + 1)                               ? 512u
                                                                             : 1u;
 }
 static_assert(BAR + 8 * NBAR + 8 <= TOTAL, "barrier area");
@@ -1326,14 +1310,15 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     // the first publishes its part (Phi, S_loc) as soon as its chunk loop ends; segment s then folds
     // the parts of segments 1 .. s itself, starting from the first segment's published end state,
     // instead of waiting for its predecessor's end state (a chain of s cross-CTA hand-offs). A step
-    // is P = split(S_end(j - 1)) Phi(j) on the tensor cores (bf16 hi/lo operands: hi hi + hi lo +
-    // lo hi, fp32 accumulation; A in TMEM), then S_end(j) = P + S_loc(j) in fp32 and its split for
-    // the next step; the last step accumulates onto this segment's own S_loc in TMEM.
+    // is F(j) = S_loc(j) + F(j - 1) Phi(j) on the tensor cores with no thread work on the chain: A is
+    // F(j - 1), the previous step's fp32 accumulator read as tf32 from TMEM, B the published Phi(j)
+    // (tf32), D a buffer the threads filled with S_loc(j) beforehand; the last step accumulates onto
+    // this segment's own S_loc in TMEM.
     //   X warps   publish the part (Phi from X, S_loc from S)
-    //   S warps   the first step's A = the first segment's published end state (already split)
+    //   S warps   F(0) = the first segment's published end state
     //   loader    Phi_j into buffer j & 1
-    //   S issuer  the step's 24 MMAs
-    //   S, X warps  (16, 32 columns each) add S_loc(j) and split into TM_A; S warps publish S_end(s)
+    //   S issuer  the step's 16 MMAs
+    //   S, X warps  (32 columns each) load S_loc(j) into F(j) before step j; S warps publish S_end(s)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -1341,20 +1326,35 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     const int nfold = sg.s;                              // fold steps; the last is this segment's own
     const size_t slot0 = (size_t)(gseg - sg.s) * H + h;  // the sequence's first segment
     auto part_of = [&](int j) { return part + (slot0 + (size_t)j * H) * PART_BYTES; };
+    // TMEM buffers of the fold's intermediate end states F(j), j = 0 .. nfold - 1 (F(0) the first
+    // segment's end state; F(j), j >= 1, holds S_loc(j) before step j accumulates onto it): columns 256
+    // and 384 in turn. (A third buffer over the X state's columns 128 .. 255 gave wrong end states
+    // from the third fold step on, on B200, although the part had been read out of them first; two
+    // buffers cost one S_loc load per step on the chain.)
+    auto fbuf = [&](int j) { return tm + ((j & 1) ? 384u : 256u); };
     if (has_x) {
         if (warp < 16) {
             const int r = quarter_lane;
             const uint32_t tl = lane_base(tm, warp);
             if (warp >= 8) {
+                // X warps: publish the part. Phi as a ready tf32 B operand of the fold (K-major, rows k',
+                // 128-byte swizzle: Phi[k][k'] at (k / 32) 16 KB + 128 k' + the swizzled 16-byte group of k);
+                // S_loc as [k / 4][v][4]
                 const int half = (warp >> 2) & 1;
                 if (ok) {
                     uint8_t *pt = part_of(nfold);
                     float4 *ps = reinterpret_cast<float4 *>(pt + PART_S);
+                    uint32_t *pphi = reinterpret_cast<uint32_t *>(pt + PART_PHI);
+                    const uint32_t kbase = (uint32_t)(r >> 5) * 4096u + (uint32_t)(r & 3), kgrp = (uint32_t)(r & 31) >> 2;
 #pragma unroll 1
                     for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
                         float x[32];
                         tc::tmem_ld32(tl + TM_X + c0, x);
-                        st_split32_global(pt + PART_PHI, r, c0, x);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const uint32_t n = (uint32_t)(c0 + i);
+                            pphi[kbase + 32u * n + ((kgrp ^ (n & 7u)) << 2)] = tc::to_tf32(x[i]);
+                        }
                         tc::tmem_ld32(tl + TM_S + c0, x);
 #pragma unroll
                         for (int i = 0; i < 32; i += 4)
@@ -1362,67 +1362,63 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                     }
                     __threadfence();
                 }
-                tc::fence_before_sync();  // the reads of S_loc precede the own fold step, which accumulates onto it
+                // TM_S is read: the own step may accumulate onto S_loc
+                tc::fence_before_sync();
+                tc::mbar_arrive(&bar[PUBD]);
                 tc::named_sync(1, 256);
                 if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
             } else if (ok) {
+                // S warps: F(0) = the first segment's published end state, hi + lo in fp32
                 const int half = (warp >> 2) & 1;
                 if ((ok = __all_sync(0xffffffffu, wait_flag(flags + slot0, ctl, err, flag_ns)))) {
                     const uint8_t *src = link + slot0 * LINK_BYTES;
 #pragma unroll 1
                     for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
-                        // K step c0 / 16: the hi runs of columns c0 .., c0 + 8 .., then the lo runs
-                        const uint4 h0 = __ldcg(reinterpret_cast<const uint4 *>(src + tc::tile_off(r, c0, 128, 2048)));
-                        const uint4 h1 = __ldcg(reinterpret_cast<const uint4 *>(src + tc::tile_off(r, c0 + 8, 128, 2048)));
-                        const uint4 l0 = __ldcg(reinterpret_cast<const uint4 *>(src + 32768 + tc::tile_off(r, c0, 128, 2048)));
-                        const uint4 l1 =
-                            __ldcg(reinterpret_cast<const uint4 *>(src + 32768 + tc::tile_off(r, c0 + 8, 128, 2048)));
-                        const float u[16] = {__uint_as_float(h0.x), __uint_as_float(h0.y), __uint_as_float(h0.z),
-                                             __uint_as_float(h0.w), __uint_as_float(h1.x), __uint_as_float(h1.y),
-                                             __uint_as_float(h1.z), __uint_as_float(h1.w), __uint_as_float(l0.x),
-                                             __uint_as_float(l0.y), __uint_as_float(l0.z), __uint_as_float(l0.w),
-                                             __uint_as_float(l1.x), __uint_as_float(l1.y), __uint_as_float(l1.z),
-                                             __uint_as_float(l1.w)};
-                        tc::tmem_st16(tl + TM_A + c0, u);
+                        float u[16];
+#pragma unroll
+                        for (int h8 = 0; h8 < 16; h8 += 8) {
+                            const uint32_t off = tc::tile_off(r, c0 + h8, 128, 2048);
+                            const uint4 hi = __ldcg(reinterpret_cast<const uint4 *>(src + off));
+                            const uint4 lo = __ldcg(reinterpret_cast<const uint4 *>(src + 32768 + off));
+                            const uint32_t *wh = reinterpret_cast<const uint32_t *>(&hi);
+                            const uint32_t *wl = reinterpret_cast<const uint32_t *>(&lo);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wh[q]));
+                                const float2 e = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wl[q]));
+                                u[h8 + 2 * q] = a.x + e.x;
+                                u[h8 + 2 * q + 1] = a.y + e.y;
+                            }
+                        }
+                        tc::tmem_st16(lane_base(fbuf(0), warp) + c0, u);
                     }
                     tc::tmem_st_wait();
                 }
                 tc::fence_before_sync();
                 tc::mbar_arrive(&bar[A1R]);
             }
-            // S_end(j) = P + S_loc(j) and its split, steps 1 .. nfold - 1 (columns c0 .. c0 + 31)
+            // F(j) = S_loc(j), j = 1 .. nfold - 1, columns c0 .. c0 + 31 (S and X warps): the buffer's
+            // earlier content F(j - 2) was last read by step j - 1
             const int c0 = 32 * (warp >> 2);
             for (int j = 1; ok && j < nfold; ++j) {
-                const int b = j & 1;
                 if (!(ok = __all_sync(0xffffffffu, wait_flag(pflags + slot0 + (size_t)j * H, ctl, err, flag_ns)))) break;
                 const float4 *src = reinterpret_cast<const float4 *>(part_of(j) + PART_S) + (c0 >> 2) * D + r;
-                float4 sl[8];  // in flight during the step's MMAs
+                float4 sl[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) sl[i] = __ldcg(src + i * D);
-                if (!(ok = wait_bar(&bar[MDONE + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err))) break;
+                if (j >= 2 && !(ok = __all_sync(0xffffffffu, wait_bar(&bar[MDONE + ((j - 1) & 1)],
+                                                                      (uint32_t)(((j - 2) >> 1) & 1), ctl, err))))
+                    break;
                 tc::fence_after_sync();
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    float x[16], u[16];
-                    tc::tmem_ld16(tl + TM_D + c0 + 16 * t, x);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 s4 = sl[4 * t + (i >> 1)];
-                        const float a0 = x[2 * i] + ((i & 1) ? s4.z : s4.x);
-                        const float a1 = x[2 * i + 1] + ((i & 1) ? s4.w : s4.y);
-                        const float h0 = __bfloat162float(__float2bfloat16_rn(a0));
-                        const float h1 = __bfloat162float(__float2bfloat16_rn(a1));
-                        u[i] = __uint_as_float(tc::pack_bf16x2(h0, h1));
-                        u[8 + i] = __uint_as_float(tc::pack_bf16x2(a0 - h0, a1 - h1));
-                    }
-                    tc::tmem_st16(tl + TM_A + c0 + 16 * t, u);
-                }
+                tc::tmem_st32(lane_base(fbuf(j), warp) + c0, *reinterpret_cast<const uint32_t(*)[32]>(sl));
                 tc::tmem_st_wait();
                 tc::fence_before_sync();
-                tc::mbar_arrive(&bar[AREADY]);
+                tc::mbar_arrive(&bar[AREADY + (j & 1)]);
             }
+            // (S warps) the own step is complete before S_end is published
             if (warp < 8 && ok)
-                ok = wait_bar(&bar[MDONE + (nfold & 1)], (uint32_t)(((nfold - 1) >> 1) & 1), ctl, err);
+                ok = __all_sync(0xffffffffu,
+                                wait_bar(&bar[MDONE + (nfold & 1)], (uint32_t)(((nfold - 1) >> 1) & 1), ctl, err));
         } else if (warp == W_LOAD) {
             if (lane == 0 && ok) {
                 int last[2] = {0, 0};
@@ -1443,24 +1439,25 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             }
         } else if (warp == W_MMA) {
             if (__all_sync(0xffffffffu, ok)) {  // the whole warp, lane 0 issuing
-                const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
+                const uint32_t it128 = tc::make_idesc_tf32(128, 128);
                 for (int j = 1; j <= nfold; ++j) {
                     const int b = j & 1;
                     const bool own = j == nfold;
-                    if (!(j == 1 ? wait_bar_w(&bar[A1R], 0, ctl, err)
-                                 : wait_bar_w(&bar[AREADY], (uint32_t)((j - 2) & 1), ctl, err)))
+                    // A = F(j - 1) (loaded, or the previous step complete: a product does not wait for the
+                    // tensor-memory writes of an earlier one by itself); D = F(j) holding S_loc(j), or this
+                    // segment's S_loc once its part is read out; Phi_j landed
+                    if (!((j == 1 ? wait_bar_w(&bar[A1R], 0, ctl, err)
+                                  : wait_bar_w(&bar[MDONE + ((j - 1) & 1)], (uint32_t)(((j - 2) >> 1) & 1), ctl, err)) &&
+                          (own ? wait_bar_w(&bar[PUBD], 0, ctl, err)
+                               : wait_bar_w(&bar[AREADY + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) &&
+                          wait_bar_w(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)))
                         break;
-                    if (!wait_bar_w(&bar[PFULL + b], (uint32_t)(((j - 1) >> 1) & 1), ctl, err)) break;
                     tc::fence_after_sync();
-                    const uint32_t d = tm + (own ? TM_S : TM_D);
-                    const tc::Desc dph = tc::split_desc(tc::make_desc(sb + PHI + 65536u * b, 128, 2048));
-#pragma unroll 1
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t ah = tm + TM_A + 16 * kk, al = ah + 8;
-                        tc::mma_bf16_ts_off_w(d, ah, dph, kk * 256, id_km128, (own || kk > 0) ? 1u : 0u);
-                        tc::mma_bf16_ts_off_w(d, ah, dph, 32768 + kk * 256, id_km128, 1);
-                        tc::mma_bf16_ts_off_w(d, al, dph, kk * 256, id_km128, 1);
-                    }
+                    const uint32_t d = own ? tm + TM_S : fbuf(j), a = fbuf(j - 1);
+                    const tc::Desc dph = tc::split_desc(tc::make_desc_sw128(sb + PHI + 65536u * b, 16, 1024));
+#pragma unroll
+                    for (int kk = 0; kk < D / 8; ++kk)
+                        tc::mma_tf32_ts_off_w(d, a + 8 * kk, dph, (kk >> 2) * 16384 + (kk & 3) * 32, it128, 1);
                     tc::mma_commit_w(&bar[MDONE + b]);
                 }
             }

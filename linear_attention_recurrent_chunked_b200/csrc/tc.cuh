@@ -166,6 +166,37 @@ __device__ __forceinline__ void mma_bf16_ts_off_w(uint32_t d_tmem, uint32_t a_tm
         "r"(a_tmem), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// Instruction descriptor: kind::tf32 (fp32 bit patterns in shared or tensor memory, read as tf32:
+// the low 13 mantissa bits are dropped), fp32 D, dense, both operands K-major.
+__host__ __device__ constexpr uint32_t make_idesc_tf32(int M, int N) {
+    return (1u << 4)                      // D format: f32
+           | (2u << 7)                    // A format: tf32
+           | (2u << 10)                   // B format: tf32
+           | ((uint32_t)(N >> 3) << 17)   // N / 8
+           | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+// Warp-issued D[tmem] (+)= A[tmem] * B^T, kind::tf32: A is M rows in lanes with one 32-bit element per
+// column (an fp32 accumulator read as it stands; one K = 8 step spans 8 columns from a_tmem), B a
+// shared-memory descriptor base + byte offset. A later MMA is not ordered after this one's reads or
+// writes of tensor memory: wait for its commit before another product writes or reads the same columns.
+__device__ __forceinline__ void mma_tf32_ts_off_w(uint32_t d_tmem, uint32_t a_tmem, Desc b, uint32_t b_off,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b64 bd;\n\t"
+        "mov.b64 bd, {%2, %3};\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b.lo + (b_off >> 4)), "r"(b.hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// fp32 -> tf32 bit pattern rounded to nearest (ties away), so that the tensor core's truncation of
+// the low bits keeps this value.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
 __device__ __forceinline__ void mma_commit_w(uint64_t *mbar) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"
