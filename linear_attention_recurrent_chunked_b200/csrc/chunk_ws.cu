@@ -398,12 +398,25 @@ template <bool raw>
 __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
     k_ws_prep(const __grid_constant__ CUtensorMap tm_k, const float *__restrict__ g, const float *__restrict__ beta,
               const int32_t *__restrict__ cu, int N, int T_tot, int H, uint32_t *__restrict__ err,
-              const int32_t *__restrict__ chunk_off, uint8_t *__restrict__ rec) {
+              int32_t *__restrict__ chunk_off, uint8_t *__restrict__ rec, int32_t *__restrict__ seg_off,
+              int seg_chunks) {
     extern __shared__ __align__(1024) uint8_t smem[];
     // Equal lengths (no cu_seqlens): item positions are arithmetic, so the first item's loads, its
-    // K K^T product and its scalars run before this grid waits for the plan (which writes nothing
-    // prep reads then; the wait comes before the first dependent launch and before any error bit).
+    // K K^T product and its scalars run before this grid waits for the preceding work on the stream
+    // (the wait comes before the first dependent launch and before any workspace write). There is
+    // no plan kernel then: the host clears the error word and the flags, and block 0 writes the
+    // segment and chunk offsets the later passes read before it lets them launch.
     const bool fixed = cu == nullptr;
+    auto plan_fixed = [&]() {  // block 0, equal lengths: seg_off[0..N], chunk_off[0..N]
+        const int nc = (T_tot / N + C - 1) / C;
+        const int ns = seg_chunks > 0 ? max(1, (nc + seg_chunks - 1) / seg_chunks) : 1;
+        for (int n = threadIdx.x; n <= N; n += blockDim.x) {
+            if (seg_off) seg_off[n] = n * ns;
+            chunk_off[n] = n * nc;
+        }
+        __threadfence();
+        __syncthreads();
+    };
     if (!fixed) {
         griddep_wait();
         griddep_launch();
@@ -419,6 +432,7 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
     const uint32_t sb = tc::smem_u32(smem);
     if (sb & 1023u) {
         griddep_wait();
+        if (fixed && blockIdx.x == 0) plan_fixed();
         if (tid == 0) atomicOr(err, ERRBIT_INTERNAL);
         return;
     }
@@ -548,6 +562,7 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         }
         if (fixed && it == 0) {
             griddep_wait();
+            if (blockIdx.x == 0) plan_fixed();
             griddep_launch();
         }
         ok = tc::mbar_wait(&bars[2], (uint32_t)(it & 1));
@@ -1679,12 +1694,25 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
             S0 = reinterpret_cast<const float *>(wsb + l.s0copy);
         }
     }
-    *stage = "plan";
-    void *pr = prof_start("ws_plan", st);
+    // The plan: a kernel that validates cu_seqlens and writes the offsets; with equal lengths (no
+    // cu_seqlens) one memset clears the error word, the offsets and the flags, and the prep
+    // kernel's block 0 writes the offsets.
     const int nflags = seg_chunks > 0 ? 2 * l.nslots * H + 2 : 0;
-    k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
-    prof_stop(pr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const bool plan_in_prep = cu == nullptr && T_tot > 0;
+    void *pr = nullptr;
+    if (plan_in_prep) {
+        *stage = "plan (memset)";
+        pr = prof_start("ws_plan", st);
+        e = cudaMemsetAsync(wsb, 0, l.flags + (size_t)nflags * sizeof(uint32_t), st);
+        prof_stop(pr);
+        if (e != cudaSuccess) return e;
+    } else {
+        *stage = "plan";
+        pr = prof_start("ws_plan", st);
+        k_ws_plan<<<1, 256, 0, st>>>(cu, N, T_tot, seg_chunks, err, seg_off, chunk_off, flags, nflags);
+        prof_stop(pr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     if (T_tot == 0 && seg_chunks == 0) {
         // nothing to prepare; the output pass still writes S_T = S0
     } else {
@@ -1696,7 +1724,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
         const int grid = (int)std::max(1L, std::min(items_bound, (long)pp::CTAS_PER_SM * num_sms()));
         pr = prof_start("ws_prep", st);
         e = launch_pdl(prep_kernel, dim3(grid), dim3(256), pp::TOTAL, st, tm_k, g, beta, cu, N, T_tot, H, err,
-                       (const int32_t *)chunk_off, rec);
+                       chunk_off, rec, seg_chunks > 0 ? seg_off : nullptr, seg_chunks);
         prof_stop(pr);
         if (e != cudaSuccess) return e;
     }
