@@ -222,7 +222,10 @@ def gpu_arm(args):
         flush_buf.random_(0, 255)  # writes 256 MiB: evicts the 126 MB L2
 
     def dev_inputs(w):
-        return {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in w.items()}
+        t = {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in w.items()}
+        if t.get("N") == 1 and "cu_seqlens" in t:
+            t["cu_seqlens"] = None  # one sequence: the equal-length form of the call (no offsets to read)
+        return t
 
     def prefill_call(t, o, S_T):
         return lambda: gdn.chunk_fwd(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], t["cu_seqlens"],
@@ -328,6 +331,8 @@ def gpu_arm(args):
     # e2e: host (pinned) inputs -> device -> chunk_fwd -> host outputs, all inside the events
     host = {k: (w2k[k].pin_memory() if w2k[k] is not None else None) for k in ("q", "k", "v", "g", "beta", "S0",
                                                                               "cu_seqlens")}
+    if w2k["N"] == 1:
+        host["cu_seqlens"] = None  # one sequence: the equal-length form of the call, as in the device-timed loop
     dbuf = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in host.items()}
     o_dev = torch.empty_like(dbuf["v"])
     S_dev = torch.empty((w2k["N"], w2k["H"], w2k["d"], w2k["d"]), dtype=torch.float32, device=dev)
@@ -690,6 +695,8 @@ def case_arm(args):
         name = {"2k": "prefill_2k", "10k": "prefill_10k"}.get(name, name)
         w = make_prefill(name, seed=0)
         t = {k: (v.to(dev) if hasattr(v, "to") else v) for k, v in w.items()}
+        if w["N"] == 1:
+            t["cu_seqlens"] = None  # as the timed arm calls it
         fn = gdn.seq_scan if args.case.startswith("scan_") else gdn.chunk_fwd
         for _ in range(n):
             fn(t["q"], t["k"], t["v"], t["g"], t["beta"], t["S0"], t["cu_seqlens"])

@@ -1702,9 +1702,7 @@ cudaError_t launch_chunk_ws(const bf16 *q, const bf16 *k, const bf16 *v, const f
     void *pr = nullptr;
     if (plan_in_prep) {
         *stage = "plan (memset)";
-        pr = prof_start("ws_plan", st);
         e = cudaMemsetAsync(wsb, 0, l.flags + (size_t)nflags * sizeof(uint32_t), st);
-        prof_stop(pr);
         if (e != cudaSuccess) return e;
     } else {
         *stage = "plan";

@@ -131,6 +131,17 @@ def test_chunk_full_configs(name):
     check(o, S_T, o_ref, S_ref, w["dtype"], name)
 
 
+@pytest.mark.parametrize("name", ["prefill_2k", "prefill_10k"])
+def test_chunk_full_configs_equal_length_form(name):
+    """The single-sequence workloads called without cu_seqlens (the form bench.py times): no plan
+    kernel, offsets written by the prep kernel, item positions computed arithmetically."""
+    w = make_prefill(name, seed=0)
+    dw = to_dev(w)
+    o, S_T = gdn.chunk_fwd(dw["q"], dw["k"], dw["v"], dw["g"], dw["beta"], dw["S0"], None, N=1, check=True)
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, w["dtype"], name + " (equal-length form)")
+
+
 @pytest.mark.parametrize("T1", [64, 100])
 def test_chunk_resume_from_state(T1):
     """Running [0, T) equals running [0, T1) then [T1, T) from S_T1 (on and off a chunk boundary)."""
