@@ -62,20 +62,29 @@ struct Ctl {
     uint32_t tmem, abort;
 };
 
-__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
-    if (tc::mbar_try_wait(bar, parity)) return true;
+// The timeout branch of wait_bar: sets the error word and aborts the CTA.
+__device__ __noinline__ void wait_bar_timed_out(Ctl *ctl, uint32_t *err) {
+    if (err) atomicOr(err, ERRBIT_TIMEOUT);
+    *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+}
+// Bounded wait for the phase `parity` of an mbarrier; gives up when another role has aborted, or
+// after kWaitNs. The first test is inlined, the polling loop is a call (as a call the whole wait cost
+// some 400 cycles even for a completed phase).
+__device__ __noinline__ bool wait_bar_poll(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
     const uint64_t t0 = tc::globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0) {
             if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
             if (tc::globaltimer() - t0 > kWaitNs) {
-                if (err) atomicOr(err, ERRBIT_TIMEOUT);
-                *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+                wait_bar_timed_out(ctl, err);
                 return false;
             }
         }
     }
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    return tc::mbar_try_wait(bar, parity) || wait_bar_poll(bar, parity, ctl, err);
 }
 // wait_bar for a warp that issues MMAs as a whole (tc::*_w): every lane waits (converged), so that
 // the warp stays converged for the elected issue.

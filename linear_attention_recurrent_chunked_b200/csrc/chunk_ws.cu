@@ -107,23 +107,34 @@ __device__ __forceinline__ void record_timeout_site(uint32_t *err, uint32_t what
         err[3] = threadIdx.x | (parity << 16);
     }
 }
+// The timeout branch of wait_bar: sets the error word, records the site and aborts the CTA.
+__device__ __noinline__ void wait_bar_timed_out(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    atomicOr(err, ERRBIT_TIMEOUT);
+    record_timeout_site(err, 1u + tc::smem_u32(bar), parity);
+    *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+}
 // Bounded wait for the phase `parity` of an mbarrier. Gives up when another
 // role has aborted, or after kWaitNs (then it records the timeout and aborts).
-__device__ __noinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
-    if (tc::mbar_try_wait(bar, parity)) return true;
+// The first test is inlined into every caller and the polling loop is a call:
+// made a call as a whole, the wait cost the calling warp some 400 cycles even
+// for a phase that had already completed, on the chain of every chunk; inlined
+// as a whole, the larger code of the many wait sites made the output pass
+// slower.
+__device__ __noinline__ bool wait_bar_poll(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
     const uint64_t t0 = tc::globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (tc::mbar_try_wait(bar, parity)) return true;
         if ((i & 15u) == 0) {
             if (*reinterpret_cast<volatile uint32_t *>(&ctl->abort)) return false;
             if (tc::globaltimer() - t0 > kWaitNs) {
-                atomicOr(err, ERRBIT_TIMEOUT);
-                record_timeout_site(err, 1u + tc::smem_u32(bar), parity);
-                *reinterpret_cast<volatile uint32_t *>(&ctl->abort) = 1u;
+                wait_bar_timed_out(bar, parity, ctl, err);
                 return false;
             }
         }
     }
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, Ctl *ctl, uint32_t *err) {
+    return tc::mbar_try_wait(bar, parity) || wait_bar_poll(bar, parity, ctl, err);
 }
 // wait_bar for a warp that issues MMAs as a whole (tc::*_w): every lane waits (converged), so that
 // the warp stays converged for the elected issue.
