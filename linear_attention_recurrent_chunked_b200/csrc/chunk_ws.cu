@@ -41,12 +41,15 @@
 // mbarriers, so that the next chunk's loads and operand preparation and the
 // current chunk's outputs overlap the dependent state step:
 //   loader (1 thread)  K, Q, V by TMA (128-byte swizzle), the record by bulk copy
-//   MMA    (1 or 3 threads) every tcgen05.mma; the state step's MMAs are issued
+//   MMA    (1 or 3 warps) every tcgen05.mma; the state step's MMAs are issued
 //                      as soon as their inputs are ready, the rest fills in after
-//   state  (8 warps)   Delta^T (accumulated onto U^T in TMEM) -> bf16 tile;
+//   state  (8 warps)   Delta^T (accumulated onto U^T in TMEM) -> bf16 tile (in
+//                      k_ws_trans with its columns scaled by e, Delta^T diag(e));
 //                      S -> bf16 tile and S <- gamma_C' S in TMEM, so that the
 //                      next update accumulates onto it (two threads per row)
-//   prep   (8 / 4 warps) T1 from T2; -W from W^T; P from X1 = Q K^T; K <- diag(e) K in place
+//   prep   (8 / 4 warps) T1 from T2; -W from W^T; P from X1 = Q K^T and
+//                      K <- diag(e) K in place (k_ws_out, where the Delta^T tile
+//                      also feeds the outputs and stays unscaled)
 //   output (4 warps)   gamma_r O1 + O2 -> bf16 rows -> TMA store   (k_ws_out)
 //   X-state (8 warps)  the Phi chain                               (k_ws_trans)
 // Every wait is bounded in time; a timeout sets the error word and makes all
@@ -274,6 +277,25 @@ __device__ __forceinline__ void tile32_epilogue(uint32_t tile, uint32_t taddr, i
     tc::tmem_ld32(taddr, x);
 #pragma unroll
     for (int i = 0; i < 32; ++i) x[i] *= scale;
+#pragma unroll
+    for (int i = 0; i < 32; i += 8) st_run8(tile + tc::tile_off(row, col0 + i, 128, 2048), x + i);
+}
+
+// tile32_epilogue with column j scaled by cs[j] (times cs2[j] where cs2 is given) instead of a
+// constant: the transition pass's Delta^T diag(e) tiles.
+__device__ __forceinline__ void tile32_epilogue_cs(uint32_t tile, uint32_t taddr, int row, int col0, const float *cs,
+                                                   const float *cs2) {
+    float x[32];
+    tc::tmem_ld32(taddr, x);
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        float4 f = *reinterpret_cast<const float4 *>(cs + col0 + i);
+        if (cs2) {
+            const float4 f2 = *reinterpret_cast<const float4 *>(cs2 + col0 + i);
+            f.x *= f2.x; f.y *= f2.y; f.z *= f2.z; f.w *= f2.w;
+        }
+        x[i] *= f.x; x[i + 1] *= f.y; x[i + 2] *= f.z; x[i + 3] *= f.w;
+    }
 #pragma unroll
     for (int i = 0; i < 32; i += 8) st_run8(tile + tc::tile_off(row, col0 + i, 128, 2048), x + i);
 }
@@ -1031,26 +1053,25 @@ enum {
     WUF = 10, M3S = 11, M4S = 12, M3X = 13, M4X = 14,
     T1R = 15,   // T1 tile written (prep, 128)
     WR = 16,    // -W tile written (prep, 128)
-    KR = 17,    // [4] diag(e) K written (prep, 128)
-    SR = 21,    // S state (256)
-    XR = 22,    // X state (256)
-    DSR = 23,   // [2] Delta_S^T tile written (S state, 256)
-    DXR = 25,   // X state (256)
-    FIN = 26,   // every MMA of the S issuer done (drained before TMEM is freed)
-    FINX = 27,  // the same for the X issuer
-    FINW = 28,  // the same for the W issuer
+    SR = 17,    // S state (256)
+    XR = 18,    // X state (256)
+    DSR = 19,   // [2] Delta_S^T diag(e) tile written (S state, 256)
+    DXR = 21,   // X state (256)
+    FIN = 22,   // every MMA of the S issuer done (drained before TMEM is freed)
+    FINX = 23,  // the same for the X issuer
+    FINW = 24,  // the same for the W issuer
     // link phase, fold step j (buffer j & 1 where there are two)
-    A1R = 29,     // F(0), the first segment's end state, is in TMEM (S warps, 256)
-    AREADY = 30,  // [2] F(j) holds S_loc(j) (S and X warps, 512)
-    PUBD = 32,    // the part has been read out of TMEM (X warps, 256)
-    PFULL = 33,   // [2] Phi_j landed
-    MDONE = 35,   // [2] the step's MMAs are done
-    NBAR = 37
+    A1R = 25,     // F(0), the first segment's end state, is in TMEM (S warps, 256)
+    AREADY = 26,  // [2] F(j) holds S_loc(j) (S and X warps, 512)
+    PUBD = 28,    // the part has been read out of TMEM (X warps, 256)
+    PFULL = 29,   // [2] Phi_j landed
+    MDONE = 31,   // [2] the step's MMAs are done
+    NBAR = 33
 };
 // (EMPTYK takes a commit from each issuer: count 2 with an X chain, 1 without.)
 __device__ __forceinline__ constexpr uint32_t bar_count(int i, bool has_x) {
     return (i >= EMPTYK && i < EMPTYK + 3)                                  ? (has_x ? 2u : 1u)
-           : (i >= T1R && i < KR + 4)                                       ? 128u
+           : (i == T1R || i == WR)                                          ? 128u
            : (i >= SR && i <= DXR)                                          ? 256u
            : (i == A1R || i == PUBD)                                        ? 256u
            : (i == AREADY || i == AREADY + 1)                               ? 512u
@@ -1225,9 +1246,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 for (int kk = 0; kk < D / 16; ++kk)
                     tc::mma_bf16_off_w(tm + TM_U + 64 * b, ds, kk * 4096, dw, kk * 256, id_km64, 1);
                 tc::mma_commit_w(&bar[M3S]);
-                // S <- gamma_C S + Delta_S^T (diag(e) K)
+                // S <- gamma_C S + (Delta_S^T diag(e)) K (K as loaded: the tile's columns carry e)
                 if (!(ok = wait_bar_w(&bar[DSR + b], (uint32_t)((c >> 1) & 1), ctl, err) &&
-                           wait_bar_w(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                           wait_bar_w(&bar[FULLK + c % 3], kpar(c), ctl, err)))
                     break;
                 tc::fence_after_sync();
 #pragma unroll
@@ -1256,9 +1277,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 for (int kk = 0; kk < D / 16; ++kk)
                     tc::mma_bf16_off_w(tm + TM_DX, dx, kk * 4096, dw, kk * 256, id_km64, kk > 0);
                 tc::mma_commit_w(&bar[M3X]);
-                // X <- gamma_C X + X (-W)^T diag(e) K
-                if (!(ok = wait_bar_w(&bar[DXR], par, ctl, err) &&
-                           wait_bar_w(&bar[KR + (c & 3)], (uint32_t)((c >> 2) & 1), ctl, err)))
+                // X <- gamma_C X + (X (-W)^T diag(e)) K
+                if (!(ok = wait_bar_w(&bar[DXR], par, ctl, err) && wait_bar_w(&bar[FULLK + c % 3], kpar(c), ctl, err)))
                     break;
                 tc::fence_after_sync();
 #pragma unroll
@@ -1288,7 +1308,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             for (int c = 0; ok && c < nch; ++c) {
                 if (!(ok = wait_bar(b_m3, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
-                tile32_epilogue(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * (c & 1)) + 32 * half, v, 32 * half, 1.f);
+                // Delta^T diag(e) (raw inputs: times the keys' 1 / ||k||), so that the update reads K as loaded
+                tile32_epilogue_cs(dt_tile, tl + (is_x ? TM_DX : TM_U + 64 * (c & 1)) + 32 * half, v, 32 * half,
+                                   vecp(c) + 128, raw ? vecp(c) + 192 : nullptr);
                 handoff(&bar[is_x ? DXR : DSR + (c & 1)]);
                 if (!(ok = wait_bar(b_m4, (uint32_t)(c & 1), ctl, err))) break;
                 tc::fence_after_sync();
@@ -1312,7 +1334,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             if (!(ok = wait_bar(&bar[FULLK + c % 3], kpar(c), ctl, err) &&
                        wait_bar(&bar[FULLV + (c & 1)], vpar(c), ctl, err)))
                 break;
-            // (raw inputs: the keys' 1 / ||k|| from the record is folded into T1 and diag(e) K)
+            // (raw inputs: the keys' 1 / ||k|| from the record is folded into T1 here and into the
+            // Delta tiles' column scales)
             make_t1(smem + T1, smem + vslot(c) + VS_T2, vecp(c) + 64, t128, 128, raw ? vecp(c) + 192 : nullptr);
             tc::fence_smem_to_async();
             tc::mbar_arrive(&bar[T1R]);
@@ -1325,10 +1348,6 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             tile32_epilogue(sb + W, tl + TM_WT, k, 0, -1.f);
             tile32_epilogue(sb + W, tl + TM_WT + 32, k, 32, -1.f);
             handoff(&bar[WR]);
-            scale_rows_sw128(smem + kslot(c) + KS_K, vecp(c) + 128, t128, 128,
-                             raw ? vecp(c) + 192 : nullptr);  // W^T has read K
-            tc::fence_smem_to_async();
-            tc::mbar_arrive(&bar[KR + (c & 3)]);
         }
     }
     // ---------------------------------------------------------------- link (all threads)
