@@ -13,8 +13,10 @@
 //
 // Steps 2 and 3 are 16-row-granular products, below the M = 64 minimum of
 // tcgen05.mma, so they use warp-level mma.sync m16n8k8 with tf32 operands and
-// fp32 accumulation (operand rounding 2^-11, below the bf16 rounding the
-// solve's result receives when it becomes an MMA operand).
+// fp32 accumulation. The fp32 values go in as they are, with no rounding
+// instruction: the tensor cores take them at tf32 precision (relative error at
+// most 2^-10, that of truncation), under the bf16 rounding the solve's result
+// receives when it becomes an MMA operand.
 #pragma once
 
 #include <stdint.h>
@@ -26,11 +28,7 @@ constexpr int AP = 68;   // pitch of A and T: rows 16-byte aligned; 8 consecutiv
                          // mma fragment patterns (4 g + t) hit distinct banks
 constexpr int XP = 40;   // pitch of the product scratch
 
-__device__ __forceinline__ uint32_t tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+__device__ __forceinline__ uint32_t tf32(float x) { return __float_as_uint(x); }
 
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
     asm volatile(
@@ -65,8 +63,8 @@ __device__ __forceinline__ void warp_store(float *Z, int p, const float (&d)[4],
 // Block-wide solve; requires blockDim.x == 256. A, T: [64][AP] fp32 in shared
 // memory, 16-byte aligned (A zero on and above the diagonal). X: scratch of 32 * XP floats.
 // T may be the same buffer as A: every block of A is read (and the reads
-// synchronised) before the block of T at its place is written. Ends with a
-// __syncthreads.
+// synchronised) before the block of T at its place is written, and T's blocks
+// above the diagonal are then A's zeros already. Ends with a __syncthreads.
 __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // ---- 1. diagonal blocks (warps 0-3) and the zero upper blocks (warps 4-7)
@@ -76,24 +74,25 @@ __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                // row i of the block in 16-byte broadcast loads (rows are 16-byte aligned: AP % 4 == 0)
+                // row i of the block in 16-byte broadcast loads (rows are 16-byte aligned: AP % 4 == 0);
+                // four partial sums, so that the dependent chain of a row is a quarter as long
                 const float *arow = A + (o + i) * AP + o;
-                float acc = (i == j) ? 1.f : 0.f;
+                float acc[4] = {(i == j) ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int s4 = 0; s4 < i; s4 += 4) {
                     const float4 a4 = *reinterpret_cast<const float4 *>(arow + s4);
-                    acc = fmaf(-a4.x, x[s4], acc);
-                    if (s4 + 1 < i) acc = fmaf(-a4.y, x[s4 + 1], acc);
-                    if (s4 + 2 < i) acc = fmaf(-a4.z, x[s4 + 2], acc);
-                    if (s4 + 3 < i) acc = fmaf(-a4.w, x[s4 + 3], acc);
+                    acc[0] = fmaf(-a4.x, x[s4], acc[0]);
+                    if (s4 + 1 < i) acc[1] = fmaf(-a4.y, x[s4 + 1], acc[1]);
+                    if (s4 + 2 < i) acc[2] = fmaf(-a4.z, x[s4 + 2], acc[2]);
+                    if (s4 + 3 < i) acc[3] = fmaf(-a4.w, x[s4 + 3], acc[3]);
                 }
-                x[i] = acc;
+                x[i] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
             __syncwarp(0x0000ffffu);  // every lane has read its block of A before T overwrites it (A may be T)
 #pragma unroll
             for (int i = 0; i < 16; ++i) T[(o + i) * AP + o + j] = x[i];
         }
-    } else {
+    } else if (A != T) {
         for (int e = tid - 128; e < 6 * 256; e += 128) {
             const int b = e >> 8, ri = (e >> 4) & 15, cj = e & 15;
             const int bi = (b < 3) ? 0 : (b < 5 ? 1 : 2);
