@@ -513,15 +513,16 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         tc::tma_load_3d(sb + pp::K0, &tm_k, &bars[0], 0, h, cs);
         tc::tma_load_3d(sb + pp::K0 + 8192u, &tm_k, &bars[0], 64, h, cs);
     };
-    auto issue = [&](int w, int b) {  // g, beta
+    auto issue = [&](int w, int b) {  // g, beta (warp 0; lane l: rows 2 l, 2 l + 1)
         int h, cs, L, gc;
         locate(w, h, cs, L, gc);
-        if (tid < 2 * C) {
-            const int r = tid & 63;
+        const int lane = tid & 31;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int r = 2 * lane + (q & 1);
             const bool ok = r < L;
             const size_t off = (size_t)(cs + (ok ? r : 0)) * H + h;
-            cp_async4(sb + pp::RAW + b * 512u + (tid < C ? 0u : 256u) + 4u * r, (tid < C ? g : beta) + off,
-                      ok ? 4u : 0u);
+            cp_async4(sb + pp::RAW + b * 512u + (q < 2 ? 0u : 256u) + 4u * r, (q < 2 ? g : beta) + off, ok ? 4u : 0u);
         }
         cp_async_commit();
     };
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
     const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
     bool ok = true;
     if (tid == 32) issue_k(blockIdx.x);
-    issue(blockIdx.x, 0);
+    if (warp == 0) issue(blockIdx.x, 0);
     int it = 0;
     for (int w = blockIdx.x; w < items; w += gridDim.x, ++it) {
         const int b = it & 1;
@@ -552,42 +553,49 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
             }
             tc::mma_commit(&bars[2]);
         }
-        if (wn < items) {
-            issue(wn, b ^ 1);
-            cp_async_wait_1();
-        } else {
-            cp_async_wait_all();
-        }
-        __syncthreads();
-        // ---- scalars: G = cumsum(g) (log2 units), gamma, e, beta. Raw inputs: g = -softplus(a),
-        // beta = sigmoid(b) from the logits, zero past the chunk's valid length L
-        const float *graw = reinterpret_cast<const float *>(smem + pp::RAW + b * 512u);
-        int L_item = C;
-        if (raw) {
-            int h_, cs_, gc_;
-            locate(w, h_, cs_, L_item, gc_);
-        }
-        if (tid < 32) {
-            float x0 = graw[2 * tid], x1 = graw[2 * tid + 1];
+        // ---- scalars, by warp 0 alone (lane l: rows 2 l, 2 l + 1, from the g, beta it fetched itself):
+        // G = cumsum(g) (log2 units), gamma, e, beta. Raw inputs: g = -softplus(a), beta = sigmoid(b)
+        // from the logits, zero past the chunk's valid length L. (The previous item's readers of these
+        // vectors are behind its last __syncthreads; the first readers of this item's come after the
+        // barrier below that waits for the product.)
+        if (warp == 0) {
+            if (wn < items) {
+                issue(wn, b ^ 1);
+                cp_async_wait_1();
+            } else {
+                cp_async_wait_all();
+            }
+            const int lane = tid & 31;
+            const float *graw = reinterpret_cast<const float *>(smem + pp::RAW + b * 512u);
+            int L_item = C;
             if (raw) {
-                x0 = 2 * tid < L_item ? neg_softplus(x0) : 0.f;
-                x1 = 2 * tid + 1 < L_item ? neg_softplus(x1) : 0.f;
+                int h_, cs_, gc_;
+                locate(w, h_, cs_, L_item, gc_);
+            }
+            float x0 = graw[2 * lane], x1 = graw[2 * lane + 1];
+            float b0 = graw[64 + 2 * lane], b1 = graw[64 + 2 * lane + 1];
+            if (raw) {
+                x0 = 2 * lane < L_item ? neg_softplus(x0) : 0.f;
+                x1 = 2 * lane + 1 < L_item ? neg_softplus(x1) : 0.f;
+                b0 = 2 * lane < L_item ? sigmoid_f(b0) : 0.f;
+                b1 = 2 * lane + 1 < L_item ? sigmoid_f(b1) : 0.f;
             }
             const float a = x0 * kLog2e, b2 = a + x1 * kLog2e;
             float sc = b2;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, sc, off);
-                if (tid >= off) sc += y;
+                if (lane >= off) sc += y;
             }
-            Gl[2 * tid] = sc - b2 + a;
-            Gl[2 * tid + 1] = sc;
-        }
-        __syncthreads();
-        if (tid < C) {
-            gam[tid] = ex2(Gl[tid]);
-            dte[tid] = ex2(Gl[C - 1] - Gl[tid]);
-            bet[tid] = raw ? (tid < L_item ? sigmoid_f(graw[64 + tid]) : 0.f) : graw[64 + tid];
+            const float G0 = sc - b2 + a, G1 = sc, GC = __shfl_sync(0xffffffffu, sc, 31);
+            Gl[2 * lane] = G0;
+            Gl[2 * lane + 1] = G1;
+            gam[2 * lane] = ex2(G0);
+            gam[2 * lane + 1] = ex2(G1);
+            dte[2 * lane] = ex2(GC - G0);
+            dte[2 * lane + 1] = ex2(GC - G1);
+            bet[2 * lane] = b0;
+            bet[2 * lane + 1] = b1;
         }
         if (raw) {  // key norms from the landed K tile (read before the next item's K can be loaded)
             tc::mbar_wait(&bars[0], (uint32_t)(it & 1));

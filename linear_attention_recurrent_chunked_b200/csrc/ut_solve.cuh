@@ -101,17 +101,18 @@ __device__ __forceinline__ void solve64(const float *A, float *T, float *X) {
         }
     }
     __syncthreads();
-    // ---- 2. blocks (1,0) and (3,2): X_b = A_ij T_jj, then T_ij = -T_ii X_b (warps 0-3: block b = w/2, n-tile w%2)
+    // ---- 2. blocks (1,0) and (3,2): X_b = A_ij T_jj, then T_ij = -T_ii X_b (warps 0-3: block b = w/2, n-tile w%2).
+    // A warp's second product reads back only its own 16 x 8 tile of X_b; the two warps of a block
+    // meet (named barrier 2 + b, 64 threads) so that both have read A_ij before T_ij overwrites it.
     if (warp < 4) {
         const int b = warp >> 1, nt = warp & 1, i = 1 + 2 * b, j = i - 1;
         float d[4];
         warp_mm(d, A + (16 * i) * AP + 16 * j, AP, T + (16 * j) * AP + 16 * j + 8 * nt, AP, 16);
         warp_store(X + b * 16 * XP + 8 * nt, XP, d, 1.f);
-    }
-    __syncthreads();
-    if (warp < 4) {
-        const int b = warp >> 1, nt = warp & 1, i = 1 + 2 * b, j = i - 1;
-        float d[4];
+        if (b == 0)
+            asm volatile("bar.sync 2, 64;" ::: "memory");
+        else
+            asm volatile("bar.sync 3, 64;" ::: "memory");
         warp_mm(d, T + (16 * i) * AP + 16 * i, AP, X + b * 16 * XP + 8 * nt, XP, 16);
         warp_store(T + (16 * i) * AP + 16 * j + 8 * nt, AP, d, -1.f);
     }
