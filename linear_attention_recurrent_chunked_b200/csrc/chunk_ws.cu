@@ -614,18 +614,13 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         }
         if (tid == 32 && wn < items) issue_k(wn);  // the product has read the K buffer
         // ---- A_rs = beta_r exp(G_r - G_s) X1_rs for s < r (warp w: rows 16 (w%4) + lane % 16, columns
-        // 32 (w/4) + 16 (lane / 16) ..: the accumulator rows sit in lanes 0-15, whose upper 16 columns
-        // lanes 16-31 take over by shuffle)
+        // 32 (w/4) + 16 (lane / 16) ..: the accumulator rows sit in lanes 0-15 of the quarter; lanes
+        // 16-31 read the same rows' next 16 columns)
         {
             const int lane = tid & 31, l16 = lane & 15, hf = lane >> 4;
             const int r = 16 * (warp & 3) + l16, c0 = 32 * (warp >> 2) + 16 * hf;
-            float x[32];
-            tc::tmem_ld32(tl + 32 * (warp >> 2), x);  // warp-wide; lanes >= 16 receive nothing of use
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float y = __shfl_sync(0xffffffffu, x[16 + i], l16);
-                x[i] = hf ? y : x[i];
-            }
+            float x[16];
+            tc::tmem_ld16_split16(tl + 32 * (warp >> 2), x);
             // (raw inputs: X1 holds raw k_r . k_s, scaled here by 1 / (||k_r|| ||k_s||); otherwise by 1)
             const float Gr = Gl[r], br = bet[r] * rnv[r];
 #pragma unroll

@@ -354,6 +354,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
     for (int i = 0; i < 32; ++i) r[i] = __uint_as_float(u[i]);
 }
 
+// TMEM -> registers for an M = 64 accumulator, whose rows sit in the first 16 lanes of each warp's
+// quarter: shape 16x32bx2, threads 0-15 read lanes 0-15 of the quarter at columns [c, c + 16) and
+// threads 16-31 the same lanes at columns [c + 16, c + 32) (the half-split offset), 16 values each.
+__device__ __forceinline__ void tmem_ld16_split16(uint32_t taddr, float (&r)[16]) {
+    uint32_t u[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(u[i]);
+}
+
 // The same load without the wait, and the wait that ties the loaded registers to
 // it (the "+r" operands keep every use of them after the wait).
 __device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&u)[32]) {
