@@ -316,6 +316,15 @@ def test_segmented_slow_decay_stress():
     check(o, S_T, o_ref, S_ref, "bf16", "segmented stress")
 
 
+def test_long_sequence_many_segments_long_fold():
+    """One long sequence on one head: ~24 segments, so the last segment folds ~22 published parts
+    (tf32 products) onto the first segment's end state; slow decay keeps the early state alive."""
+    w = make_prefill("prefill_2k", seqlens=[24576], H=1, s0=True, stress=True, seed=61)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "24 segments, long fold")
+
+
 def test_medium_workspace_falls_back_correctly():
     """Workspaces between the error word and the preferred size select a plan that fits."""
     w = make_prefill("prefill_2k", seqlens=[1500], H=2, s0=True, stress=True, seed=24)
