@@ -14,14 +14,16 @@
 // product runs on bf16 operands with fp32 accumulation and the scale is applied to the fp32
 // result: the dequantisation is exact and the weights cross HBM as int8 (half the bytes of bf16).
 //
-// One persistent CTA per SM walks output tiles of 128 tokens x BN channels (BN = 256, or 128 / 64
-// when there are too few tiles to fill the GPU, as for one decode step), K steps of 64:
+// One persistent CTA per SM walks output tiles of MT x 128 tokens x BN channels, K steps of 64:
+// at prefill sizes MT = 2, BN = 128 (each converted weight tile serves two token tiles, halving the
+// conversion per product), else MT = 1 and BN = 256, or 128 / 64 when there are too few tiles to
+// fill the GPU (as for one decode step):
 //   loaders   (2 threads)  TMA: x tiles (bf16, 128-byte swizzle) and int8 weight tiles, two 4-deep
 //                          rings, freed by the MMAs and by the converters respectively
 //   convert   (8 warps)    int8 tile -> bf16 K-major 128-byte-swizzled operand tile, 3-deep ring
 //                          (exact, on integer and fp32 pipes: codes_to_bf16x4)
-//   MMA       (1 thread)   4 tcgen05.mma (M=128, N=BN, K=16) per K step into a TMEM accumulator
-//                          (two accumulators of BN columns: one tile's epilogue overlaps the next)
+//   MMA       (1 warp)     4 tcgen05.mma (M=128, N=BN, K=16) per K step and token tile into a TMEM
+//                          accumulator (two sets of MT x BN columns: one tile's epilogue overlaps the next)
 //   epilogue  (4 warps)    TMEM -> fp32 registers -> * scale -> bf16 / fp32 rows in global memory
 // Every wait is bounded in time; a timeout sets the error word and all roles leave their loops.
 #include <cuda.h>
@@ -42,8 +44,8 @@ constexpr int BM = 128, BK = 64;
 constexpr int NBSLOT = 3;
 // ring depth of the x and int8 stages: deeper for the narrow tiles of small T, where each CTA's
 // K loop is a chain of load latencies rather than of products
-template <int BN>
-constexpr int nstage() { return BN >= 256 ? 4 : BN >= 128 ? 6 : 8; }
+template <int BN, int MT>
+constexpr int nstage() { return MT > 1 ? 4 : BN >= 256 ? 4 : BN >= 128 ? 6 : 8; }
 constexpr int NSTAGE_MAX = 8;
 constexpr uint64_t kWaitNs = 1000000000ull;
 constexpr int NCONV = 256;                       // converter threads (8 warps)
@@ -66,16 +68,19 @@ __host__ __device__ constexpr uint32_t bar_count(int i) {
            : (i >= AEMPTY && i < AEMPTY + 2) ? 128u : 1u;
 }
 
-// Shared-memory layout for a channel tile of BN (x: 128 x 64 bf16; w8: BN x 64 int8; bf16 weight tile BN x 64).
-template <int BN>
+// Shared-memory layout for a tile of MT x 128 tokens and BN channels (x: MT x 128 x 64 bf16; w8: BN x 64
+// int8; bf16 weight tile BN x 64).
+template <int BN, int MT>
 struct Lay {
-    static constexpr int NSTAGE = nstage<BN>();
-    static constexpr uint32_t A_BYTES = BM * BK * 2, W8_BYTES = BN * BK, B_BYTES = BN * BK * 2;
+    static constexpr int NSTAGE = nstage<BN, MT>();
+    static constexpr uint32_t A_BYTES = MT * BM * BK * 2, W8_BYTES = BN * BK, B_BYTES = BN * BK * 2;
     static constexpr uint32_t OFF_A = 0, OFF_W8 = OFF_A + NSTAGE * A_BYTES, OFF_B = OFF_W8 + NSTAGE * W8_BYTES;
     static constexpr uint32_t OFF_BAR = OFF_B + NBSLOT * B_BYTES, OFF_CTL = OFF_BAR + 8 * NBAR;
     static constexpr uint32_t TOTAL = OFF_CTL + 16 + 1024;  // + slack for the 1024-byte alignment
 };
-static_assert(Lay<256>::TOTAL <= 232448 && Lay<128>::TOTAL <= 232448 && Lay<64>::TOTAL <= 232448, "shared memory");
+static_assert(Lay<256, 1>::TOTAL <= 232448 && Lay<128, 1>::TOTAL <= 232448 && Lay<64, 1>::TOTAL <= 232448 &&
+                  Lay<128, 2>::TOTAL <= 232448,
+              "shared memory");
 
 struct Ctl {
     uint32_t tmem, abort;
@@ -143,12 +148,13 @@ struct Route {
     int Hdk, Hdv, H, N;
 };
 
-template <int BN>
+template <int BN, int MT>
 __global__ void __launch_bounds__(NTHREADS, 1)
     k_proj_w8(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
               const float *__restrict__ scale, int T, int D, Route rt, bf16_t *__restrict__ q, bf16_t *__restrict__ k,
               bf16_t *__restrict__ v, float *__restrict__ ga, float *__restrict__ gb, uint32_t *__restrict__ err) {
-    using L = Lay<BN>;
+    using L = Lay<BN, MT>;
+    constexpr uint32_t TMEM_COLS = 2 * MT * BN < 32 ? 32 : 2 * MT * BN;
     constexpr int NSTAGE = L::NSTAGE;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = tc::smem_u32(smem_raw);
@@ -157,7 +163,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L::OFF_BAR);
     Ctl *ctl = reinterpret_cast<Ctl *>(smem + L::OFF_CTL);
-    if (warp == 0) tc::tmem_alloc(&ctl->tmem, 2 * BN < 32 ? 32 : 2 * BN);
+    if (warp == 0) tc::tmem_alloc(&ctl->tmem, TMEM_COLS);
     if (tid == 32) {
         for (int i = 0; i < NBAR; ++i) tc::mbar_init(&bar[i], bar_count(i));
         ctl->abort = 0;
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tm = ctl->tmem;
-    const int mt = (T + BM - 1) / BM, nt = (rt.N + BN - 1) / BN, ksteps = D / BK;
+    const int mt = (T + MT * BM - 1) / (MT * BM), nt = (rt.N + BN - 1) / BN, ksteps = D / BK;
     const int ntiles = mt * nt;
 
     if (warp == W_LOAD || warp == W_LOADW) {
@@ -179,7 +185,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             int it = 0, issued = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-                const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+                const int m0 = (tile / nt) * MT * BM, n0 = (tile % nt) * BN;
                 for (int ks = 0; ks < ksteps; ++ks, ++it) {
                     const int s = it % NSTAGE;
                     if (it >= NSTAGE && !(ok = wait_bar(&empty[s], (uint32_t)(((it / NSTAGE) - 1) & 1), ctl, err)))
@@ -215,9 +221,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         break;
                     tc::fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk)
-                        tc::mma_bf16_off_w(tm + acc * BN, da, s * L::A_BYTES + kk * 32, db, bs * L::B_BYTES + kk * 32,
-                                         idesc, (ks > 0 || kk > 0) ? 1u : 0u);
+                    for (int m = 0; m < MT; ++m)
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk)
+                            tc::mma_bf16_off_w(tm + (acc * MT + m) * BN, da, s * L::A_BYTES + m * BM * 128 + kk * 32, db,
+                                               bs * L::B_BYTES + kk * 32, idesc, (ks > 0 || kk > 0) ? 1u : 0u);
                     tc::mma_commit_w(&bar[EMPTY + s]);
                     tc::mma_commit_w(&bar[BEMPTY + bs]);
                 }
@@ -264,21 +272,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue (128 threads)
-        const int row = (warp & 3) * 32 + lane;  // this thread's TMEM lane = token row of the tile
+        const int row = (warp & 3) * 32 + lane;  // this thread's TMEM lane = token row of each token tile
         const uint32_t tl = tm + ((uint32_t)((warp & 3) * 32) << 16);
         int ti = 0;
         bool ok = true;
         for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++ti) {
             const int acc = ti & 1;
-            const int m0 = (tile / nt) * BM, n0 = (tile % nt) * BN;
+            const int m0 = (tile / nt) * MT * BM, n0 = (tile % nt) * BN;
             if (!(ok = __all_sync(0xffffffffu, wait_bar(&bar[AFULL + acc], (uint32_t)((ti >> 1) & 1), ctl, err))))
                 break;
             tc::fence_after_sync();
-            const int t = m0 + row;
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+            for (int cm = 0; cm < MT * BN; cm += 32) {
+                const int m = cm / BN, c0 = cm % BN;
+                const int t = m0 + m * BM + row;
                 float x[32];
-                tc::tmem_ld32(tl + acc * BN + c0, x);
+                tc::tmem_ld32(tl + acc * MT * BN + cm, x);
                 const int n = n0 + c0;
                 if (t >= T || n >= rt.N) continue;
                 if (n + 32 <= rt.N) {
@@ -321,7 +330,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tm, 2 * BN < 32 ? 32 : 2 * BN);
+    if (warp == 0) tc::tmem_dealloc(tm, TMEM_COLS);
 }
 
 }  // namespace
@@ -375,29 +384,23 @@ cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float 
     if ((e = cudaMemsetAsync(err, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
     const int N = H * (2 * dk + dv) + 2 * H;
     if (T == 0) return cudaSuccess;
-    CUtensorMap tm_x;
-    *stage = "TMA descriptor encoding";
-    if ((e = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, BK, BM,
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
-        return e;
     *stage = "proj_w8";
-    // Channel tile: the widest of 256 / 128 / 64 that still gives every SM a tile (small T, e.g.
-    // one decode step, is bound by reading the weights and needs many CTAs to do so).
-    const long mt = (T + BM - 1) / BM;
-    int bn = 64;
-    for (int cand : {256, 128})
-        if (mt * ((N + cand - 1) / cand) >= sm_count()) {
-            bn = cand;
-            break;
-        }
-    auto launch = [&](auto kernel, int BNv, uint32_t smem_bytes) -> cudaError_t {
+    // Tiles: at prefill sizes two token tiles of 128 per tile with 128 channels, when that still
+    // gives every SM a tile; otherwise one token tile and the widest channel tile of 256 / 128 / 64
+    // that does (small T, e.g. one decode step, is bound by reading the weights and needs many CTAs
+    // to do so).
+    const long mt1 = (T + BM - 1) / BM, mt2 = (T + 2 * BM - 1) / (2 * BM);
+    auto launch = [&](auto kernel, int BNv, int MTv, uint32_t smem_bytes) -> cudaError_t {
         cudaError_t ea = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
         if (ea != cudaSuccess) return ea;
-        CUtensorMap tm_w2;
+        CUtensorMap tm_x, tm_w2;
+        ea = encode_2d(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, BK,
+                       BM * MTv, CU_TENSOR_MAP_SWIZZLE_128B);
+        if (ea != cudaSuccess) return ea;
         ea = encode_2d(&tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w, (uint64_t)D, (uint64_t)N, (uint64_t)D, BK, BNv,
                        CU_TENSOR_MAP_SWIZZLE_NONE);
         if (ea != cudaSuccess) return ea;
-        const long tiles = mt * ((N + BNv - 1) / BNv);
+        const long tiles = (MTv > 1 ? mt2 : mt1) * ((N + BNv - 1) / BNv);
         const int grid = (int)std::min<long>(tiles, sm_count());
         void *pr = prof_start("proj_w8", st);
         kernel<<<grid, NTHREADS, smem_bytes, st>>>(tm_x, tm_w2, scale, T, D, Route{H * dk, H * dv, H, N}, q, k, v,
@@ -405,9 +408,19 @@ cudaError_t launch_proj_w8(const __nv_bfloat16 *x, const int8_t *w, const float 
         prof_stop(pr);
         return cudaSuccess;
     };
-    if (bn == 256) e = launch(k_proj_w8<256>, 256, Lay<256>::TOTAL);
-    else if (bn == 128) e = launch(k_proj_w8<128>, 128, Lay<128>::TOTAL);
-    else e = launch(k_proj_w8<64>, 64, Lay<64>::TOTAL);
+    if (mt2 * ((N + 127) / 128) >= sm_count()) {
+        e = launch(k_proj_w8<128, 2>, 128, 2, Lay<128, 2>::TOTAL);
+    } else {
+        int bn = 64;
+        for (int cand : {256, 128})
+            if (mt1 * ((N + cand - 1) / cand) >= sm_count()) {
+                bn = cand;
+                break;
+            }
+        if (bn == 256) e = launch(k_proj_w8<256, 1>, 256, 1, Lay<256, 1>::TOTAL);
+        else if (bn == 128) e = launch(k_proj_w8<128, 1>, 128, 1, Lay<128, 1>::TOTAL);
+        else e = launch(k_proj_w8<64, 1>, 64, 1, Lay<64, 1>::TOTAL);
+    }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

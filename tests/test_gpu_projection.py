@@ -50,6 +50,7 @@ def check(p, got, rows=None):
     (130, 128, 2, 64, 128),   # dk != dv, N = 516
     (1, 64, 1, 8, 8),         # one token, one K step, N = 26
     (513, 320, 3, 40, 24),    # odd head sizes: a 32-column group straddles the q | k and v | a boundaries
+    (3000, 256, 8, 64, 64),   # two token tiles per tile (enough tiles), ragged in tokens and channels (N = 1552)
 ])
 def test_projection_small(T, D, H, dk, dv):
     p = make_projection(T, D, H, dk, dv, seed=T + D)
