@@ -695,15 +695,16 @@ enum {
     M4O = 8,    // O1 and O2 ready
     T1R = 9,    // T1 tile written (prep, 256)
     WR = 10,    // -W tile written (prep, 256)
-    PR = 11,    // P tile and diag(e) K written (prep, 256)
+    PR = 11,    // P tile written, X1 read out (prep, 256)
     DLR = 12,   // Delta^T tile written (state, 256)
     SR = 13,    // S tile written, S scaled in TMEM (state, 256)
     OF = 14,    // O1, O2 read out of TMEM (output, 128)
     FIN = 15,   // every MMA of the CTA done (drained before TMEM is freed)
-    NBAR = 16
+    KR = 16,    // diag(e) K written (prep, 256)
+    NBAR = 17
 };
 __device__ __forceinline__ constexpr uint32_t bar_count(int i) {
-    return i == EMPTY || i == EMPTY + 1 ? 2u : (i >= T1R && i <= SR) ? 256u : i == OF ? 128u : 1u;
+    return i == EMPTY || i == EMPTY + 1 ? 2u : (i >= T1R && i <= SR) || i == KR ? 256u : i == OF ? 128u : 1u;
 }
 }  // namespace ob
 
@@ -800,6 +801,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
         // ---------------------------------------------------------------- MMA issuer
         if (nch > 0) {  // the whole warp, lane 0 issuing
             const uint32_t id_kk64 = tc::make_idesc_bf16(128, 64, 0, 0);
+            const uint32_t id_x1 = tc::make_idesc_bf16(64, 64, 0, 0);
             const uint32_t id_mk64 = tc::make_idesc_bf16(128, 64, 1, 0);
             const uint32_t id_km64 = tc::make_idesc_bf16(128, 64, 0, 1);
             const uint32_t id_km128 = tc::make_idesc_bf16(128, 128, 0, 1);
@@ -814,13 +816,13 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const tc::Desc dw = tc::split_desc(tc::make_desc(sb + W, 128, 2048));
             const tc::Desc ddl = tc::split_desc(tc::make_desc(sb + DL, 2048, 128));
             const tc::Desc dp = tc::split_desc(tc::make_desc(sb + P, 1024, 128));
-            // X1 = Q K^T (rows 64..127 of the A operand read the next 64 rows of the buffer; never used)
+            // X1 = Q K^T (M = 64: accumulator row r in TMEM lane (r % 16) + 32 (r / 16))
             auto issue_x1 = [&](int c) {
                 const uint32_t bo = (uint32_t)(c & 1) * BUF;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = bo + (kk >> 2) * 8192 + (kk & 3) * 32;
-                    tc::mma_bf16_off_w(tm + TM_X1, dq, off, dk, off, id_kk64, kk > 0);
+                    tc::mma_bf16_off_w(tm + TM_X1, dq, off, dk, off, id_x1, kk > 0);
                 }
                 tc::mma_commit_w(&bar[X1F]);
             };
@@ -855,22 +857,24 @@ __global__ void __launch_bounds__(NT_WS, 1)
                     tc::mma_bf16_off_w(tm + TM_O1 + 64 * b, ds, kk * 4096, dq, bo + (kk >> 2) * 8192 + (kk & 3) * 32,
                                      id_kk64, kk > 0);
                 // S <- gamma_C S + Delta^T (diag(e) K) (B: MN-major view of K)
-                if (!(ok = wait_bar_w(&bar[DLR], par, ctl, err) && wait_bar_w(&bar[PR], par, ctl, err))) break;
+                if (!(ok = wait_bar_w(&bar[DLR], par, ctl, err) && wait_bar_w(&bar[KR], par, ctl, err))) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk)
                     tc::mma_bf16_off_w(tm + TM_S, ddl, kk * 4096, dkm, bo + kk * 2048, id_km128, 1);
                 tc::mma_commit_w(&bar[M4S]);
                 tc::mma_commit_w(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
-                // the next chunk's W^T, U^T and X1
+                // the next chunk's W^T, U^T; its X1 once this chunk's X1 has been read out (PR)
                 if (c + 1 < nch) {
                     if (!(ok = wait_bar_w(&bar[FULL + (b ^ 1)], full_par(c + 1), ctl, err) &&
                                wait_bar_w(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
                         break;
                     tc::fence_after_sync();
                     issue_wu(c + 1);
-                    issue_x1(c + 1);
                 }
+                if (!(ok = wait_bar_w(&bar[PR], par, ctl, err))) break;
+                tc::fence_after_sync();
+                if (c + 1 < nch) issue_x1(c + 1);
                 // O2 = Delta^T P^T (after the output warps have read the previous O2)
                 if (c >= 1 && !(ok = wait_bar_w(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err))) break;
                 tc::fence_after_sync();
@@ -941,26 +945,27 @@ __global__ void __launch_bounds__(NT_WS, 1)
             tc::fence_after_sync();
             tile32_epilogue(sb + W, tl + TM_WT + 32 * half, k, 32 * half, -1.f);
             handoff(&bar[WR]);
-            // P_rs = exp(G_r - G_s) X1_rs for s <= r (rows r = TMEM lanes 0..63), then K <- diag(e) K
+            // K <- diag(e) K (X1 and W^T, U^T have read K), which the update waits for; then
+            // P_rs = exp(G_r - G_s) X1_rs for s <= r (X1 is M = 64: row r in TMEM lane (r % 16) + 32 (r / 16);
+            // warp quarter q holds rows 16 q .. 16 q + 15, each warp 32 of the 64 columns)
             if (!(ok = wait_bar(&bar[X1F], (uint32_t)(c & 1), ctl, err))) break;
             tc::fence_after_sync();
             const float *vec = vecp(c);
-            if ((warp & 3) < 2) {
-                const int r = k, s0 = 32 * half;
+            scale_rows_sw128(smem + b * BUF + B_K, vec + 128, t256, 256, raw ? vec + 192 : nullptr);
+            handoff(&bar[KR]);
+            {
+                const int l16 = lane & 15, r = 16 * (warp & 3) + l16, s0 = 32 * half + 16 * (lane >> 4);
                 const float Gr = vec[r];
-                float x[32];
-                tc::tmem_ld32(tl + TM_X1 + s0, x);
+                float x[16];
+                tc::tmem_ld16_split16(lane_base(tm, warp) + TM_X1 + 32 * half, x);
                 if (raw)
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] *= vec[192 + s0 + i];  // raw keys: 1 / ||k_s||
+                    for (int i = 0; i < 16; ++i) x[i] *= vec[192 + s0 + i];  // raw keys: 1 / ||k_s||
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - vec[s0 + i]) * x[i] : 0.f;
+                for (int i = 0; i < 16; ++i) x[i] = (s0 + i <= r) ? ex2(Gr - vec[s0 + i]) * x[i] : 0.f;
 #pragma unroll
-                for (int i = 0; i < 32; i += 8) st_run8(sb + P + b * 8192 + tc::tile_off(r, s0 + i, 128, 1024), x + i);
+                for (int i = 0; i < 16; i += 8) st_run8(sb + P + b * 8192 + tc::tile_off(r, s0 + i, 128, 1024), x + i);
             }
-            tc::fence_before_sync();
-            scale_rows_sw128(smem + b * BUF + B_K, vec + 128, t256, 256,
-                             raw ? vec + 192 : nullptr);  // X1 and W^T, U^T have read K
             handoff(&bar[PR]);
         }
     } else {
