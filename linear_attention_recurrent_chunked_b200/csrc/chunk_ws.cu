@@ -864,24 +864,25 @@ __global__ void __launch_bounds__(NT_WS, 1)
                     tc::mma_bf16_off_w(tm + TM_S, ddl, kk * 4096, dkm, bo + kk * 2048, id_km128, 1);
                 tc::mma_commit_w(&bar[M4S]);
                 tc::mma_commit_w(&bar[EMPTY + b]);  // last MMAs reading this buffer's K and Q
-                // the next chunk's W^T, U^T; its X1 once this chunk's X1 has been read out (PR)
+                // O2 = Delta^T P^T (after the output warps have read the previous O2) first: its inputs are
+                // ready by now, while the next chunk's T1 may still be in the making
+                if (!(ok = (c < 1 || wait_bar_w(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err)) &&
+                           wait_bar_w(&bar[PR], par, ctl, err)))
+                    break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    tc::mma_bf16_off_w(tm + TM_O2, ddl, kk * 4096, dp, b * 8192 + kk * 2048, id_kk64, kk > 0);
+                tc::mma_commit_w(&bar[M4O]);
+                // the next chunk's W^T, U^T, then its X1 (this chunk's X1 has been read out: PR above)
                 if (c + 1 < nch) {
                     if (!(ok = wait_bar_w(&bar[FULL + (b ^ 1)], full_par(c + 1), ctl, err) &&
                                wait_bar_w(&bar[T1R], (uint32_t)((c + 1) & 1), ctl, err)))
                         break;
                     tc::fence_after_sync();
                     issue_wu(c + 1);
+                    issue_x1(c + 1);
                 }
-                if (!(ok = wait_bar_w(&bar[PR], par, ctl, err))) break;
-                tc::fence_after_sync();
-                if (c + 1 < nch) issue_x1(c + 1);
-                // O2 = Delta^T P^T (after the output warps have read the previous O2)
-                if (c >= 1 && !(ok = wait_bar_w(&bar[OF], (uint32_t)((c - 1) & 1), ctl, err))) break;
-                tc::fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    tc::mma_bf16_off_w(tm + TM_O2, ddl, kk * 4096, dp, b * 8192 + kk * 2048, id_kk64, kk > 0);
-                tc::mma_commit_w(&bar[M4O]);
             }
         }
     } else if (warp < 8) {
