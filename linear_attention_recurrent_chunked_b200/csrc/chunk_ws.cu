@@ -1414,11 +1414,12 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                         for (int i = 0; i < 32; i += 4)
                             ps[((c0 + i) >> 2) * D + r] = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
                     }
-                    __threadfence();
                 }
                 // TM_S is read: the own step may accumulate onto S_loc
                 tc::fence_before_sync();
                 tc::mbar_arrive(&bar[PUBD]);
+                // the part's stores of all 256 X threads precede the barrier, and the release store of the
+                // flag after it is cumulative: a CTA that acquires the flag sees the whole part
                 tc::named_sync(1, 256);
                 if (tid == 256) tc::st_release_gpu(pflags + slot0 + (size_t)nfold * H, ok ? FLAG_DONE : FLAG_FAILED);
             } else if (ok) {
@@ -1529,7 +1530,6 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
             tc::tmem_ld32(tl + TM_S + c0, x);
             st_split32_global(dst, v, c0, x);
         }
-        __threadfence();
     }
     if (warp == W_MMA || warp == W_XMMA || warp == W_WMMA) {
         uint64_t *fin = &bar[warp == W_MMA ? FIN : warp == W_XMMA ? FINX : FINW];
@@ -1539,7 +1539,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
-    // (failure-injection test: segment 0 of head 0 withholds its end-state flag, so that the
+    // (the end state's stores precede the barrier and the flag's release store after it is cumulative.
+    // Failure-injection test: segment 0 of head 0 withholds its end-state flag, so that the
     // CTAs waiting for it give up after the injected bound; nothing else changes)
     if (tid == 0 && !(withhold && h == 0 && gseg == 0)) {
         const bool good = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
