@@ -701,7 +701,8 @@ enum {
     OF = 14,    // O1, O2 read out of TMEM (output, 128)
     FIN = 15,   // every MMA of the CTA done (drained before TMEM is freed)
     KR = 16,    // diag(e) K written (prep, 256)
-    NBAR = 17
+    LINKF = 17, // a later segment's start state (hi into the S tile, lo over DL and OST) landed
+    NBAR = 18
 };
 __device__ __forceinline__ constexpr uint32_t bar_count(int i) {
     return i == EMPTY || i == EMPTY + 1 ? 2u : (i >= T1R && i <= SR) || i == KR ? 256u : i == OF ? 128u : 1u;
@@ -787,6 +788,17 @@ __global__ void __launch_bounds__(NT_WS, 1)
             // (a failed or timed-out flag aborts the CTA; the record loads still complete the barriers)
             if (split) wait_flag(start_flag, ctl, err, flag_ns);
             else griddep_wait();
+            // a later segment's start state, published as a bf16 hi / lo tile pair: hi is the S operand
+            // tile as it stands, lo goes over the Delta^T and staging tiles (unused until the first
+            // chunk's products), and the state warps add the two into TMEM
+            const bool smem_link = split && sg.s > 0 && nch > 0;
+            if (smem_link) {
+                const uint8_t *lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
+                tc::fence_proxy_async_global();  // written with generic stores, read by the bulk copies
+                tc::mbar_arrive_expect_tx(&bar[LINKF], 65536u);
+                tc::bulk_load(sb + S, lk, 32768u, &bar[LINKF]);
+                tc::bulk_load(sb + DL, lk + 32768, 32768u, &bar[LINKF]);
+            }
             for (int c = 0; c < pre; ++c) load_record(c);
             int issued = pre;
             for (int c = pre; c < nch; ++c) {
@@ -796,6 +808,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 issued = c + 1;
             }
             for (int c = max(0, issued - 2); c < issued; ++c) drain_bar(&bar[FULL + (c & 1)], full_par(c));
+            if (smem_link) drain_bar(&bar[LINKF], 0);
         }
     } else if (warp == W_MMA) {
         // ---------------------------------------------------------------- MMA issuer
@@ -895,8 +908,36 @@ __global__ void __launch_bounds__(NT_WS, 1)
             ok = wait_bar(&bar[FULL], 0, ctl, err);
             if (ok) g0 = vecp(0)[64 + C - 1];
         }
-        if (ok && split && sg.s > 0) ok = __all_sync(0xffffffffu, wait_flag(start_flag, ctl, err, flag_ns));
-        if (ok) {
+        const bool smem_link = split && sg.s > 0 && nch > 0;
+        if (ok && smem_link) {
+            // the start state from shared memory (the loader's bulk copies): S tile = hi already
+            if ((ok = wait_bar(&bar[LINKF], 0, ctl, err))) {
+                const uint8_t *hi = smem + S, *lo = smem + DL;
+#pragma unroll 1
+                for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
+                    uint32_t u[32];
+#pragma unroll
+                    for (int h8 = 0; h8 < 32; h8 += 8) {
+                        const uint32_t off = tc::tile_off(v, c0 + h8, 128, 2048);
+                        const uint4 a = *reinterpret_cast<const uint4 *>(hi + off);
+                        const uint4 b = *reinterpret_cast<const uint4 *>(lo + off);
+                        const uint32_t *wh = reinterpret_cast<const uint32_t *>(&a);
+                        const uint32_t *wl = reinterpret_cast<const uint32_t *>(&b);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 p = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wh[j]));
+                            const float2 q = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wl[j]));
+                            u[h8 + 2 * j] = __float_as_uint(g0 * (p.x + q.x));
+                            u[h8 + 2 * j + 1] = __float_as_uint(g0 * (p.y + q.y));
+                        }
+                    }
+                    tc::tmem_st32(tl + TM_S + c0, u);
+                }
+                tc::tmem_st_wait();
+                handoff(&bar[SR]);
+            }
+        } else if (ok && split && sg.s > 0) ok = __all_sync(0xffffffffu, wait_flag(start_flag, ctl, err, flag_ns));
+        if (ok && !smem_link) {
             const uint8_t *lk = nullptr;
             const float *src = nullptr;
             if (sg.s > 0)
