@@ -786,20 +786,26 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const int pre = min(nch, 2);
             for (int c = 0; c < pre; ++c) load_inputs(c);
             // (a failed or timed-out flag aborts the CTA; the record loads still complete the barriers)
-            if (split) wait_flag(start_flag, ctl, err, flag_ns);
-            else griddep_wait();
-            // a later segment's start state, published as a bf16 hi / lo tile pair: hi is the S operand
+            // A later segment's start state, published as a bf16 hi / lo tile pair: hi is the S operand
             // tile as it stands, lo goes over the Delta^T and staging tiles (unused until the first
-            // chunk's products), and the state warps add the two into TMEM
+            // chunk's products), and the state warps add the two into TMEM. Its first records load as
+            // soon as the records flag is set, so that the first chunk's W^T, -W, X1 and P can be
+            // ready before its start state arrives.
             const bool smem_link = split && sg.s > 0 && nch > 0;
             if (smem_link) {
+                wait_flag(flags + (size_t)2 * gridDim.y * H, ctl, err, flag_ns);
+                for (int c = 0; c < pre; ++c) load_record(c);
+                wait_flag(start_flag, ctl, err, flag_ns);
                 const uint8_t *lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
                 tc::fence_proxy_async_global();  // written with generic stores, read by the bulk copies
                 tc::mbar_arrive_expect_tx(&bar[LINKF], 65536u);
                 tc::bulk_load(sb + S, lk, 32768u, &bar[LINKF]);
                 tc::bulk_load(sb + DL, lk + 32768, 32768u, &bar[LINKF]);
+            } else {
+                if (split) wait_flag(start_flag, ctl, err, flag_ns);
+                else griddep_wait();
+                for (int c = 0; c < pre; ++c) load_record(c);
             }
-            for (int c = 0; c < pre; ++c) load_record(c);
             int issued = pre;
             for (int c = pre; c < nch; ++c) {
                 if (!wait_bar(&bar[EMPTY + (c & 1)], full_par(c - 2), ctl, err)) break;
