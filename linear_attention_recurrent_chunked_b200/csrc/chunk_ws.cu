@@ -721,9 +721,10 @@ __global__ void __launch_bounds__(NT_WS, 1)
     // What this CTA waits for before reading what earlier passes wrote (the plan's error word and
     // offsets are complete before the preceding grid can launch this one):
     //  * with a transition pass before this one (flags given): a later segment of a split
-    //    sequence, the end-state flag of the segment before it (which also orders it after the
-    //    records); an unsplit sequence, or the first of two segments, the records flag the
-    //    transition CTAs set once the prep grid is complete; the first of three or more segments,
+    //    sequence, the records flag for its first records, then the end-state flag of the
+    //    segment before it for its start state; an unsplit sequence, or the first of two
+    //    segments, the records flag the transition CTAs set once the prep grid is complete;
+    //    the first of three or more segments,
     //    its own end-state flag (a short segment whose output is off the critical path: started
     //    early it would only compete with the transition CTAs that are on it). Not the whole
     //    transition grid, so output CTAs run beside transition CTAs that still run or fold;
