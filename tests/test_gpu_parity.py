@@ -316,6 +316,16 @@ def test_segmented_slow_decay_stress():
     check(o, S_T, o_ref, S_ref, "bf16", "segmented stress")
 
 
+def test_segmented_last_segment_one_partial_chunk():
+    """1034 tokens over 2 heads split 4 + 4 + 4 + 4 + 1 chunks: every later segment takes its start
+    state from the one before it (copied into shared memory), and the last one is a single
+    10-token chunk. Slow decay keeps each start state in the outputs."""
+    w = make_prefill("prefill_2k", seqlens=[1034], H=2, s0=True, stress=True, seed=62)
+    o, S_T = chunk(to_dev(w))
+    o_ref, S_ref = run_oracle(w)
+    check(o, S_T, o_ref, S_ref, "bf16", "last segment of one partial chunk")
+
+
 def test_long_sequence_many_segments_long_fold():
     """One long sequence on one head: ~24 segments, so the last segment folds ~22 published parts
     (tf32 products) onto the first segment's end state; slow decay keeps the early state alive."""
