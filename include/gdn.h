@@ -56,7 +56,8 @@ typedef enum {
     GDN_ERR_SEQLENS = 5,   /* cu_seqlens not 0 = c0 <= c1 <= ... <= cN = T_tot */
     GDN_ERR_WORKSPACE = 6, /* workspace missing or smaller than required */
     GDN_ERR_CUDA = 7,      /* a CUDA launch or runtime call failed */
-    GDN_ERR_TIMEOUT = 8    /* a bounded device-side wait gave up */
+    GDN_ERR_TIMEOUT = 8,   /* a bounded device-side wait gave up */
+    GDN_ERR_BOUNDS = 9     /* a device-side index check failed (library built with GDN_DEBUG_CHECKS) */
 } gdn_status;
 
 typedef enum { GDN_F32 = 0, GDN_BF16 = 1 } gdn_dtype;
@@ -180,9 +181,13 @@ gdn_status gdn_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
 
 /*
  * Synchronises `stream` and reads the device error word that the last
- * gdn_chunk_fwd on this workspace wrote: GDN_OK, GDN_ERR_SEQLENS or
+ * gdn_chunk_fwd on this workspace wrote: GDN_OK, GDN_ERR_SEQLENS,
  * GDN_ERR_TIMEOUT (a bounded inter-block wait gave up; outputs are then
- * incomplete). The word is reset by every gdn_chunk_fwd call. On a timeout
+ * incomplete) or, from a library built with GDN_DEBUG_CHECKS (the
+ * libgdn_b200_debug.so variant, whose kernels check their indices into the
+ * workspace and the outputs), GDN_ERR_BOUNDS (an index was out of range; the
+ * access went to index 0 of its region instead). The word is reset by every
+ * gdn_chunk_fwd call. On a timeout
  * of the pipelined path, gdn_last_error() names the first wait that gave up
  * (the mbarrier's shared-memory address and awaited parity, or the flag's
  * word offset in the workspace, with the block and thread), a diagnostic for

@@ -403,6 +403,13 @@ __device__ __forceinline__ void handoff(uint64_t *bar) {
 }
 
 // Index of the (chunk, head) record; the segment's first chunk is chunk_off[n] + s * seg_chunks.
+// Sizes of the workspace regions in their units, for the GDN_DEBUG_CHECKS index checks: records
+// ((chunk, head) pairs: the host's bound on the chunk count times H) and per-(segment, head) slots
+// (parts, links and flags: the transition and output grids' nslots = gridDim.y, times H).
+__device__ __forceinline__ size_t rec_capacity(int N, int T_tot, int H) {
+    return (size_t)(((long)T_tot + (long)(C - 1) * N) / C) * (size_t)H;
+}
+
 __device__ __forceinline__ size_t rec_index(const int32_t *chunk_off, const Segment &sg, int seg_chunks, int c, int H,
                                             int h) {
     return ((size_t)chunk_off[sg.n] + (size_t)sg.s * seg_chunks + c) * H + h;
@@ -660,7 +667,8 @@ __global__ void __launch_bounds__(256, pp::CTAS_PER_SM)
         if (tid == 0) {
             int h, cs, L, gc;
             locate(w, h, cs, L, gc);
-            tc::bulk_store(rec + ((size_t)gc * H + h) * REC_BYTES, sb + pp::REC, REC_BYTES);
+            const size_t ri = checked((size_t)gc * H + h, rec_capacity(N, T_tot, H), err);
+            tc::bulk_store(rec + ri * REC_BYTES, sb + pp::REC, REC_BYTES);
         }
     }
     cp_async_wait_all();
@@ -759,7 +767,8 @@ __global__ void __launch_bounds__(NT_WS, 1)
     tc::fence_after_sync();
     const uint32_t tm = ctl->tmem;
     const int nch = (sg.b - sg.a + C - 1) / C;
-    const size_t sidx = ((size_t)sg.n * H + h) * D * D;
+    const size_t sidx = checked(((size_t)sg.n * H + h) * D * D, (size_t)N * H * D * D, err);
+    const size_t rec_cap = rec_capacity(N, T_tot, H), slot_cap = (size_t)gridDim.y * H;
     const bool last_seg = sg.s == sg.ns - 1;
     const int quarter_lane = (warp & 3) * 32 + lane;  // this thread's TMEM lane
     auto buf = [&](int c) { return sb + (uint32_t)(c & 1) * BUF; };
@@ -781,7 +790,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 }
             };
             auto load_record = [&](int c) {
-                tc::bulk_load(buf(c) + B_T2, rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES,
+                tc::bulk_load(buf(c) + B_T2, rec + checked(rec_index(chunk_off, sg, seg_chunks, c, H, h), rec_cap, err) * REC_BYTES,
                               REC_BYTES, &bar[FULL + (c & 1)]);
             };
             const int pre = min(nch, 2);
@@ -797,7 +806,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 wait_flag(flags + (size_t)2 * gridDim.y * H, ctl, err, flag_ns);
                 for (int c = 0; c < pre; ++c) load_record(c);
                 wait_flag(start_flag, ctl, err, flag_ns);
-                const uint8_t *lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
+                const uint8_t *lk = link + checked(((size_t)seg_off[sg.n] + sg.s - 1) * H + h, slot_cap, err) * LINK_BYTES;
                 tc::fence_proxy_async_global();  // written with generic stores, read by the bulk copies
                 tc::mbar_arrive_expect_tx(&bar[LINKF], 65536u);
                 tc::bulk_load(sb + S, lk, 32768u, &bar[LINKF]);
@@ -948,7 +957,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
             const uint8_t *lk = nullptr;
             const float *src = nullptr;
             if (sg.s > 0)
-                lk = link + (((size_t)seg_off[sg.n] + sg.s - 1) * H + h) * LINK_BYTES;
+                lk = link + checked(((size_t)seg_off[sg.n] + sg.s - 1) * H + h, slot_cap, err) * LINK_BYTES;
             else if (S0)
                 src = S0 + sidx + (size_t)v * D;
             state_init64(sb + S, tl + TM_S, v, 64 * half, g0, src, lk, false);
@@ -1061,7 +1070,7 @@ __global__ void __launch_bounds__(NT_WS, 1)
                 for (int it = 0; it < 8; ++it) {
                     const int idx = it * 128 + v, r = idx >> 4, j = idx & 15;
                     if (r < L)
-                        *reinterpret_cast<uint4 *>(o + ((size_t)(cs + r) * H + h) * D + 8 * j) =
+                        *reinterpret_cast<uint4 *>(o + (checked((size_t)(cs + r), (size_t)T_tot, err) * H + h) * D + 8 * j) =
                             *reinterpret_cast<const uint4 *>(ost + r * 256 + j * 16);
                 }
             }
@@ -1199,7 +1208,8 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     tc::fence_after_sync();
     const uint32_t tm = ctl->tmem;
     const int nch = (sg.b - sg.a + C - 1) / C;
-    const size_t sidx = ((size_t)sg.n * H + h) * D * D;
+    const size_t sidx = checked(((size_t)sg.n * H + h) * D * D, (size_t)N * H * D * D, err);
+    const size_t rec_cap = rec_capacity(N, T_tot, H), slot_cap = (size_t)gridDim.y * H;
     const int quarter_lane = (warp & 3) * 32 + lane;
     auto kslot = [&](int c) { return KRING + (uint32_t)(c % 3) * KSLOT; };
     auto vslot = [&](int c) { return VRING + (uint32_t)(c & 1) * VSLOT; };
@@ -1209,7 +1219,9 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
 
     if (warp == W_LOAD) {
         if (lane == 0) {
-            auto rp = [&](int c) { return rec + rec_index(chunk_off, sg, seg_chunks, c, H, h) * REC_BYTES; };
+            auto rp = [&](int c) {
+                return rec + checked(rec_index(chunk_off, sg, seg_chunks, c, H, h), rec_cap, err) * REC_BYTES;
+            };
             auto load_k = [&](int c) {
                 uint64_t *fk = &bar[FULLK + c % 3];
                 tc::mbar_arrive_expect_tx(fk, 16384u + 1024u);
@@ -1427,7 +1439,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
     bool ok = !*reinterpret_cast<volatile uint32_t *>(&ctl->abort) && nch > 0;
     const int nfold = sg.s;                              // fold steps; the last is this segment's own
     const size_t slot0 = (size_t)(gseg - sg.s) * H + h;  // the sequence's first segment
-    auto part_of = [&](int j) { return part + (slot0 + (size_t)j * H) * PART_BYTES; };
+    auto part_of = [&](int j) { return part + checked(slot0 + (size_t)j * H, slot_cap, err) * PART_BYTES; };
     // TMEM buffers of the fold's intermediate end states F(j), j = 0 .. nfold - 1 (F(0) the first
     // segment's end state; F(j), j >= 1, holds S_loc(j) before step j accumulates onto it): columns 256
     // and 384 in turn. (A third buffer over the X state's columns 128 .. 255 gave wrong end states
@@ -1474,7 +1486,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
                 // S warps: F(0) = the first segment's published end state, hi + lo in fp32
                 const int half = (warp >> 2) & 1;
                 if ((ok = __all_sync(0xffffffffu, wait_flag(flags + slot0, ctl, err, flag_ns)))) {
-                    const uint8_t *src = link + slot0 * LINK_BYTES;
+                    const uint8_t *src = link + checked(slot0, slot_cap, err) * LINK_BYTES;
 #pragma unroll 1
                     for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 16) {
                         float u[16];
@@ -1571,7 +1583,7 @@ __global__ void __launch_bounds__(NT_TRANS, 1)
         tc::fence_after_sync();
         const int v = quarter_lane, half = (warp >> 2) & 1;
         const uint32_t tl = lane_base(tm, warp);
-        uint8_t *dst = link + ((size_t)gseg * H + h) * LINK_BYTES;
+        uint8_t *dst = link + checked((size_t)gseg * H + h, slot_cap, err) * LINK_BYTES;
 #pragma unroll 1
         for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
             float x[32];

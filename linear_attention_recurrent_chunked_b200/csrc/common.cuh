@@ -10,7 +10,27 @@
 namespace gdn {
 
 // Device error word layout (first 4 bytes of the chunk workspace).
-enum : uint32_t { ERRBIT_SEQLENS = 1u, ERRBIT_TIMEOUT = 2u, ERRBIT_INTERNAL = 4u };
+enum : uint32_t { ERRBIT_SEQLENS = 1u, ERRBIT_TIMEOUT = 2u, ERRBIT_INTERNAL = 4u, ERRBIT_BOUNDS = 8u };
+
+// Index checks of the GDN_DEBUG_CHECKS build: an index into a workspace region or an output,
+// checked against the region's size. Out of range, the error word gets ERRBIT_BOUNDS and the
+// access goes to index 0 instead (in range), so that the kernel finishes without touching memory
+// outside the region and the host reads the error. In the normal build the index passes unchanged
+// and no code is generated.
+#ifdef GDN_DEBUG_CHECKS
+__device__ __noinline__ inline void debug_out_of_bounds(uint32_t *err) { atomicOr(err, ERRBIT_BOUNDS); }
+template <typename I>
+__device__ __forceinline__ I checked(I idx, I lim, uint32_t *err) {
+    if (idx < lim) return idx;
+    debug_out_of_bounds(err);
+    return I(0);
+}
+#else
+template <typename I>
+__device__ __forceinline__ I checked(I idx, I, uint32_t *) {
+    return idx;
+}
+#endif
 
 template <typename T> struct Elem;
 template <> struct Elem<float> {

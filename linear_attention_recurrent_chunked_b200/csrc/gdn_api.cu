@@ -12,6 +12,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -127,7 +129,11 @@ struct ProfHandle {
     cudaEvent_t start;
 };
 
+// Every launch site brackets its kernel with these: an NVTX range named after the kernel (seen by
+// Nsight tools when one is attached; a few nanoseconds otherwise) and, while profiling is enabled,
+// a pair of CUDA events on the launch stream.
 void *prof_start(const char *name, cudaStream_t st) {
+    nvtxRangePushA(name);
     std::lock_guard<std::mutex> lk(g_prof.mu);
     if (!g_prof.on) return nullptr;
     ProfHandle *hd = new ProfHandle{name, st, prof_event()};
@@ -136,6 +142,7 @@ void *prof_start(const char *name, cudaStream_t st) {
 }
 
 void prof_stop(void *handle) {
+    nvtxRangePop();
     if (!handle) return;
     ProfHandle *hd = static_cast<ProfHandle *>(handle);
     std::lock_guard<std::mutex> lk(g_prof.mu);
@@ -278,6 +285,9 @@ gdn_status gdn_chunk_fwd_check(const void *workspace, size_t ws_bytes, void *str
         return fail(GDN_ERR_TIMEOUT, "a bounded device-side wait gave up");
     }
     if (word & gdn::ERRBIT_INTERNAL) return fail(GDN_ERR_CUDA, "internal: misaligned shared-memory base, nothing written");
+    if (word & gdn::ERRBIT_BOUNDS)
+        return fail(GDN_ERR_BOUNDS, "a device-side index check failed (GDN_DEBUG_CHECKS build): an index into the "
+                                    "workspace or an output was out of range and was redirected to 0");
     return ok();
 }
 

@@ -14,13 +14,16 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
+# GDN_DEBUG_CHECKS=1 in the environment selects the index-checking build (see build.py --debug)
+_LIB_PATH = os.path.join(_HERE, "libgdn_b200_debug.so" if os.environ.get("GDN_DEBUG_CHECKS") == "1"
+                         else "libgdn_b200.so")
 _lib = None
 
 GDN_F32, GDN_BF16 = 0, 1
 _DTYPE = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 STATUS = {0: "GDN_OK", 1: "GDN_ERR_NULL", 2: "GDN_ERR_SHAPE", 3: "GDN_ERR_DTYPE", 4: "GDN_ERR_ALIGN",
-          5: "GDN_ERR_SEQLENS", 6: "GDN_ERR_WORKSPACE", 7: "GDN_ERR_CUDA", 8: "GDN_ERR_TIMEOUT"}
+          5: "GDN_ERR_SEQLENS", 6: "GDN_ERR_WORKSPACE", 7: "GDN_ERR_CUDA", 8: "GDN_ERR_TIMEOUT",
+          9: "GDN_ERR_BOUNDS"}
 
 # Every symbol include/gdn.h declares, with its ctypes signature.
 _VP, _SZ, _I = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int

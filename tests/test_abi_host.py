@@ -42,6 +42,22 @@ def test_every_declared_symbol_is_exported(lib):
         assert getattr(lib, name) is not None
 
 
+def test_debug_checks_variant_builds_and_exports_the_same_symbols():
+    """The GDN_DEBUG_CHECKS build (kernels that check their indices into the workspace and the
+    outputs, a failed check reported as GDN_ERR_BOUNDS) links, loads and exports the same C ABI."""
+    from linear_attention_recurrent_chunked_b200 import build
+    path = build.build(debug=True)
+    assert os.path.basename(path) == "libgdn_b200_debug.so"
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (gdn_[a-z0-9_]+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+    dbg = ctypes.CDLL(path)
+    assert dbg.gdn_version() == ctypes.CDLL(build.LIB).gdn_version()
+    # the status the check entry point returns for a failed index check is declared
+    assert re.search(r"GDN_ERR_BOUNDS\s*=\s*9", open(HEADER).read())
+
+
 def test_header_compiles_as_c_and_cpp(tmp_path):
     src = tmp_path / "t.c"
     src.write_text('#include "gdn.h"\nint main(void){return gdn_version()==0;}\n')
